@@ -1,0 +1,343 @@
+"""AutoRound layer tuning, written out plainly (oracle side).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring for the sources and the
+readings of the pages that this file follows).
+
+Notation: W is [out, in]; a group is ``g`` consecutive columns of one row
+(g = in when group_size is -1); Q = 2^bits - 1.  fp32 arrays hold the quantiser
+state; every expression on fp32 arrays below is evaluated by numpy one IEEE
+fp32 operation at a time.  Contractions and derivatives are fp64.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+from .schedule import block_schedule
+
+F32 = np.float32
+F64 = np.float64
+
+
+def qmax(bits: int) -> np.float32:
+    """Largest code, 2^bits - 1 ("[SGLang] AutoRound ...", 1. AutoRoundConfig: bits 2/3/4/8)."""
+    if bits not in (2, 3, 4, 8):
+        raise ValueError("bits must be one of 2, 3, 4, 8")
+    return F32(2 ** bits - 1)
+
+
+def _group(inn: int, group_size: int) -> int:
+    g = inn if group_size == -1 else group_size
+    if g <= 0 or inn % g:
+        raise ValueError("group_size must be -1 or a positive divisor of in")
+    return g
+
+
+def _to_f32(a: np.ndarray) -> np.ndarray:
+    """Accept fp32/fp64 values or uint16 bf16 bit patterns; return fp32."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32)
+    return a.astype(F32)
+
+
+def _rows_f64(X: np.ndarray, r0: int, r1: int) -> np.ndarray:
+    blk = X[r0:r1]
+    if blk.dtype == np.uint16:
+        return (blk.astype(np.uint32) << 16).view(np.float32).astype(F64)
+    return blk.astype(F64)
+
+
+def _expand(a: np.ndarray, g: int) -> np.ndarray:
+    """Per-group [out, G] values broadcast to the elements [out, G*g]."""
+    return np.repeat(a, g, axis=1)
+
+
+# --------------------------------------------------------------------------
+# forward: min-max init, scale / zero-point, offset fake-quant
+# --------------------------------------------------------------------------
+
+def group_minmax(W: np.ndarray, group_size: int):
+    """Min-max statistics per group, widened to include 0.
+
+    "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END":
+    ``_init_scale_zp`` is min-max.  Reading: wmin = min(0, min W_grp),
+    wmax = max(0, max W_grp), so 0 is always representable; taken from the
+    original W and never updated.
+    """
+    W = _to_f32(W)
+    out, inn = W.shape
+    g = _group(inn, group_size)
+    Wg = W.reshape(out, inn // g, g)
+    wmin = np.minimum(Wg.min(axis=2), F32(0))
+    wmax = np.maximum(Wg.max(axis=2), F32(0))
+    return wmin, wmax
+
+
+def scale_zero_point(wmin, wmax, alpha, beta, bits: int, sym: bool):
+    """Scale and zero-point from the clip factors.
+
+    Asymmetric: s = (alpha*wmax - beta*wmin) / Q and zp = clamp(rint(-beta*wmin / s), 0, Q),
+    the clipped min-max range whose bounds are learned jointly with the rounding
+    ("Introducing AutoRound ...", section 2).  An all-zero group gets s = 1.
+    Symmetric (reading): amax = max(-wmin, wmax), s = 2*alpha*amax / Q,
+    zp = 2^(bits-1); beta is unused.
+    """
+    Q = qmax(bits)
+    wmin = _to_f32(wmin)
+    wmax = _to_f32(wmax)
+    alpha = _to_f32(alpha)
+    beta = _to_f32(beta)
+    if sym:
+        amax = np.maximum(-wmin, wmax)
+        s = (F32(2) * (alpha * amax)) / Q
+        s = np.where(s == 0, F32(1), s).astype(F32)
+        zp = np.full(s.shape, F32(2 ** (bits - 1)), dtype=F32)
+    else:
+        s = (alpha * wmax - beta * wmin) / Q
+        s = np.where(s == 0, F32(1), s).astype(F32)
+        zp = np.clip(np.rint(-(beta * wmin) / s), F32(0), Q).astype(F32)
+    return s, zp
+
+
+@dataclasses.dataclass
+class FakeQuant:
+    u: np.ndarray      # W / s
+    t: np.ndarray      # u + V
+    r: np.ndarray      # rint(t), ties to even
+    p: np.ndarray      # r + zp
+    q: np.ndarray      # clamp(p, 0, Q): the integer code
+    m: np.ndarray      # 0 <= p <= Q (bool): the clamp's pass-through mask
+    Wq: np.ndarray     # s * (q - zp)
+
+
+def fake_quant(W, V, s, zp, group_size: int, bits: int) -> FakeQuant:
+    """Offset rounding of every element.
+
+    "[llm-compressor] AutoRound ...", section "논문 핵심 내용": w^ = s*round(w/s + V);
+    ``_fake_quantize_with_offset``: q = clamp(round(W/s + zp + V), qmin, qmax),
+    W' = s*(q - zp).  The rounding argument is formed as rint(W/s + V) + zp
+    (equal in exact arithmetic; this fp32 order is the contract); round is
+    torch.round, i.e. half to even.
+    """
+    W = _to_f32(W)
+    V = _to_f32(V)
+    g = _group(W.shape[1], group_size)
+    Q = qmax(bits)
+    se = _expand(_to_f32(s), g)
+    ze = _expand(_to_f32(zp), g)
+    u = W / se
+    t = u + V
+    r = np.rint(t)
+    p = r + ze
+    q = np.clip(p, F32(0), Q)
+    m = (p >= 0) & (p <= Q)
+    Wq = se * (q - ze)
+    return FakeQuant(u, t, r, p, q, m, Wq)
+
+
+def rtn(W, bits: int, group_size: int, sym: bool):
+    """Round-to-nearest: V = 0, alpha = beta = 1 ("논문 핵심 내용": w^ = s*round(w/s)).
+
+    Returns (codes uint8 [out, in], scale fp32 [out, G], zero-point int32 [out, G], W' fp32).
+    """
+    W = _to_f32(W)
+    wmin, wmax = group_minmax(W, group_size)
+    one = np.ones_like(wmin)
+    s, zp = scale_zero_point(wmin, wmax, one, one, bits, sym)
+    fq = fake_quant(W, np.zeros_like(W), s, zp, group_size, bits)
+    return fq.q.astype(np.uint8), s, zp.astype(np.int32), fq.Wq
+
+
+# --------------------------------------------------------------------------
+# backward: straight-through derivatives of W' with respect to V, alpha, beta
+# --------------------------------------------------------------------------
+
+def step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size: int, bits: int, sym: bool):
+    """Gradients of the loss at (V, alpha, beta), given G = dL/dW' up to a positive factor.
+
+    The page's loop back-propagates through ``torch.round``; reading: a
+    straight-through estimator -- every rint (the code's and the zero-point's)
+    passes the gradient as the identity, and every clamp passes it only where its
+    input lies inside the closed interval (torch.clamp's rule).
+
+    Returns (sgn_dV fp32 [out, in] in {-1, 0, 1}, dalpha fp64 [out, G], dbeta fp64 [out, G]).
+    With ds_a = ds/dalpha, ds_b = ds/dbeta:
+      in range (m = 1):  W' = s*r, so dW'/dtheta = ds_theta * (r - W/s)  (zp cancels);
+      clamped  (m = 0):  W' = s*(q - zp), so dW'/dtheta = ds_theta*(q - zp) - s*dzp/dtheta,
+                         zp following z0 = -beta*wmin/s unless zp itself was clamped;
+      dL/dV = G * s * m, and s > 0, so sign(dL/dV) = sign(G) * m.
+    """
+    W = _to_f32(W)
+    out, inn = W.shape
+    g = _group(inn, group_size)
+    Q = qmax(bits)
+    s, zp = scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
+    fq = fake_quant(W, V, s, zp, group_size, bits)
+
+    Qd = float(Q)
+    wmin64 = _to_f32(wmin).astype(F64)
+    wmax64 = _to_f32(wmax).astype(F64)
+    s64 = s.astype(F64)
+    if sym:
+        amax64 = np.maximum(-wmin64, wmax64)
+        ds_a = 2.0 * amax64 / Qd
+        ds_b = np.zeros_like(ds_a)
+        dzp_a = np.zeros_like(ds_a)
+        dzp_b = np.zeros_like(ds_a)
+    else:
+        ds_a = wmax64 / Qd
+        ds_b = -wmin64 / Qd
+        z0 = -_to_f32(beta).astype(F64) * wmin64 / s64
+        rz = np.rint(-(_to_f32(beta) * _to_f32(wmin)) / s)   # the forward's pre-clamp zp
+        zfree = ((rz >= 0) & (rz <= Q)).astype(F64)
+        dzp_a = (-z0 * ds_a / s64) * zfree
+        dzp_b = (-wmin64 / s64 - z0 * ds_b / s64) * zfree
+
+    W64 = W.astype(F64)
+    se = _expand(s64, g)
+    ratio = W64 / se
+    r = fq.r.astype(F64)
+    qz = fq.q.astype(F64) - _expand(zp.astype(F64), g)
+    m = fq.m
+    dWa = np.where(m, _expand(ds_a, g) * (r - ratio), _expand(ds_a, g) * qz - se * _expand(dzp_a, g))
+    dWb = np.where(m, _expand(ds_b, g) * (r - ratio), _expand(ds_b, g) * qz - se * _expand(dzp_b, g))
+    G = np.asarray(G, dtype=F64)
+    dalpha = (G * dWa).reshape(out, inn // g, g).sum(axis=2)
+    dbeta = (G * dWb).reshape(out, inn // g, g).sum(axis=2)
+    if sym:
+        dbeta = np.zeros_like(dbeta)
+    sgn_dV = (np.sign(G) * m).astype(F32)
+    return sgn_dV, dalpha, dbeta
+
+
+# --------------------------------------------------------------------------
+# the tuning loop
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class TuneResult:
+    codes: np.ndarray        # uint8 [out, in]: codes of the applied iterate
+    scale: np.ndarray        # fp32 [out, G]
+    zero_point: np.ndarray   # int32 [out, G]
+    Wq: np.ndarray           # fp32 [out, in], the applied fake-quantised weight
+    V: np.ndarray            # fp32 [out, in]: live state after the last update
+    alpha: np.ndarray        # fp32 [out, G]
+    beta: np.ndarray         # fp32 [out, G]
+    loss_trace: np.ndarray   # fp64 [iters]: batch MSE at each step, before its update
+    final_mse: float | None  # MSE over all calibration rows with the applied W'
+    best_loss: np.ndarray    # fp64 [out]: per output row, lowest batch loss seen (inf if none)
+    V_best: np.ndarray       # per row, the state at that row's best step (initial if none)
+    alpha_best: np.ndarray
+    beta_best: np.ndarray
+
+
+def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
+               minmax_lr: float, batch_rows: int, seed: int, minmax_shrink: float = 1.0,
+               keep_best: bool = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
+               best0=None, want_final_mse: bool = True) -> TuneResult:
+    """SignSGD tuning of one linear layer.
+
+    "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END": per step,
+    fake-quantise W, run the layer on a calibration batch, take the MSE against
+    the full-precision output, back-propagate, then V <- clamp(V - lr*sign(dV), -0.5, 0.5)
+    ("논문 핵심 내용": V <- V - eta*sign(grad_V L)).  The clip factors follow the
+    same rule with minmax_lr (None -> lr, here minmax_lr < 0), clamped to [0.5, 1].
+    All variables are updated together from gradients taken at the same point.
+    One calibration block of ``batch_rows`` rows is used per step (see
+    ``schedule.block_schedule``).  The bias cancels in Y' - Y and is not an input.
+
+    Which iterate is applied at the end: the page's loop computes the step loss
+    (``total_loss``) and then applies the final V.  With a constant lr the sign
+    steps keep oscillating across rounding boundaries, and the final iterate can
+    be worse than RTN.  Reading used by default (keep_best): the state with the
+    lowest step loss is applied.  The loss is a sum over output rows, and a
+    row's V, alpha and beta only enter its own term, so the choice is made per
+    output row: row j keeps its state from the step where its batch loss
+    mean_b (Y' - Y)_bj^2 was lowest.  This keeps every row's tuning independent
+    of the others, and is never worse than one layer-wide choice.  Step 0, the
+    min-max RTN state, is a candidate, so with one full batch the result is never
+    worse than RTN.  keep_best=False applies the last state, as the page's
+    listing does.  The comparison is strict (a tie keeps the earlier state).
+
+    W: [out, in] fp32 values (or bf16 bit patterns); X: [n, in] bf16-exact values.
+    ``start_step`` continues the block schedule of an interrupted run, with the
+    live state passed in V0 / alpha0 / beta0 and the best state in
+    best0 = (best_loss, V_best, alpha_best, beta_best).
+    """
+    W = _to_f32(W)
+    out, inn = W.shape
+    n = X.shape[0]
+    if X.shape[1] != inn:
+        raise ValueError("X must be [n, in]")
+    if batch_rows <= 0 or n % batch_rows:
+        raise ValueError("n_rows must be a multiple of batch_rows")
+    if iters < 0 or lr < 0:
+        raise ValueError("iters and lr must be >= 0")
+    g = _group(inn, group_size)
+    lr32 = F32(lr)
+    mlr32 = F32(lr if minmax_lr < 0 else minmax_lr)
+
+    wmin, wmax = group_minmax(W, g)
+    V = np.zeros_like(W) if V0 is None else _to_f32(V0).copy()
+    alpha = np.full(wmin.shape, F32(minmax_shrink)) if alpha0 is None else _to_f32(alpha0).copy()
+    beta = np.full(wmin.shape, F32(minmax_shrink)) if beta0 is None else _to_f32(beta0).copy()
+    if best0 is None:
+        best_loss = np.full(out, np.inf)
+        V_best, a_best, b_best = V.copy(), alpha.copy(), beta.copy()
+    else:
+        best_loss = np.asarray(best0[0], dtype=F64).copy()
+        V_best, a_best, b_best = (_to_f32(x).copy() for x in best0[1:])
+
+    sched = block_schedule(n // batch_rows, start_step + iters, seed)[start_step:]
+    W64 = W.astype(F64)
+    cache: dict[int, np.ndarray] = {}
+    trace = np.zeros(iters, dtype=F64)
+    for t in range(iters):
+        blk = sched[t]
+        if blk not in cache:
+            cache[blk] = _rows_f64(X, blk * batch_rows, (blk + 1) * batch_rows)
+        Xb = cache[blk]
+        s, zp = scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
+        Wq = fake_quant(W, V, s, zp, g, bits).Wq
+        R = Xb @ (Wq.astype(F64) - W64).T          # Y' - Y  [B, out]
+        row_loss = np.sum(R * R, axis=0) / batch_rows
+        trace[t] = float(np.sum(row_loss)) / out
+        better = row_loss < best_loss
+        best_loss = np.where(better, row_loss, best_loss)
+        V_best[better] = V[better]
+        a_best[better] = alpha[better]
+        b_best[better] = beta[better]
+        G = R.T @ Xb                                # dL/dW' * (B*out/2)  [out, in]
+        sgn_dV, dalpha, dbeta = step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym)
+        V = np.clip(V - lr32 * sgn_dV, F32(-0.5), F32(0.5)).astype(F32)
+        alpha = np.clip(alpha - mlr32 * np.sign(dalpha).astype(F32), F32(0.5), F32(1.0)).astype(F32)
+        if not sym:
+            beta = np.clip(beta - mlr32 * np.sign(dbeta).astype(F32), F32(0.5), F32(1.0)).astype(F32)
+
+    Va, aa, ba = (V_best, a_best, b_best) if keep_best else (V, alpha, beta)
+    s, zp = scale_zero_point(wmin, wmax, aa, ba, bits, sym)
+    fq = fake_quant(W, Va, s, zp, g, bits)
+    mse = None
+    if want_final_mse:
+        D = fq.Wq.astype(F64) - W64
+        acc = 0.0
+        for r0 in range(0, n, batch_rows):
+            Xb = cache.get(r0 // batch_rows)
+            if Xb is None:
+                Xb = _rows_f64(X, r0, r0 + batch_rows)
+            R = Xb @ D.T
+            acc += float(np.sum(R * R))
+        mse = acc / (n * out)
+    return TuneResult(fq.q.astype(np.uint8), s, zp.astype(np.int32), fq.Wq, V, alpha, beta,
+                      trace, mse, best_loss, V_best, a_best, b_best)
+
+
+def layer_mse(W, Wq, X) -> float:
+    """Mean over rows and outputs of (X W'^T - X W^T)^2, from the two outputs directly
+    (the page's ``(y_hat - y_true).pow(2).mean()``), in fp64."""
+    X64 = _rows_f64(X, 0, X.shape[0])
+    Y = X64 @ _to_f32(W).astype(F64).T
+    Yq = X64 @ _to_f32(Wq).astype(F64).T
+    return float(np.mean((Yq - Y) ** 2))
