@@ -1,0 +1,349 @@
+"""Benchmark of the AutoRound layer-tuning hot path on B200.
+
+One benchmark step = one complete ``ar_tune_layer`` call on the LLaMA-7B-shaped
+q_proj workload (W 4096x4096 bf16 ~N(0, 0.02), asymmetric W4 g128, 262144 x 4096
+bf16 calibration activations with lognormal channel scales and 1% x20 outliers,
+16384 rows per SignSGD step, 200 steps, lr = minmax_lr = 0.005), followed by
+``ar_pack`` of its codes.  Every row of the hot path runs inside it: min-max
+init, the fake-quant prologue, both tensor-core contractions with their fused
+epilogues per step, the final codes and the final MSE pass, and packing.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload q_proj|tiny|down_7b|down_72b]
+
+Prints one JSON line (rank 0).  Metric: SignSGD steps per second (whole job:
+every rank tunes its own 4096-row shard of a layer, no collective on the data
+path, so the scaling is weak), plus the layer tune time and the fraction of
+the bf16 tensor-core peak.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import DOWN_7B, DOWN_72B, Q_PROJ_7B, TINY, make_activations, make_activations_cuda, make_weight  # noqa: E402
+
+WORKLOADS = {"q_proj": Q_PROJ_7B, "tiny": TINY, "down_7b": DOWN_7B, "down_72b": DOWN_72B}
+METRIC = "signsgd_steps_per_sec"
+UNIT = "steps/s"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import signed_gradient_rounding_b200 as ar
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    c = WORKLOADS[args.workload]
+    # Each rank tunes its own shard of output rows (weak scaling): rank r's rows
+    # are drawn with seed r; the calibration activations are the same on every rank.
+    W = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=rank))
+    Wd = (W.to(torch.bfloat16) if c.w_dtype == "bf16" else W).to(dev)
+    Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0)
+    ws = torch.empty(ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
+    G = c.inn // c.group_size
+    outs = (torch.empty((c.out, c.inn), dtype=torch.uint8, device=dev),
+            torch.empty((c.out, G), dtype=torch.float32, device=dev),
+            torch.empty((c.out, G), dtype=torch.int32, device=dev),
+            torch.empty((c.iters,), dtype=torch.float32, device=dev),
+            torch.empty((1,), dtype=torch.float64, device=dev))
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(timing=None):
+        res = ar.tune_layer(Wd, Xd, p, workspace=ws, outputs=outs, timing=timing)
+        packed = ar.pack(res.codes, c.bits)
+        return res, packed
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if ar.tune_status(ws) != ar.AR_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    timings = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            t = ar.TuneTiming()
+            one_step(t)
+            timings.append(t)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if ar.tune_status(ws) != ar.AR_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    mse = float(outs[4].item())
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # End to end through the host API: pinned host inputs copied in and the
+    # results copied out inside the timed region, every step.
+    e2e = None
+    if args.e2e_steps > 0:
+        Wh = W.to(torch.bfloat16 if c.w_dtype == "bf16" else torch.float32).pin_memory()
+        Xh = Xd.cpu().pin_memory()
+        h2d = Wh.numel() * Wh.element_size() + Xh.numel() * Xh.element_size()
+        d2h = c.out * c.inn + 2 * c.out * G * 4 + c.iters * 4 + 8
+        del Xd
+        torch.cuda.empty_cache()
+        ar.tune_layer_host(Wh, Xh, p, device=dev)          # warm
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            ar.tune_layer_host(Wh, Xh, p, device=dev)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * c.iters * args.e2e_steps / (float(ems.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks = _peaks()
+    flops_gemm = 2.0 * c.batch_rows * c.out * c.inn             # one contraction, one launch
+    res_ms = sum(t.residual_ms for t in timings) / sum(t.gemm_launches for t in timings)
+    upd_ms = sum(t.update_ms for t in timings) / sum(t.gemm_launches for t in timings)
+    dom_name, dom_ms = ("update", upd_ms) if upd_ms >= res_ms else ("residual", res_ms)
+    achieved = flops_gemm / (dom_ms * 1e-3) / 1e12
+    layer_s = ms_max / args.steps / 1e3
+    step_tflops = c.flops_per_step * c.iters / layer_s / 1e12
+    launches = sum(t.kernel_launches for t in timings) + args.steps    # + one pack per step
+    line = {
+        "metric": METRIC,
+        "value": world * c.iters * args.steps / (ms_max / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": c.name, "out": c.out, "in": c.inn, "n_rows": c.n_rows,
+                   "batch_rows": c.batch_rows, "iters": c.iters, "bits": c.bits, "group_size": c.group_size,
+                   "sym": c.sym, "lr": c.lr, "minmax_lr": c.minmax_lr, "keep_best": True,
+                   "bench_step": "one ar_tune_layer call (all iters) + ar_pack",
+                   "l2": "inputs larger than L2: X is %.1f GB, one step reads a %.0f MB block"
+                         % (c.n_rows * c.inn * 2 / 1e9, c.batch_rows * c.inn * 2 / 1e6),
+                   "parallelism": f"row shards x{world}, no data-path collective"},
+        "layer_tune_s": layer_s,
+        "fused_step_tflops": step_tflops,
+        "tensor_peak_frac": step_tflops / peaks["bf16_tflops_sustained"],
+        "final_mse": mse,
+        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel<{dom_name}>", "achieved": achieved,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "peak_source": peaks["source"] + " sustained bf16",
+                     "per_launch_ms": {"residual": res_ms, "update": upd_ms}},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(c, Xd if args.e2e_steps == 0 else None, args.cpu_rows, args.cpu_steps)
+    return line
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def _host_x(c, Xd=None):
+    """The workload's activations on the host as bf16 bit patterns (same bytes as the GPU run)."""
+    try:
+        import torch
+        if Xd is None and torch.cuda.is_available():
+            Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0)
+        if Xd is not None:
+            return Xd.view(torch.int16).cpu().numpy().view(np.uint16)
+    except ImportError:
+        pass
+    from workloads import bf16_bits
+    return bf16_bits(make_activations(c.n_rows, c.inn, c.x_kind, seed=0))
+
+
+def cpu_baseline(c, Xd, rows: int, steps: int):
+    """The oracle, as it stands, on `rows` sampled output rows for `steps` SignSGD
+    steps of the same workload; rows tune independently and every row-step costs
+    the same, so the rate scales to the full layer by rows / out."""
+    import oracle
+    X = _host_x(c, Xd)
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    sel = np.sort(np.random.default_rng(0).choice(c.out, min(rows, c.out), replace=False))
+    t0 = time.perf_counter()
+    oracle.tune_layer(W[sel], X, c.bits, c.group_size, c.sym, steps, c.lr, c.minmax_lr, c.batch_rows, 0,
+                      want_final_mse=False)
+    dt = time.perf_counter() - t0
+    return {"value": steps * (len(sel) / c.out) / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{len(sel)} of {c.out} output rows x {steps} steps on the full activations, "
+                      f"{dt:.1f} s; rate scaled by rows/out (rows tune independently)",
+            "host_cpu": os.cpu_count()}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return None
+    c = WORKLOADS[args.workload]
+    import oracle
+    X = _host_x(c)
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    sel = np.sort(np.random.default_rng(0).choice(c.out, min(args.cpu_rows, c.out), replace=False))
+
+    def one_step():
+        oracle.tune_layer(W[sel], X, c.bits, c.group_size, c.sym, args.cpu_steps, c.lr, c.minmax_lr,
+                          c.batch_rows, 0, want_final_mse=False)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = time.perf_counter() - t0
+    value = args.steps * args.cpu_steps * (len(sel) / c.out) / dt
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": c.name, "out": c.out, "in": c.inn, "n_rows": c.n_rows,
+                       "batch_rows": c.batch_rows, "iters": c.iters, "bits": c.bits,
+                       "group_size": c.group_size, "sym": c.sym},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                             "sample": f"each step: {len(sel)} of {c.out} output rows x {args.cpu_steps} "
+                                       f"SignSGD steps; rate scaled by rows/out"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q_proj")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

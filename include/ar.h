@@ -1,0 +1,214 @@
+/*
+ * ar.h -- C ABI of libar, AutoRound per-layer SignSGD tuning on one B200.
+ *
+ * The method (sources cited by page title and section):
+ *   "[llm-compressor] AutoRound: 부호 경사 하강법으로 라운딩 최적화"
+ *     - "논문 핵심 내용": RTN w^ = s*round(w/s); offset rounding w^ = s*round(w/s + V)
+ *       with V in [-0.5, 0.5]; loss |W^x - Wx|^2; SignSGD V <- V - lr*sign(dL/dV).
+ *     - "on_event with SEQUENTIAL_EPOCH_END": the per-layer loop and
+ *       _fake_quantize_with_offset, q = clamp(round(W/s + zp + V)), W' = s*(q - zp).
+ *     - "AutoRoundModifier 생성자 파라미터": iters 200, lr 0.005, minmax_lr None -> lr,
+ *       minmax_shrink 1.0.
+ *   "Introducing AutoRound: Intel's Advanced Quantization for LLMs and VLMs",
+ *     section 2: rounding and the clipping range are tuned jointly; section 4:
+ *     iters = 0 is RTN.
+ *   "[SGLang] AutoRound: 자동 라운딩 최적화 양자화", "1. AutoRoundConfig": bits in
+ *     {2, 3, 4, 8}; pack_factor = 32 / bits.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned DEVICE memory, row-major and contiguous,
+ *     unless a parameter says otherwise.  The library allocates nothing; scratch
+ *     memory comes from the caller as a workspace.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  Results are valid once the stream has
+ *     been synchronised.
+ *   - The return value reports argument errors (AR_EINVAL, AR_EUNSUPPORTED) and
+ *     launch errors (AR_ECUDA).  On any non-AR_OK return nothing has been
+ *     enqueued and no output has been written.  Errors detected on the device
+ *     (a bounded wait that ran out) are recorded in the workspace and read with
+ *     ar_tune_status().  Nothing aborts the process.
+ *   - Shapes: W is [out, in]; a quantisation group is `group_size` consecutive
+ *     elements of one row (-1: the whole row); G = in / group_size groups per row.
+ *     Q = 2^bits - 1.  Codes are unsigned in [0, Q].
+ *   - Arithmetic of the quantiser is IEEE fp32, one correctly rounded operation
+ *     at a time, in this order (asymmetric):
+ *       wmin = min(0, min W_grp), wmax = max(0, max W_grp)
+ *       s  = (alpha*wmax - beta*wmin) / Q   (s = 1 for an all-zero group)
+ *       zp = clamp(rint(-(beta*wmin) / s), 0, Q)
+ *       q  = clamp(rint(W/s + V) + zp, 0, Q),  W' = s*(q - zp)
+ *     symmetric: amax = max(-wmin, wmax), s = (2*(alpha*amax)) / Q, zp = 2^(bits-1).
+ *     rint rounds half to even.  Same inputs give bit-identical codes, scales
+ *     and zero-points on every call.
+ */
+#ifndef AR_H_
+#define AR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AR_OK = 0,
+  AR_EINVAL = 1,        /* an argument is out of its documented range */
+  AR_EUNSUPPORTED = 2,  /* valid for the method, not implemented by this library */
+  AR_ENOMEM = 3,        /* the workspace is smaller than ar_tune_workspace_bytes() */
+  AR_ECUDA = 4,         /* a CUDA call failed (no device, launch failure, ...) */
+  AR_ETIMEOUT = 5       /* a device-side bounded wait ran out (see ar_tune_status) */
+} ar_status;
+
+typedef enum { AR_F32 = 0, AR_BF16 = 1 } ar_dtype;
+
+/* Hyper-parameters of ar_tune_layer ("AutoRoundModifier" fields, plus the
+ * readings this library makes where the pages are silent). */
+typedef struct {
+  int32_t bits;          /* 2, 3, 4 or 8 */
+  int32_t group_size;    /* -1 (whole row) or a divisor of in; see ar_tune_layer */
+  int32_t sym;           /* 0: asymmetric (alpha, beta); 1: symmetric (alpha only) */
+  int32_t iters;         /* SignSGD steps, >= 0; 0 gives RTN */
+  float lr;              /* step of V, >= 0 (0.005) */
+  float minmax_lr;       /* step of alpha and beta; < 0 means "same as lr" */
+  float minmax_shrink;   /* initial alpha = beta (1.0) */
+  int32_t keep_best;     /* 1: apply, per output row, the state of its lowest batch
+                            loss (step 0 = RTN state included); 0: the last state */
+  int64_t batch_rows;    /* rows of X per step; n_rows must be a multiple */
+  uint64_t seed;         /* seeds the calibration-block schedule */
+  int64_t start_step;    /* first step index (resume); 0 for a fresh run */
+} ar_tune_params;
+
+/* Optional caller-owned tuning state (device memory, fp32).  Lets a caller
+ * inspect the learned variables, and resume: a run of k steps followed by a run
+ * with start_step = k and initialized = 1 equals one run of both. */
+typedef struct {
+  float* V;            /* [out, in]  rounding offsets, in [-0.5, 0.5] */
+  float* alpha;        /* [out, G]   clip factor of the maximum, in [0.5, 1] */
+  float* beta;         /* [out, G]   clip factor of the minimum, in [0.5, 1] */
+  float* best_loss;    /* [out]      per row, lowest batch loss seen (+inf if none) */
+  float* V_best;       /* [out, in]  per row, the state at that row's best step */
+  float* alpha_best;   /* [out, G] */
+  float* beta_best;    /* [out, G] */
+  int32_t initialized; /* 0: the call initialises the state (V = 0, alpha = beta =
+                          minmax_shrink, best_loss = +inf); 1: the call reads it */
+} ar_tune_state;
+
+/* Library version string, e.g. "ar 0.1.0 sm_100a". */
+const char* ar_version(void);
+
+/* Human-readable name of a status code. */
+const char* ar_status_string(ar_status status);
+
+/* Round-to-nearest quantisation (V = 0, alpha = beta = 1).
+ * "[llm-compressor] AutoRound ...", "논문 핵심 내용": w^ = s*round(w/s), with the
+ * min-max scale and zero-point above.
+ *   W      [out, in], fp32 or bf16 (w_dtype), 16-byte aligned.
+ *   codes  [out, in] uint8 out;  scale [out, G] fp32 out;  zp [out, G] int32 out.
+ * out == 0 or in == 0 is a no-op.  AR_EINVAL: bits not in {2,3,4,8}, group_size
+ * not -1 and not a positive divisor of in, a NULL pointer with out*in > 0. */
+ar_status ar_rtn(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, int32_t bits,
+                 int32_t group_size, int32_t sym, uint8_t* codes, float* scale,
+                 int32_t* zp, void* stream);
+
+/* Offset fake-quantisation with given V, alpha, beta ("_fake_quantize_with_offset").
+ *   V [out, in], alpha [out, G], beta [out, G]: fp32 inputs (beta unused when sym).
+ *   codes, scale, zp as for ar_rtn;  Wq [out, in] fp32 out = s*(q - zp), may be NULL.
+ * Errors as for ar_rtn. */
+ar_status ar_fake_quant(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
+                        const float* V, const float* alpha, const float* beta,
+                        int32_t bits, int32_t group_size, int32_t sym, uint8_t* codes,
+                        float* scale, int32_t* zp, float* Wq, void* stream);
+
+/* Pack b-bit codes into int32 words ("[SGLang] AutoRound ...", "1. AutoRoundConfig":
+ * pack_factor = 32/bits, exact for 3 bits).  Each row is one little-endian bit
+ * stream: bit j of code i is bit (i*bits + j) % 32 of word (i*bits + j) / 32.
+ *   codes  [rows, cols] uint8, every value < 2^bits (higher bits are ignored).
+ *   packed [rows, cols*bits/32] int32 out.
+ * AR_EINVAL: bits not in {2,3,4,8}, cols*bits not a multiple of 32, NULL pointer.
+ * rows == 0 or cols == 0 is a no-op. */
+ar_status ar_pack(const uint8_t* codes, int64_t rows, int64_t cols, int32_t bits,
+                  int32_t* packed, void* stream);
+
+/* Bytes of workspace ar_tune_layer needs for these sizes (0 if they are invalid).
+ * Dominated by a transposed copy of X (n_rows*in*2 bytes). */
+size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
+                               const ar_tune_params* params);
+
+/* Tune one linear layer with SignSGD and return its codes, scales and zero-points.
+ * "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END".  Each step t:
+ *   1. fake-quantise W with (V, alpha, beta) (as ar_fake_quant);
+ *   2. R = X_b (W' - W)^T on the step's calibration block X_b of batch_rows rows,
+ *      and the batch loss mean(R^2) (= mean((Y' - Y)^2), Y = X_b W^T; a bias cancels);
+ *   3. G = R^T X_b (dL/dW' up to a positive factor), straight-through through
+ *      every rint, masked where a clamp is active;
+ *   4. V <- clamp(V - lr*sign(dL/dV), -0.5, 0.5); alpha, beta <- clamp(. - mlr*sign(.),
+ *      0.5, 1) with mlr = minmax_lr (lr if < 0); all from gradients at the same point.
+ * Step t uses block perm_e[t mod (n_rows/batch_rows)], perm_e a Fisher-Yates shuffle
+ * per epoch driven by one SplitMix64 stream seeded with `seed`.  The contractions
+ * run on bf16 tensor cores with fp32 accumulation: W' - W and R are rounded to
+ * bf16 before their products.
+ *   W           [out, in], fp32 or bf16, 16-byte aligned.
+ *   X           [n_rows, in] bf16 (uint16 bit patterns), 16-byte aligned.
+ *   params      host pointer, see ar_tune_params.
+ *   state       host pointer to device buffers, or NULL (state kept in the workspace).
+ *   workspace   device scratch of at least ar_tune_workspace_bytes(), 256-byte
+ *               aligned; its first 4 bytes hold the device status (ar_tune_status).
+ *   codes/scale/zp  outputs as for ar_rtn, from the applied state (keep_best).
+ *   loss_trace  [iters] fp32 out (batch loss of each step), may be NULL.
+ *   final_mse   1 double out: mean((X W'^T - X W^T)^2) over all n_rows rows with
+ *               the applied W', may be NULL (skips one pass over X).
+ * Supported shapes: in a multiple of 32; batch_rows a multiple of 8; group_size a
+ * multiple of 32 that divides 256 or equals in with in <= 256 (else
+ * AR_EUNSUPPORTED).  out == 0 or in == 0 is a no-op.
+ * AR_EINVAL: bad bits/group_size, iters < 0, lr < 0, batch_rows <= 0 or not a
+ * divisor of n_rows, NULL or misaligned pointers.  AR_ENOMEM: ws_bytes too small.
+ * Calls sharing a workspace or state must not overlap on the device. */
+ar_status ar_tune_layer(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
+                        const uint16_t* X, int64_t n_rows, const ar_tune_params* params,
+                        ar_tune_state* state, void* workspace, size_t ws_bytes,
+                        uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
+                        double* final_mse, void* stream);
+
+/* Per-call kernel timing of ar_tune_layer_timed (host struct, filled on return). */
+typedef struct {
+  float residual_ms;         /* summed device time of the R = X_b (W' - W)^T contractions */
+  float update_ms;           /* summed device time of the G = R^T X_b contractions + updates */
+  float total_ms;            /* device time of the whole call */
+  int32_t gemm_launches;     /* launches of each of the two contractions (= iters) */
+  int32_t kernel_launches;   /* every kernel this call launched */
+} ar_tune_timing;
+
+/* ar_tune_layer, with CUDA events recorded on `stream` around each contraction;
+ * synchronises `stream` before returning and fills *timing.  Same arguments,
+ * results and errors as ar_tune_layer; timing must not be NULL. */
+ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
+                              const uint16_t* X, int64_t n_rows, const ar_tune_params* params,
+                              ar_tune_state* state, void* workspace, size_t ws_bytes,
+                              uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
+                              double* final_mse, void* stream, ar_tune_timing* timing);
+
+/* The calibration-block schedule ar_tune_layer follows (host only, no GPU):
+ * blocks[i] = block index of step first + i, i < count, for n_blocks blocks.
+ * Each epoch is a Durstenfeld shuffle of 0..n_blocks-1 (for i = n_blocks-1 down
+ * to 1, swap i with x mod (i+1)), x the successive outputs of one SplitMix64
+ * stream (Steele, Lea & Flood 2014) seeded with `seed`, continued across
+ * epochs; one block draws nothing.  AR_EINVAL if n_blocks < 1, first < 0,
+ * count < 0 or blocks is NULL with count > 0. */
+ar_status ar_block_schedule(int64_t n_blocks, int64_t first, int64_t count, uint64_t seed,
+                            int64_t* blocks);
+
+/* Device status of the last ar_tune_layer call that used `workspace`: synchronises
+ * `stream`, then returns AR_OK, or AR_ETIMEOUT if a kernel's bounded wait ran out
+ * (its results are then invalid), or AR_ECUDA if the stream reports an error. */
+ar_status ar_tune_status(const void* workspace, void* stream);
+
+/* Test hook for the bounded-wait path: one CTA waits on a barrier that nothing
+ * arrives on, gives up after timeout_ns nanoseconds, writes AR_ETIMEOUT into
+ * status[0] (device int) and exits cleanly.  Returns AR_OK once launched. */
+ar_status ar_selftest_timeout(int32_t* status, uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AR_H_ */

@@ -1,0 +1,287 @@
+"""Python binding of libar: AutoRound per-layer SignSGD tuning on one B200.
+
+Argument marshalling only: every step of the computation runs in libar's CUDA
+kernels (``libar.so``, built in-tree by ``python signed_gradient_rounding_b200/build.py``).
+PyTorch provides device memory and streams.  Importing this package fails
+loudly when the library is missing; there is no CPU fallback.
+
+Entry points (same names as the C ABI in include/ar.h):
+  rtn, fake_quant, pack, tune_workspace_bytes, tune_layer, tune_status,
+  and tune_layer_host (host arrays in and out, the copies included).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libar.so")
+
+AR_OK, AR_EINVAL, AR_EUNSUPPORTED, AR_ENOMEM, AR_ECUDA, AR_ETIMEOUT = range(6)
+AR_F32, AR_BF16 = 0, 1
+
+# Every exported symbol of include/ar.h.
+EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
+           "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
+           "ar_tune_status", "ar_selftest_timeout")
+
+
+class ArError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.ar_status_string(status).decode()}")
+
+
+class TuneParams(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("sym", ctypes.c_int32),
+                ("iters", ctypes.c_int32), ("lr", ctypes.c_float), ("minmax_lr", ctypes.c_float),
+                ("minmax_shrink", ctypes.c_float), ("keep_best", ctypes.c_int32),
+                ("batch_rows", ctypes.c_int64), ("seed", ctypes.c_uint64), ("start_step", ctypes.c_int64)]
+
+
+class _TuneStateC(ctypes.Structure):
+    _fields_ = [("V", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("best_loss", ctypes.c_void_p), ("V_best", ctypes.c_void_p),
+                ("alpha_best", ctypes.c_void_p), ("beta_best", ctypes.c_void_p),
+                ("initialized", ctypes.c_int32)]
+
+
+class TuneTiming(ctypes.Structure):
+    _fields_ = [("residual_ms", ctypes.c_float), ("update_ms", ctypes.c_float), ("total_ms", ctypes.c_float),
+                ("gemm_launches", ctypes.c_int32), ("kernel_launches", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python signed_gradient_rounding_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    lib.ar_version.restype = ctypes.c_char_p
+    lib.ar_version.argtypes = []
+    lib.ar_status_string.restype = ctypes.c_char_p
+    lib.ar_status_string.argtypes = [ctypes.c_int]
+    lib.ar_rtn.restype = ctypes.c_int
+    lib.ar_rtn.argtypes = [P, ctypes.c_int, I64, I64, I32, I32, I32, P, P, P, P]
+    lib.ar_fake_quant.restype = ctypes.c_int
+    lib.ar_fake_quant.argtypes = [P, ctypes.c_int, I64, I64, P, P, P, I32, I32, I32, P, P, P, P, P]
+    lib.ar_pack.restype = ctypes.c_int
+    lib.ar_pack.argtypes = [P, I64, I64, I32, P, P]
+    lib.ar_tune_workspace_bytes.restype = SZ
+    lib.ar_tune_workspace_bytes.argtypes = [I64, I64, I64, ctypes.POINTER(TuneParams)]
+    lib.ar_tune_layer.restype = ctypes.c_int
+    lib.ar_tune_layer.argtypes = [P, ctypes.c_int, I64, I64, P, I64, ctypes.POINTER(TuneParams),
+                                  ctypes.POINTER(_TuneStateC), P, SZ, P, P, P, P, P, P]
+    lib.ar_tune_layer_timed.restype = ctypes.c_int
+    lib.ar_tune_layer_timed.argtypes = lib.ar_tune_layer.argtypes + [ctypes.POINTER(TuneTiming)]
+    lib.ar_block_schedule.restype = ctypes.c_int
+    lib.ar_block_schedule.argtypes = [I64, I64, I64, U64, P]
+    lib.ar_tune_status.restype = ctypes.c_int
+    lib.ar_tune_status.argtypes = [P, P]
+    lib.ar_selftest_timeout.restype = ctypes.c_int
+    lib.ar_selftest_timeout.argtypes = [P, U64, P]
+    return lib
+
+
+_lib = _load()
+lib = _lib
+
+
+def version() -> str:
+    return _lib.ar_version().decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != AR_OK:
+        raise ArError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return t
+
+
+def _wdtype(W: torch.Tensor) -> int:
+    if W.dtype == torch.float32:
+        return AR_F32
+    if W.dtype == torch.bfloat16:
+        return AR_BF16
+    raise ValueError("W must be float32 or bfloat16")
+
+
+def _groups(inn: int, group_size: int) -> int:
+    g = inn if group_size == -1 else group_size
+    return inn // g if g > 0 and inn % g == 0 else 0
+
+
+def rtn(W: torch.Tensor, bits: int, group_size: int, sym: bool = False, stream=None):
+    """Round-to-nearest codes (uint8 [out, in]), scales (fp32 [out, G]), zero-points (int32 [out, G])."""
+    _dev(W, "W")
+    out, inn = W.shape
+    G = max(_groups(inn, group_size), 1)
+    codes = torch.empty((out, inn), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((out, G), dtype=torch.float32, device=W.device)
+    zp = torch.empty((out, G), dtype=torch.int32, device=W.device)
+    _check(_lib.ar_rtn(_ptr(W), _wdtype(W), out, inn, bits, group_size, int(sym), _ptr(codes), _ptr(scale),
+                       _ptr(zp), _stream(stream)), "ar_rtn")
+    return codes, scale, zp
+
+
+def fake_quant(W, V, alpha, beta, bits: int, group_size: int, sym: bool = False, want_wq=True, stream=None):
+    """Offset fake-quantisation: (codes, scale, zp, Wq fp32 or None)."""
+    _dev(W, "W")
+    out, inn = W.shape
+    for t, n in ((V, "V"), (alpha, "alpha"), (beta, "beta")):
+        _dev(t, n, torch.float32)
+    G = max(_groups(inn, group_size), 1)
+    codes = torch.empty((out, inn), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((out, G), dtype=torch.float32, device=W.device)
+    zp = torch.empty((out, G), dtype=torch.int32, device=W.device)
+    Wq = torch.empty((out, inn), dtype=torch.float32, device=W.device) if want_wq else None
+    _check(_lib.ar_fake_quant(_ptr(W), _wdtype(W), out, inn, _ptr(V), _ptr(alpha), _ptr(beta), bits,
+                              group_size, int(sym), _ptr(codes), _ptr(scale), _ptr(zp), _ptr(Wq),
+                              _stream(stream)), "ar_fake_quant")
+    return codes, scale, zp, Wq
+
+
+def pack(codes: torch.Tensor, bits: int, stream=None) -> torch.Tensor:
+    """int32 [rows, cols*bits/32]: each row one little-endian bit stream of b-bit codes."""
+    _dev(codes, "codes", torch.uint8)
+    rows, cols = codes.shape
+    packed = torch.empty((rows, cols * bits // 32), dtype=torch.int32, device=codes.device)
+    _check(_lib.ar_pack(_ptr(codes), rows, cols, bits, _ptr(packed), _stream(stream)), "ar_pack")
+    return packed
+
+
+def make_params(bits=4, group_size=128, sym=False, iters=200, lr=0.005, minmax_lr=-1.0, minmax_shrink=1.0,
+                keep_best=True, batch_rows=16384, seed=0, start_step=0) -> TuneParams:
+    return TuneParams(bits, group_size, int(sym), iters, lr, minmax_lr, minmax_shrink, int(keep_best),
+                      batch_rows, seed, start_step)
+
+
+def tune_workspace_bytes(out: int, inn: int, n_rows: int, params: TuneParams) -> int:
+    return int(_lib.ar_tune_workspace_bytes(out, inn, n_rows, ctypes.byref(params)))
+
+
+@dataclasses.dataclass
+class TuneState:
+    """Caller-owned tuning state on the device (see ar_tune_state)."""
+
+    V: torch.Tensor
+    alpha: torch.Tensor
+    beta: torch.Tensor
+    best_loss: torch.Tensor
+    V_best: torch.Tensor
+    alpha_best: torch.Tensor
+    beta_best: torch.Tensor
+    initialized: bool = False
+
+    @classmethod
+    def empty(cls, out: int, inn: int, group_size: int, device="cuda") -> "TuneState":
+        G = max(_groups(inn, group_size), 1)
+        f = dict(dtype=torch.float32, device=device)
+        return cls(torch.empty((out, inn), **f), torch.empty((out, G), **f), torch.empty((out, G), **f),
+                   torch.empty((out,), **f), torch.empty((out, inn), **f), torch.empty((out, G), **f),
+                   torch.empty((out, G), **f))
+
+    def _c(self) -> _TuneStateC:
+        return _TuneStateC(self.V.data_ptr(), self.alpha.data_ptr(), self.beta.data_ptr(),
+                           self.best_loss.data_ptr(), self.V_best.data_ptr(), self.alpha_best.data_ptr(),
+                           self.beta_best.data_ptr(), int(self.initialized))
+
+
+@dataclasses.dataclass
+class TuneResult:
+    codes: torch.Tensor
+    scale: torch.Tensor
+    zero_point: torch.Tensor
+    loss_trace: torch.Tensor | None
+    final_mse: torch.Tensor | None   # 1-element float64 tensor on the device
+    workspace: torch.Tensor
+
+
+def block_schedule(n_blocks: int, first: int, count: int, seed: int) -> list[int]:
+    """The calibration-block index of steps first .. first+count-1 (host computation)."""
+    buf = (ctypes.c_int64 * max(count, 1))()
+    _check(_lib.ar_block_schedule(n_blocks, first, count, seed, ctypes.cast(buf, ctypes.c_void_p)),
+           "ar_block_schedule")
+    return [int(buf[i]) for i in range(count)]
+
+
+def tune_layer(W: torch.Tensor, X: torch.Tensor, params: TuneParams, state: TuneState | None = None,
+               workspace: torch.Tensor | None = None, want_loss_trace: bool = True,
+               want_final_mse: bool = True, outputs=None, stream=None, timing: TuneTiming | None = None
+               ) -> TuneResult:
+    """Run ar_tune_layer on device tensors.  W fp32/bf16 [out, in]; X bf16 [n_rows, in].
+
+    ``outputs`` may pass preallocated (codes, scale, zp, loss_trace, final_mse)
+    tensors so that repeated calls allocate nothing.  With ``timing`` the timed
+    variant runs (synchronising the stream) and fills it.
+    """
+    _dev(W, "W")
+    _dev(X, "X", torch.bfloat16)
+    out, inn = W.shape
+    n_rows = X.shape[0]
+    if X.shape[1] != inn:
+        raise ValueError("X must be [n_rows, in]")
+    need = tune_workspace_bytes(out, inn, n_rows, params)
+    if need == 0:
+        raise ArError(AR_EINVAL, "ar_tune_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    G = max(_groups(inn, params.group_size), 1)
+    if outputs is None:
+        codes = torch.empty((out, inn), dtype=torch.uint8, device=W.device)
+        scale = torch.empty((out, G), dtype=torch.float32, device=W.device)
+        zp = torch.empty((out, G), dtype=torch.int32, device=W.device)
+        trace = torch.empty((max(params.iters, 1),), dtype=torch.float32, device=W.device) if want_loss_trace else None
+        mse = torch.empty((1,), dtype=torch.float64, device=W.device) if want_final_mse else None
+    else:
+        codes, scale, zp, trace, mse = outputs
+    st = ctypes.byref(state._c()) if state is not None else None
+    args = (_ptr(W), _wdtype(W), out, inn, _ptr(X), n_rows, ctypes.byref(params), st, _ptr(workspace),
+            workspace.numel(), _ptr(codes), _ptr(scale), _ptr(zp), _ptr(trace), _ptr(mse), _stream(stream))
+    if timing is None:
+        _check(_lib.ar_tune_layer(*args), "ar_tune_layer")
+    else:
+        _check(_lib.ar_tune_layer_timed(*args, ctypes.byref(timing)), "ar_tune_layer_timed")
+    if state is not None:
+        state.initialized = True
+    return TuneResult(codes, scale, zp, trace[:params.iters] if trace is not None else None, mse, workspace)
+
+
+def tune_status(workspace: torch.Tensor, stream=None) -> int:
+    """Device status of the last tuning call on this workspace (synchronises the stream)."""
+    return int(_lib.ar_tune_status(_ptr(workspace), _stream(stream)))
+
+
+def tune_layer_host(W, X, params: TuneParams, device="cuda", want_final_mse: bool = True):
+    """Host arrays in, host arrays out: copies W and X to the device (from pinned
+    memory when given), tunes, and copies codes, scales, zero-points, the loss
+    trace and the final MSE back.  W: fp32 or bf16 CPU tensor; X: bf16 CPU tensor."""
+    Wd = W.to(device, non_blocking=True)
+    Xd = X.to(device, non_blocking=True)
+    res = tune_layer(Wd, Xd, params, want_final_mse=want_final_mse)
+    out = dict(codes=res.codes.to("cpu"), scale=res.scale.to("cpu"), zero_point=res.zero_point.to("cpu"),
+               loss_trace=res.loss_trace.to("cpu") if res.loss_trace is not None else None,
+               final_mse=float(res.final_mse.item()) if res.final_mse is not None else None)
+    _check(tune_status(res.workspace), "ar_tune_layer (device)")
+    return out

@@ -1,0 +1,224 @@
+// Elementwise and reduction kernels of libar: group min-max statistics, scale and
+// zero-point, offset fake-quantisation (RTN when V = 0, alpha = beta = 1), int32
+// bit packing, the bf16 transpose of the calibration activations, and the
+// fixed-order loss reductions.
+#include <math.h>
+
+#include "ar_device.cuh"
+#include "ar_internal.h"
+
+namespace ar {
+
+namespace {
+
+__device__ __forceinline__ float load_w(const void* W, int w_bf16, int64_t idx) {
+  if (w_bf16) return bf16_bits_to_f32(static_cast<const uint16_t*>(W)[idx]);
+  return static_cast<const float*>(W)[idx];
+}
+
+// One warp per group ("[llm-compressor] AutoRound ...", _fake_quantize_with_offset,
+// min-max init).  Group j*G + gi covers W[j, gi*g : (gi+1)*g].
+__global__ void group_quant_kernel(GroupQuantArgs a) {
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= a.out * a.G) return;
+  const int64_t row = warp / a.G;
+  const int64_t col0 = (warp - row * a.G) * a.g;
+  const int64_t base = row * a.in + col0;
+
+  float wmin, wmax;
+  if (a.wmin_in) {
+    wmin = a.wmin_in[warp];
+    wmax = a.wmax_in[warp];
+  } else {
+    float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W)
+    for (int k = lane; k < a.g; k += 32) {
+      const float w = load_w(a.W, a.w_bf16, base + k);
+      mn = fminf(mn, w);
+      mx = fmaxf(mx, w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    wmin = mn;
+    wmax = mx;
+  }
+  const float alpha = a.alpha ? a.alpha[warp] : 1.0f;
+  const float beta = a.beta ? a.beta[warp] : 1.0f;
+  const GroupScale gs = group_scale(wmin, wmax, alpha, beta, a.bits, a.sym != 0);
+  if (lane == 0) {
+    if (a.wmin_out) {
+      a.wmin_out[warp] = wmin;
+      a.wmax_out[warp] = wmax;
+    }
+    if (a.scale) a.scale[warp] = gs.s;
+    if (a.zp) a.zp[warp] = static_cast<int32_t>(gs.zp);
+  }
+  if (!a.codes && !a.Wq && !a.D) return;
+  const float Q = qmaxf(a.bits);
+  for (int k = lane; k < a.g; k += 32) {
+    const float w = load_w(a.W, a.w_bf16, base + k);
+    const float v = a.V ? a.V[base + k] : 0.0f;
+    const ElemQuant e = quant_elem(w, v, gs, Q);
+    if (a.codes) a.codes[base + k] = static_cast<uint8_t>(e.q);
+    if (a.Wq) a.Wq[base + k] = e.wq;
+    if (a.D) a.D[base + k] = __float2bfloat16_rn(__fsub_rn(e.wq, w));
+  }
+}
+
+// One thread per output word; word w of a row holds stream bits [32w, 32w + 32).
+__global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t cols, int bits,
+                            int64_t words_per_row, uint32_t* __restrict__ packed) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= rows * words_per_row) return;
+  const int64_t row = idx / words_per_row;
+  const int64_t w = idx - row * words_per_row;
+  const int64_t bit0 = w * 32;
+  const int64_t first = bit0 / bits;
+  const int64_t last = (bit0 + 31) / bits;
+  const uint32_t mask = (1u << bits) - 1u;
+  const uint8_t* src = codes + row * cols;
+  uint32_t word = 0;
+  for (int64_t i = first; i <= last && i < cols; ++i) {
+    const uint32_t c = static_cast<uint32_t>(src[i]) & mask;
+    const int64_t shift = i * bits - bit0;
+    if (shift >= 0) {
+      if (shift < 32) word |= c << shift;
+    } else {
+      word |= c >> (-shift);
+    }
+  }
+  packed[idx] = word;
+}
+
+__global__ void fill_f32_kernel(float* p, int64_t n, float v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
+// 64 x 64 tiles through shared memory; 256 threads, each moving 16 elements.
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
+                                      uint16_t* __restrict__ Xt) {
+  __shared__ uint16_t tile[64][66];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 64;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int tx = threadIdx.x & 63;
+  const int ty = threadIdx.x >> 6;  // 0..3
+  for (int i = ty; i < 64; i += 4) {
+    const int64_t r = r0 + i, c = c0 + tx;
+    if (r < rows && c < cols) tile[i][tx] = X[r * cols + c];
+  }
+  __syncthreads();
+  for (int i = ty; i < 64; i += 4) {
+    const int64_t c = c0 + i, r = r0 + tx;
+    if (r < rows && c < cols) Xt[c * rows + r] = tile[tx][i];
+  }
+}
+
+// One block per step; fixed-order fp64 sums.
+__global__ void loss_trace_kernel(const float* __restrict__ rowloss, int64_t out, int64_t batch_rows,
+                                  float* __restrict__ loss_trace) {
+  __shared__ double red[256];
+  const int t = blockIdx.x;
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < out; j += blockDim.x) acc += rowloss[t * out + j];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) loss_trace[t] = static_cast<float>(red[0] / (static_cast<double>(batch_rows) * out));
+}
+
+__global__ void sum_to_double_kernel(const float* __restrict__ parts, int64_t count, double denom,
+                                     double* __restrict__ result) {
+  __shared__ double red[1024];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < count; i += blockDim.x) acc += parts[i];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) result[0] = red[0] / denom;
+}
+
+// A barrier that nothing arrives on: the bounded wait must give up, record the
+// timeout and let the kernel exit.
+__global__ void timeout_selftest_kernel(int32_t* status, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, status, timeout_ns);
+    if (ok) atomicExch(status, -1);  // cannot happen: nothing arrives
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream) {
+  const int64_t groups = a.out * a.G;
+  if (groups == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (groups * 32 + threads - 1) / threads;
+  group_quant_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits, int32_t* packed,
+                        cudaStream_t stream) {
+  const int64_t wpr = cols * bits / 32;
+  const int64_t total = rows * wpr;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  pack_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, stream>>>(
+      codes, rows, cols, bits, wpr, reinterpret_cast<uint32_t*>(packed));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, n, value);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt,
+                                  cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>((cols + 63) / 64), static_cast<unsigned>((rows + 63) / 64));
+  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, Xt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loss_trace(const float* rowloss, int64_t out, int iters, int64_t batch_rows,
+                              float* loss_trace, cudaStream_t stream) {
+  if (iters == 0) return cudaSuccess;
+  loss_trace_kernel<<<iters, 256, 0, stream>>>(rowloss, out, batch_rows, loss_trace);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sum_to_double(const float* parts, int64_t count, double denom, double* result,
+                                 cudaStream_t stream) {
+  sum_to_double_kernel<<<1, 1024, 0, stream>>>(parts, count, denom, result);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t stream) {
+  timeout_selftest_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace ar

@@ -1,0 +1,92 @@
+"""The C-ABI library: loads without a GPU, exports every declared symbol, and its
+host-only logic (argument validation, workspace sizing, block schedule) behaves."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ar():
+    import signed_gradient_rounding_b200 as ar
+    return ar
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "ar.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ar_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(ar):
+    declared = _declared_functions()
+    assert declared == sorted(ar.EXPORTS)
+    lib = ctypes.CDLL(ar.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(ar):
+    assert ar.version().startswith("ar ")
+    for s in range(6):
+        assert ar.lib.ar_status_string(s).decode().startswith("AR_")
+
+
+def test_argument_validation_needs_no_gpu(ar):
+    lib = ar.lib
+    dummy = ctypes.c_void_p(256)
+    # bad bit width, bad group size, bad pack width: rejected before any CUDA call
+    assert lib.ar_rtn(dummy, 0, 4, 64, 5, 32, 0, dummy, dummy, dummy, None) == ar.AR_EINVAL
+    assert lib.ar_rtn(dummy, 0, 4, 64, 4, 48, 0, dummy, dummy, dummy, None) == ar.AR_EINVAL
+    assert lib.ar_rtn(dummy, 0, 4, 64, 4, 32, 0, None, dummy, dummy, None) == ar.AR_EINVAL
+    assert lib.ar_pack(dummy, 4, 10, 3, dummy, None) == ar.AR_EINVAL
+    # empty inputs are a no-op
+    assert lib.ar_rtn(None, 0, 0, 64, 4, 32, 0, None, None, None, None) == ar.AR_OK
+    assert lib.ar_pack(None, 0, 32, 3, None, None) == ar.AR_OK
+
+
+def test_tune_validation(ar):
+    lib = ar.lib
+    dummy = ctypes.c_void_p(4096)
+
+    def call(out, inn, n, **kw):
+        p = ar.make_params(**kw)
+        return lib.ar_tune_layer(dummy, 1, out, inn, dummy, n, ctypes.byref(p), None, dummy, 1 << 40,
+                                 dummy, dummy, dummy, None, None, None)
+
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, bits=5) == ar.AR_EINVAL
+    assert call(64, 256, 1000, batch_rows=512, group_size=64) == ar.AR_EINVAL         # n % B
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, iters=-1) == ar.AR_EINVAL
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, lr=-0.1) == ar.AR_EINVAL
+    assert call(64, 256, 1024, batch_rows=512, group_size=16) == ar.AR_EUNSUPPORTED   # g < 32
+    assert call(64, 1024, 1024, batch_rows=512, group_size=512) == ar.AR_EUNSUPPORTED  # g straddles tiles
+    assert call(64, 250, 1024, batch_rows=512, group_size=-1) == ar.AR_EUNSUPPORTED   # in % 32
+    assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK              # empty layer
+    # too small a workspace
+    p = ar.make_params(batch_rows=512, group_size=64)
+    assert lib.ar_tune_layer(dummy, 1, 64, 256, dummy, 1024, ctypes.byref(p), None, dummy, 1024,
+                             dummy, dummy, dummy, None, None, None) == ar.AR_ENOMEM
+
+
+def test_workspace_bytes(ar):
+    p = ar.make_params(batch_rows=16384, group_size=128)
+    ws = ar.tune_workspace_bytes(4096, 4096, 262144, p)
+    assert ws >= 262144 * 4096 * 2 + 4096 * 16384 * 2 + 4096 * 4096 * (2 + 4 + 4)
+    assert ws < 3.0e9
+    assert ar.tune_workspace_bytes(4096, 4096, 262143, p) == 0
+    bad = ar.make_params(batch_rows=16384, group_size=100)
+    assert ar.tune_workspace_bytes(4096, 4096, 262144, bad) == 0
+
+
+@pytest.mark.parametrize("n_blocks,seed", [(16, 0), (16, 123), (3, 7), (1, 0), (97, 2 ** 63 + 5)])
+def test_block_schedule_matches_oracle(ar, n_blocks, seed):
+    total = 5 * n_blocks + 3
+    assert ar.block_schedule(n_blocks, 0, total, seed) == oracle.block_schedule(n_blocks, total, seed)
+    first = min(11, total // 2)
+    assert ar.block_schedule(n_blocks, first, total - first, seed) == \
+        oracle.block_schedule(n_blocks, total, seed)[first:]

@@ -1,0 +1,299 @@
+"""GPU parity: libar's CUDA path against the CPU oracle, through the C ABI.
+
+Bit-exact: RTN, fixed-offset fake-quantisation, packing, iters = 0, the block
+schedule, determinism, resume and row permutation.  The tuning loop itself
+uses bf16 tensor-core contractions (W' - W and R rounded to bf16) against the
+oracle's fp64, so gradient signs that are near zero can differ and the
+trajectories fork; there the bar is: at most 0.5% of the codes differ and the
+final layer MSE agrees within 2% relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import autoround as oar
+from workloads import (Q_PROJ_7B, TINY, bf16_round, make_activations, make_activations_cuda,
+                       make_weight)
+
+pytestmark = pytest.mark.gpu
+
+CODE_TOL = 0.005      # fraction of codes allowed to differ after tuning
+MSE_RTOL = 0.02       # relative tolerance of the final layer MSE
+
+
+@pytest.fixture(scope="module")
+def ar():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import signed_gradient_rounding_b200 as ar
+    return ar
+
+
+def _w_dev(W, dtype):
+    t = torch.from_numpy(W)
+    return (t.to(torch.bfloat16) if dtype == "bf16" else t).cuda()
+
+
+def _x_dev(X):
+    return torch.from_numpy(X).to(torch.bfloat16).cuda()
+
+
+def _x_bits(Xd):
+    return Xd.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _np(t):
+    return t.cpu().numpy()
+
+
+# ------------------------------------------------------------------ bit-exact parts
+
+RTN_SHAPES = [(3, 192, 64, "f32"), (37, 96, -1, "bf16"), (130, 320, 32, "f32"), (1, 8, 8, "f32"),
+              (256, 4096, 128, "bf16"), (64, 11008, 128, "bf16")]
+
+
+@pytest.mark.parametrize("shape", RTN_SHAPES)
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("sym", [False, True])
+def test_rtn_bitexact(ar, shape, bits, sym):
+    out, inn, g, dt = shape
+    W = make_weight(out, inn, 0.02, dt, seed=out + inn)
+    if out > 2:
+        W[1, :min(inn, 8)] = 0.0                       # zero group / zero block
+        W[2] = np.abs(W[2])                            # one-signed row
+    codes, scale, zp = ar.rtn(_w_dev(W, dt), bits, g, sym)
+    torch.cuda.synchronize()
+    c, s, z, _ = oracle.rtn(W, bits, g, sym)
+    assert np.array_equal(_np(codes), c)
+    assert np.array_equal(_np(scale), s)
+    assert np.array_equal(_np(zp), z)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("sym", [False, True])
+def test_fake_quant_bitexact(ar, bits, sym):
+    out, inn, g = 70, 384, 64
+    W = make_weight(out, inn, 0.02, "bf16", seed=bits)
+    rng = np.random.default_rng(bits + 10 * sym)
+    V = rng.uniform(-0.5, 0.5, (out, inn)).astype(np.float32)
+    V[0] = 0.5
+    V[1] = -0.5
+    G = inn // g
+    alpha = rng.uniform(0.5, 1.0, (out, G)).astype(np.float32)
+    beta = rng.uniform(0.5, 1.0, (out, G)).astype(np.float32)
+    alpha[:, 0] = 0.5
+    beta[:, 1] = 1.0
+    # offsets that land W/s + V exactly on a half-integer (ties to even)
+    wmin, wmax = oracle.group_minmax(W, g)
+    s, zp = oracle.scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
+    u = W[3] / np.repeat(s[3], g)
+    V[3] = ((np.floor(u) + np.float32(0.5)) - u).astype(np.float32)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    codes, scale, zpd, Wq = ar.fake_quant(_w_dev(W, "bf16"), dev(V), dev(alpha), dev(beta), bits, g, sym)
+    torch.cuda.synchronize()
+    fq = oracle.fake_quant(W, V, s, zp, g, bits)
+    assert np.array_equal(_np(codes), fq.q.astype(np.uint8))
+    assert np.array_equal(_np(scale), s)
+    assert np.array_equal(_np(zpd), zp.astype(np.int32))
+    assert np.array_equal(_np(Wq), fq.Wq)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("shape", [(1, 32), (5, 96), (129, 4096), (0, 64)])
+def test_pack_bitexact(ar, bits, shape):
+    rows, cols = shape
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 2 ** bits, size=(rows, cols), dtype=np.uint8)
+    packed = ar.pack(torch.from_numpy(codes).cuda(), bits)
+    torch.cuda.synchronize()
+    if rows:
+        expect = oracle.pack_codes(codes[:min(rows, 8)], bits)
+        assert np.array_equal(_np(packed)[:min(rows, 8)], expect)
+        assert np.array_equal(oracle.unpack_codes(_np(packed), bits, cols), codes)
+
+
+def test_timeout_path_reports_and_recovers(ar):
+    """A bounded wait that nothing satisfies gives up, reports AR_ETIMEOUT and the
+    context stays usable."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert ar.lib.ar_selftest_timeout(ar._ptr(status), 2_000_000, ar._stream(None)) == ar.AR_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) == ar.AR_ETIMEOUT
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum().item()) == 8.0
+
+
+# ------------------------------------------------------------------ tuning loop
+
+def _tune_both(ar, W, X, wdt, bits, g, sym, iters, lr, mlr, B, seed, keep_best=True):
+    Wd = _w_dev(W, wdt)
+    Xd = _x_dev(X)
+    p = ar.make_params(bits=bits, group_size=g, sym=sym, iters=iters, lr=lr, minmax_lr=mlr,
+                       batch_rows=B, seed=seed, keep_best=keep_best)
+    res = ar.tune_layer(Wd, Xd, p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, X, bits, g, sym, iters, lr, mlr, B, seed, keep_best=keep_best)
+    return res, ref
+
+
+def _assert_tuned_close(res, ref, what):
+    codes = _np(res.codes)
+    frac = float(np.mean(codes != ref.codes))
+    mse = float(res.final_mse.item())
+    assert frac <= CODE_TOL, f"{what}: {frac:.4%} of codes differ"
+    assert mse == pytest.approx(ref.final_mse, rel=MSE_RTOL), f"{what}: mse {mse} vs {ref.final_mse}"
+    return frac
+
+
+def test_iters_zero_is_rtn(ar):
+    W = make_weight(200, 320, 0.02, "bf16", seed=1)
+    X = make_activations(1024, 320, "llm", seed=1)
+    for sym in (False, True):
+        p = ar.make_params(bits=3, group_size=64, sym=sym, iters=0, batch_rows=512)
+        res = ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p)
+        torch.cuda.synchronize()
+        c, s, z, Wq = oracle.rtn(W, 3, 64, sym)
+        assert np.array_equal(_np(res.codes), c)
+        assert np.array_equal(_np(res.scale), s)
+        assert np.array_equal(_np(res.zero_point), z)
+        assert float(res.final_mse.item()) == pytest.approx(oar.layer_mse(W, Wq, X), rel=5e-3)
+
+
+def test_tiny_workload(ar):
+    """256x256 fp32 W, W4 g64 asymmetric, 512 rows (full batch), 50 steps."""
+    c = TINY
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    X = make_activations(c.n_rows, c.inn, c.x_kind, seed=0)
+    for keep_best in (True, False):
+        res, ref = _tune_both(ar, W, X, c.w_dtype, c.bits, c.group_size, c.sym, c.iters, c.lr,
+                              c.minmax_lr, c.batch_rows, 0, keep_best)
+        _assert_tuned_close(res, ref, f"tiny keep_best={keep_best}")
+        trace = _np(res.loss_trace).astype(np.float64)
+        np.testing.assert_allclose(trace[0], ref.loss_trace[0], rtol=5e-3)
+        np.testing.assert_allclose(trace, ref.loss_trace, rtol=0.05)
+
+
+@pytest.mark.parametrize("bits,g,sym,wdt", [(3, 64, False, "bf16"), (2, 32, False, "f32"),
+                                            (4, 128, True, "bf16"), (8, 256, False, "bf16")])
+def test_ragged_multiblock(ar, bits, g, sym, wdt):
+    """out and in not multiples of the 128 x 256 tile, three calibration blocks."""
+    out, inn, n, B = 200, 768 if g == 256 else 320 if g != 128 else 384, 1536, 512
+    W = make_weight(out, inn, 0.02, wdt, seed=7)
+    X = make_activations(n, inn, "llm", seed=7)
+    res, ref = _tune_both(ar, W, X, wdt, bits, g, sym, 24, 0.005, 0.005, B, 3)
+    _assert_tuned_close(res, ref, "ragged")
+
+
+def test_one_step_signs(ar):
+    """One step from V = 0, clip factors frozen: V1 = -lr*sign(G)*m wherever the
+    gradient is clearly away from zero."""
+    out, inn, n = 256, 512, 512
+    W = make_weight(out, inn, 0.02, "bf16", seed=11)
+    X = make_activations(n, inn, "llm", seed=11)
+    st = ar.TuneState.empty(out, inn, 128)
+    p = ar.make_params(bits=4, group_size=128, iters=1, minmax_lr=0.0, batch_rows=n, keep_best=False)
+    ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p, state=st)
+    torch.cuda.synchronize()
+    V1 = _np(st.V)
+    wmin, wmax = oracle.group_minmax(W, 128)
+    one = np.ones_like(wmin)
+    s, zp = oracle.scale_zero_point(wmin, wmax, one, one, 4, False)
+    Wq = oracle.fake_quant(W, np.zeros_like(W), s, zp, 128, 4).Wq
+    X64 = X.astype(np.float64)
+    G = (X64 @ (Wq.astype(np.float64) - W).T).T @ X64
+    sgn, _, _ = oracle.step_gradients(W, np.zeros_like(W), one, one, wmin, wmax, G, 128, 4, False)
+    expect = (-np.float32(0.005) * sgn).astype(np.float32)
+    clear = np.abs(G) > 0.02 * np.sqrt(np.mean(G ** 2))
+    assert np.array_equal(V1[clear], expect[clear])
+    assert np.mean(V1 != expect) < 0.01
+    assert np.array_equal(_np(st.alpha), one)
+
+
+def test_deterministic_and_resume(ar):
+    out, inn, n, B = 256, 512, 2048, 512
+    W = make_weight(out, inn, 0.02, "bf16", seed=21)
+    X = make_activations(n, inn, "llm", seed=21)
+    Wd, Xd = _w_dev(W, "bf16"), _x_dev(X)
+    p = ar.make_params(bits=4, group_size=128, iters=30, batch_rows=B, seed=5)
+    a = ar.tune_layer(Wd, Xd, p)
+    b = ar.tune_layer(Wd, Xd, p)
+    torch.cuda.synchronize()
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.scale, b.scale)
+    assert torch.equal(a.loss_trace, b.loss_trace)
+    st = ar.TuneState.empty(out, inn, 128)
+    p1 = ar.make_params(bits=4, group_size=128, iters=11, batch_rows=B, seed=5)
+    r1 = ar.tune_layer(Wd, Xd, p1, state=st)
+    p2 = ar.make_params(bits=4, group_size=128, iters=19, batch_rows=B, seed=5, start_step=11)
+    r2 = ar.tune_layer(Wd, Xd, p2, state=st)
+    torch.cuda.synchronize()
+    assert torch.equal(r2.codes, a.codes) and torch.equal(r2.scale, a.scale)
+    assert torch.equal(torch.cat([r1.loss_trace, r2.loss_trace]), a.loss_trace)
+
+
+def test_row_permutation(ar):
+    """Rows tune independently: permuting the rows of W permutes the results exactly."""
+    out, inn, n = 384, 512, 1024
+    W = make_weight(out, inn, 0.02, "bf16", seed=31)
+    X = make_activations(n, inn, "llm", seed=31)
+    perm = np.random.default_rng(0).permutation(out)
+    Xd = _x_dev(X)
+    p = ar.make_params(bits=2, group_size=128, iters=20, batch_rows=512, seed=2)
+    a = ar.tune_layer(_w_dev(W, "bf16"), Xd, p)
+    b = ar.tune_layer(_w_dev(np.ascontiguousarray(W[perm]), "bf16"), Xd, p)
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(b.codes), _np(a.codes)[perm])
+    assert np.array_equal(_np(b.scale), _np(a.scale)[perm])
+
+
+def test_state_ranges(ar):
+    out, inn, n = 200, 320, 1024
+    W = make_weight(out, inn, 0.02, "bf16", seed=41)
+    X = make_activations(n, inn, "llm", seed=41)
+    st = ar.TuneState.empty(out, inn, 64)
+    p = ar.make_params(bits=2, group_size=64, iters=120, lr=0.02, minmax_lr=0.02, batch_rows=512)
+    res = ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p, state=st)
+    torch.cuda.synchronize()
+    V, a, b = _np(st.V), _np(st.alpha), _np(st.beta)
+    assert V.min() >= -0.5 and V.max() <= 0.5 and (np.abs(V) == 0.5).any()
+    assert a.min() >= 0.5 and a.max() <= 1.0 and b.min() >= 0.5 and b.max() <= 1.0
+    assert _np(res.codes).max() <= 3
+    assert np.all(np.isfinite(_np(st.best_loss)))
+
+
+def test_rejects_unsupported(ar):
+    W = torch.zeros((64, 256), dtype=torch.bfloat16, device="cuda")
+    X = torch.zeros((512, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ar.ArError) as e:
+        ar.tune_layer(W, X, ar.make_params(group_size=16, batch_rows=512))
+    assert e.value.status in (ar.AR_EUNSUPPORTED, ar.AR_EINVAL)
+
+
+def test_q_proj_full_size_sampled_rows(ar):
+    """The LLaMA-7B q_proj workload at full size (4096 x 4096 W4 g128, 262144 x 4096
+    activations, 16384 rows per step, 200 steps), run as the benchmark runs it.
+    Rows tune independently, so the oracle replays 64 sampled rows exactly on the
+    full activations; the sampled rows' codes and MSE are compared."""
+    c = Q_PROJ_7B
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
+                       batch_rows=c.batch_rows, seed=0)
+    res = ar.tune_layer(_w_dev(W, "bf16"), Xd, p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    rows = np.sort(np.random.default_rng(0).choice(c.out, 64, replace=False))
+    Xh = _x_bits(Xd)
+    del Xd
+    ref = oracle.tune_layer(W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr,
+                            c.batch_rows, 0)
+    codes = _np(res.codes)[rows]
+    frac = float(np.mean(codes != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of sampled codes differ"
+    # MSE of the GPU's sampled rows, evaluated by the oracle's own fp64 loss
+    s = _np(res.scale)[rows]
+    z = _np(res.zero_point)[rows].astype(np.float32)
+    Wq_gpu = np.repeat(s, c.group_size, 1) * (codes.astype(np.float32) - np.repeat(z, c.group_size, 1))
+    mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:65536])
+    mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:65536])
+    assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
+    _, _, _, Wrtn = oracle.rtn(W[rows], c.bits, c.group_size, c.sym)
+    assert mse_gpu < oar.layer_mse(W[rows], Wrtn, Xh[:65536])
