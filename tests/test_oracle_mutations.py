@@ -1,0 +1,119 @@
+"""Planted mistakes: each plausible slip in the oracle must make one of its pins fail.
+
+The mistakes are planted in the oracle, on the CPU, by monkeypatching one of its
+functions with a wrong variant; the pins are the functions of test_oracle_pins.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import autoround as oar
+from tests import test_oracle_pins as pins
+
+F32 = np.float32
+
+
+def _szp_zp_sign(wmin, wmax, alpha, beta, bits, sym):
+    s, zp = _orig_szp(wmin, wmax, alpha, beta, bits, sym)
+    if not sym:
+        Q = oar.qmax(bits)
+        zp = np.clip(np.rint((beta * wmin) / s), F32(0), Q).astype(F32)   # lost the minus sign
+    return s, zp
+
+
+def _szp_q_plus_one(wmin, wmax, alpha, beta, bits, sym):
+    s, zp = _orig_szp(wmin, wmax, alpha, beta, bits, sym)
+    s = (s * oar.qmax(bits) / F32(2 ** bits)).astype(F32)                # divided by 2^b, not 2^b - 1
+    return s, zp
+
+
+_orig_szp = oar.scale_zero_point
+_orig_grads = oar.step_gradients
+_orig_fq = oar.fake_quant
+
+
+def _grads_no_mask(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym):
+    sgn, da, db = _orig_grads(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym)
+    return np.sign(G).astype(F32), da, db                                # forgot the clamp mask
+
+
+def _grads_alpha_flipped(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym):
+    sgn, da, db = _orig_grads(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym)
+    return sgn, -da, db                                                  # wrong sign of ds/dalpha
+
+
+def _grads_no_zp_term(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym):
+    # recompute dbeta with the zero-point's derivative dropped in the clamped branch
+    sgn, da, db = _orig_grads(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym)
+    s, zp = oar.scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
+    fq = oar.fake_quant(W, V, s, zp, group_size, bits)
+    g = group_size
+    ds_b = -np.asarray(wmin, np.float64) / float(oar.qmax(bits))
+    qz = fq.q.astype(np.float64) - np.repeat(zp.astype(np.float64), g, 1)
+    ratio = W.astype(np.float64) / np.repeat(s.astype(np.float64), g, 1)
+    dWb = np.where(fq.m, np.repeat(ds_b, g, 1) * (fq.r - ratio), np.repeat(ds_b, g, 1) * qz)
+    db2 = (np.asarray(G) * dWb).reshape(W.shape[0], -1, g).sum(-1)
+    return sgn, da, (np.zeros_like(db2) if sym else db2)
+
+
+def _fq_round_half_up(W, V, s, zp, group_size, bits):
+    fq = _orig_fq(W, V, s, zp, group_size, bits)
+    r = np.floor(fq.t + F32(0.5)).astype(F32)                           # not torch.round's half-to-even
+    Q = oar.qmax(bits)
+    ze = np.repeat(np.asarray(zp, F32), W.shape[1] // np.asarray(s).shape[1], 1)
+    se = np.repeat(np.asarray(s, F32), W.shape[1] // np.asarray(s).shape[1], 1)
+    p = r + ze
+    q = np.clip(p, F32(0), Q)
+    return oar.FakeQuant(fq.u, fq.t, r, p, q, (p >= 0) & (p <= Q), se * (q - ze))
+
+
+def _plant(monkeypatch, name, fn):
+    """Replace an oracle function everywhere it can be reached from."""
+    monkeypatch.setattr(oar, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def _caught(*checks) -> bool:
+    """True if at least one pin fails under the planted mistake."""
+    for check in checks:
+        try:
+            check()
+        except AssertionError:
+            return True
+    return False
+
+
+RTN_PINS = (lambda: pins.test_rtn_worked_grid_example(), lambda: pins.test_rtn_is_nearest_level(4, False),
+            lambda: pins.test_rtn_minmax_span(4))
+
+
+def test_zero_point_sign_is_caught(monkeypatch):
+    _plant(monkeypatch, "scale_zero_point", _szp_zp_sign)
+    assert _caught(*RTN_PINS)
+
+
+def test_wrong_level_count_is_caught(monkeypatch):
+    _plant(monkeypatch, "scale_zero_point", _szp_q_plus_one)
+    assert _caught(*RTN_PINS)
+
+
+@pytest.mark.parametrize("mutant", [_grads_no_mask, _grads_alpha_flipped, _grads_no_zp_term])
+def test_gradient_mistakes_are_caught(monkeypatch, mutant):
+    _plant(monkeypatch, "step_gradients", mutant)
+    with pytest.raises(AssertionError):
+        pins.test_gradients_match_autograd(False, 2)
+
+
+def test_update_direction_is_caught(monkeypatch):
+    def ascend(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym):
+        sgn, da, db = _orig_grads(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym)
+        return -sgn, -da, -db                                            # V += lr*sign(grad)
+    _plant(monkeypatch, "step_gradients", ascend)
+    with pytest.raises(AssertionError):
+        pins.test_one_step_from_zero()
+
+
+def test_rounding_mode_is_caught(monkeypatch):
+    _plant(monkeypatch, "fake_quant", _fq_round_half_up)
+    with pytest.raises(AssertionError):
+        pins.test_rounding_is_torch_round()

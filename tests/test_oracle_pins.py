@@ -60,6 +60,8 @@ def test_rtn_is_nearest_level(bits, sym):
     assert np.all(mine <= best + se * (2 * ulp_u + 1e-9))
     np.testing.assert_allclose(Wq, np.take_along_axis(levels, codes[..., None].astype(np.int64), -1)[..., 0],
                                rtol=1e-7, atol=0)
+    # the levels cover the group: every element within half a step of its level
+    assert np.all(np.abs(Wq.astype(np.float64) - W) <= se * (0.5 + 2 * ulp_u + 1e-9))
     clear = np.sort(dist, axis=-1)[..., 1] - best > se * (4 * ulp_u + 1e-9)
     assert np.array_equal(codes[clear], dist.argmin(axis=-1)[clear])
     assert codes.max() <= Q
@@ -120,6 +122,27 @@ def test_fixed_offset_rounding_reachable_and_monotone():
     assert np.all(fq_hi.q >= fq.q)
     fq0 = oracle.fake_quant(W, np.zeros_like(W), s, zp, g, bits)
     assert np.all(fq.q[V > 0] >= fq0.q[V > 0]) and np.all(fq.q[V < 0] <= fq0.q[V < 0])
+
+
+def test_rounding_is_torch_round():
+    """The page's code rounds with torch.round (half to even).  On offsets built to
+    put W/s + V exactly on half-integers, the codes equal torch's evaluation of
+    clamp(round(W/s + V) + zp, 0, Q) in fp32."""
+    W = make_weight(4, 64, 0.02, "f32", seed=8)
+    g, bits = 16, 4
+    wmin, wmax = oracle.group_minmax(W, g)
+    one = np.ones_like(wmin)
+    s, zp = oracle.scale_zero_point(wmin, wmax, one, one, bits, False)
+    se = np.repeat(s, g, 1)
+    ze = np.repeat(zp, g, 1)
+    u = W / se
+    V = ((np.floor(u) + F32(0.5)) - u).astype(np.float32)
+    t = u + V
+    assert np.sum(t == np.floor(t) + F32(0.5)) > 100          # many exact ties
+    fq = oracle.fake_quant(W, V, s, zp, g, bits)
+    tq = torch.clamp(torch.round(torch.from_numpy(W) / torch.from_numpy(se) + torch.from_numpy(V))
+                     + torch.from_numpy(ze), 0, 2 ** bits - 1)
+    assert np.array_equal(fq.q, tq.numpy())
 
 
 # ---------------------------------------------------------------- gradients
