@@ -126,7 +126,8 @@ def run_ours(args):
     Wd = (W.to(torch.bfloat16) if c.w_dtype == "bf16" else W).to(dev)
     Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
     p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
-                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0)
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
+                       split=bool(args.split))
     ws = torch.empty(ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
     G = c.inn // c.group_size
     outs = (torch.empty((c.out, c.inn), dtype=torch.uint8, device=dev),
@@ -203,13 +204,26 @@ def run_ours(args):
         return None
 
     peaks = _peaks()
-    flops_gemm = 2.0 * c.batch_rows * c.out * c.inn             # one contraction, one launch
-    res_ms = sum(t.residual_ms for t in timings) / sum(t.gemm_launches for t in timings)
-    upd_ms = sum(t.update_ms for t in timings) / sum(t.gemm_launches for t in timings)
-    dom_name, dom_ms = ("update", upd_ms) if upd_ms >= res_ms else ("residual", res_ms)
-    achieved = flops_gemm / (dom_ms * 1e-3) / 1e12
+    algo = {ar.AR_ALGO_DIRECT: "direct", ar.AR_ALGO_GRAM: "gram"}[timings[0].algo]
+    pieces = (3 if algo == "gram" else 2) if args.split else 1
+    if algo == "gram":
+        # one launch per step: G = D H_b, D and H_b as bf16 pairs (3 products)
+        flops_upd = pieces * 2.0 * c.out * c.inn * c.inn
+        flops_res = 0.0
+    else:
+        # two launches per step: R = X_b D^T and G = R^T X_b, operands as bf16 pairs
+        flops_res = flops_upd = pieces * 2.0 * c.batch_rows * c.out * c.inn
+    n_launch = sum(t.gemm_launches for t in timings)
+    res_ms = sum(t.residual_ms for t in timings) / n_launch
+    upd_ms = sum(t.update_ms for t in timings) / n_launch
+    if res_ms > upd_ms:
+        dom_name, dom_ms, dom_flops = "residual (kEpiStore)", res_ms, flops_res
+    else:
+        dom_name, dom_ms, dom_flops = "update (kEpiUpdate)", upd_ms, flops_upd
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     layer_s = ms_max / args.steps / 1e3
-    step_tflops = c.flops_per_step * c.iters / layer_s / 1e12
+    step_ms = res_ms + upd_ms
+    step_tflops = (flops_res + flops_upd) / (step_ms * 1e-3) / 1e12
     launches = sum(t.kernel_launches for t in timings) + args.steps    # + one pack per step
     line = {
         "metric": METRIC,
@@ -226,16 +240,22 @@ def run_ours(args):
         "data": "synthetic",
         "config": {"workload": c.name, "out": c.out, "in": c.inn, "n_rows": c.n_rows,
                    "batch_rows": c.batch_rows, "iters": c.iters, "bits": c.bits, "group_size": c.group_size,
-                   "sym": c.sym, "lr": c.lr, "minmax_lr": c.minmax_lr, "keep_best": True,
+                   "sym": c.sym, "lr": c.lr, "minmax_lr": c.minmax_lr, "keep_best": True, "algo": algo,
                    "bench_step": "one ar_tune_layer call (all iters) + ar_pack",
                    "l2": "inputs larger than L2: X is %.1f GB, one step reads a %.0f MB block"
                          % (c.n_rows * c.inn * 2 / 1e9, c.batch_rows * c.inn * 2 / 1e6),
                    "parallelism": f"row shards x{world}, no data-path collective"},
         "layer_tune_s": layer_s,
+        "algo": algo,
+        "split_operands": bool(args.split),
+        "step_ms": step_ms,
+        "setup_ms": sum(t.setup_ms for t in timings) / len(timings),
+        "executed_tflop_per_step": (flops_res + flops_upd) / 1e12,
         "fused_step_tflops": step_tflops,
         "tensor_peak_frac": step_tflops / peaks["bf16_tflops_sustained"],
+        "direct_form_tflop_per_step": c.flops_per_step / 1e12,
         "final_mse": mse,
-        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel<{dom_name}>", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel {algo} {dom_name}", "achieved": achieved,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
                      "peak_source": peaks["source"] + " sustained bf16",
@@ -337,6 +357,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--cpu-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--algo", choices=["auto", "direct", "gram"], default="auto")
+    ap.add_argument("--split", type=int, default=1, help="1: bf16-pair operands (default); 0: single bf16")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

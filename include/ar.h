@@ -61,6 +61,18 @@ typedef enum {
 
 typedef enum { AR_F32 = 0, AR_BF16 = 1 } ar_dtype;
 
+/* How ar_tune_layer evaluates the two products of each step (same mathematics):
+ *   AR_ALGO_DIRECT: R = X_b D^T (D = W' - W), then G = R^T X_b.  Per step
+ *                   4*B*out*in flops (x2 with split operands).
+ *   AR_ALGO_GRAM:   G = D H_b with H_b = X_b^T X_b, the calibration block's Gram
+ *                   matrix, computed once per call for every block; the loss is
+ *                   sum_k D_jk G_jk = sum_b R_bj^2.  Per step 2*out*in^2 flops (x3
+ *                   with split operands), plus 2*n_rows*in^2 once, and
+ *                   n_rows/B * in^2 * 4 bytes of workspace.
+ *   AR_ALGO_AUTO:   the one with fewer flops over the whole call (GRAM only while
+ *                   its matrices take at most 64 GiB). */
+typedef enum { AR_ALGO_AUTO = 0, AR_ALGO_DIRECT = 1, AR_ALGO_GRAM = 2 } ar_algo;
+
 /* Hyper-parameters of ar_tune_layer ("AutoRoundModifier" fields, plus the
  * readings this library makes where the pages are silent). */
 typedef struct {
@@ -76,6 +88,11 @@ typedef struct {
   int64_t batch_rows;    /* rows of X per step; n_rows must be a multiple */
   uint64_t seed;         /* seeds the calibration-block schedule */
   int64_t start_step;    /* first step index (resume); 0 for a fresh run */
+  int32_t algo;          /* ar_algo (0: auto) */
+  int32_t split;         /* 1: tensor-core operands as exact bf16 pairs hi + lo
+                            (hi = bf16(x), lo = bf16(x - hi): ~16 significant bits);
+                            0: single bf16 (faster, the tuning trajectory drifts
+                            further from an exact evaluation) */
 } ar_tune_params;
 
 /* Optional caller-owned tuning state (device memory, fp32).  Lets a caller
@@ -129,8 +146,9 @@ ar_status ar_fake_quant(const void* W, ar_dtype w_dtype, int64_t out, int64_t in
 ar_status ar_pack(const uint8_t* codes, int64_t rows, int64_t cols, int32_t bits,
                   int32_t* packed, void* stream);
 
-/* Bytes of workspace ar_tune_layer needs for these sizes (0 if they are invalid).
- * Dominated by a transposed copy of X (n_rows*in*2 bytes). */
+/* Bytes of workspace ar_tune_layer needs for these sizes and params (0 if they are
+ * invalid).  Dominated by a transposed copy of X (n_rows*in*2 bytes) and, for
+ * AR_ALGO_GRAM, the Gram matrices (n_rows/batch_rows * in^2 * 4 bytes). */
 size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
                                const ar_tune_params* params);
 
@@ -171,11 +189,14 @@ ar_status ar_tune_layer(const void* W, ar_dtype w_dtype, int64_t out, int64_t in
 
 /* Per-call kernel timing of ar_tune_layer_timed (host struct, filled on return). */
 typedef struct {
-  float residual_ms;         /* summed device time of the R = X_b (W' - W)^T contractions */
-  float update_ms;           /* summed device time of the G = R^T X_b contractions + updates */
+  float residual_ms;         /* DIRECT: summed device time of the R = X_b (W' - W)^T
+                                contractions; GRAM: 0 */
+  float update_ms;           /* summed device time of the G contractions + updates */
   float total_ms;            /* device time of the whole call */
-  int32_t gemm_launches;     /* launches of each of the two contractions (= iters) */
+  int32_t gemm_launches;     /* launches of each timed contraction (= iters) */
   int32_t kernel_launches;   /* every kernel this call launched */
+  int32_t algo;              /* the ar_algo the call ran (DIRECT or GRAM) */
+  float setup_ms;            /* device time before the first step (transpose, Gram matrices) */
 } ar_tune_timing;
 
 /* ar_tune_layer, with CUDA events recorded on `stream` around each contraction;

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -44,6 +45,8 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+namespace {
+
 // ---------------------------------------------------------------------------
 // Calibration-block schedule.  The pages iterate over calibration batches without
 // saying how one is picked per step; this library visits the n/B blocks once per
@@ -52,8 +55,6 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
 // stream (Steele, Lea & Flood, OOPSLA 2014) seeded with `seed` and continued
 // across epochs.  A single block draws nothing.
 // ---------------------------------------------------------------------------
-
-namespace {
 
 struct SplitMix64 {
   uint64_t state;
@@ -109,53 +110,19 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Workspace layout of ar_tune_layer (offsets in bytes from the workspace base).
-struct Layout {
-  size_t status, Xt, Rt, D, V, alpha, beta, V_best, alpha_best, beta_best, best_loss, best_alt, wmin, wmax, part,
-      rowloss, total;
-};
-
-Layout make_layout(int64_t out, int64_t in, int64_t n, int64_t B, int64_t G, int64_t iters) {
-  Layout L{};
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t o = off;
-    off = round_up(off + bytes, 1024);
-    return o;
-  };
-  const int64_t nparts = std::max(cdiv(B, kBN), cdiv(n, kBN));
-  L.status = take(256);
-  L.Xt = take(static_cast<size_t>(in) * n * 2);
-  L.Rt = take(static_cast<size_t>(out) * B * 2);
-  L.D = take(static_cast<size_t>(out) * in * 2);
-  L.V = take(static_cast<size_t>(out) * in * 4);
-  L.alpha = take(static_cast<size_t>(out) * G * 4);
-  L.beta = take(static_cast<size_t>(out) * G * 4);
-  L.V_best = take(static_cast<size_t>(out) * in * 4);
-  L.alpha_best = take(static_cast<size_t>(out) * G * 4);
-  L.beta_best = take(static_cast<size_t>(out) * G * 4);
-  L.best_loss = take(static_cast<size_t>(out) * 4);
-  L.best_alt = take(static_cast<size_t>(out) * 4);
-  L.wmin = take(static_cast<size_t>(out) * G * 4);
-  L.wmax = take(static_cast<size_t>(out) * G * 4);
-  L.part = take(static_cast<size_t>(out) * nparts * 4);
-  L.rowloss = take(static_cast<size_t>(out) * std::max<int64_t>(iters, 1) * 4);
-  L.total = off;
-  return L;
-}
-
 ar_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AR_OK : AR_ECUDA; }
 
-#define AR_CUDA_TRY(expr)                          \
-  do {                                             \
-    cudaError_t e_ = (expr);                       \
-    if (e_ != cudaSuccess) return AR_ECUDA;        \
+#define AR_CUDA_TRY(expr)                   \
+  do {                                      \
+    cudaError_t e_ = (expr);                \
+    if (e_ != cudaSuccess) return AR_ECUDA; \
   } while (0)
 
+// The update epilogue needs whole groups inside one thread's tile columns.
 bool tune_shape_supported(int64_t in, int64_t g, int64_t B) {
   if (in % 32 != 0 || B % 8 != 0) return false;
   if (g % 32 != 0) return false;
-  return (kBN % g == 0) || (g == in && in <= kBN);
+  return (256 % g == 0) || (g == in && in <= 256);
 }
 
 ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune_params* p) {
@@ -164,11 +131,530 @@ ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune
   if (p->iters < 0 || !(p->lr >= 0.0f) || !isfinite(p->lr) || !isfinite(p->minmax_lr)) return AR_EINVAL;
   if (!(p->minmax_shrink > 0.0f) || !isfinite(p->minmax_shrink)) return AR_EINVAL;
   if (p->start_step < 0) return AR_EINVAL;
+  if (p->algo < AR_ALGO_AUTO || p->algo > AR_ALGO_GRAM) return AR_EINVAL;
   if (out == 0 || in == 0) return AR_OK;
   if (!group_ok(in, p->group_size)) return AR_EINVAL;
   if (p->batch_rows <= 0 || n_rows < p->batch_rows || n_rows % p->batch_rows != 0) return AR_EINVAL;
   if (out >= (1ll << 31) || in >= (1ll << 31) || n_rows >= (1ll << 31)) return AR_EUNSUPPORTED;
   if (!tune_shape_supported(in, group_of(in, p->group_size), p->batch_rows)) return AR_EUNSUPPORTED;
+  return AR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Plan: which algorithm, tile widths, workspace layout.
+// ---------------------------------------------------------------------------
+
+struct Plan {
+  int algo = AR_ALGO_DIRECT;
+  int split = 1;
+  int64_t out = 0, in = 0, n = 0, B = 0, g = 0, G = 0, nb = 0, iters = 0;
+  int bn_res = 256;   // direct: residual GEMM (N = B)
+  int bn_upd = 256;   // update GEMM (N = in)
+  int bn_gram = 128;  // Gram matrices (N = in)
+  int bn_fin = 256;   // final-MSE GEMM
+  int64_t nparts_res = 0, nparts_upd = 0, nparts_fin = 0;
+};
+
+constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
+
+Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p) {
+  Plan P;
+  P.split = p->split != 0;
+  P.out = out;
+  P.in = in;
+  P.n = n;
+  P.B = p->batch_rows;
+  P.g = group_of(in, p->group_size);
+  P.G = in / P.g;
+  P.nb = n / P.B;
+  P.iters = p->iters;
+  const double pieces_direct = P.split ? 2.0 : 1.0;
+  const double pieces_gram = P.split ? 3.0 : 1.0;
+  const double direct = P.iters * pieces_direct * 4.0 * P.B * out * in + pieces_direct * 2.0 * n * out * in;
+  const double gram = P.iters * pieces_gram * 2.0 * out * in * in + 2.0 * n * in * in + pieces_gram * 2.0 * out * in * in;
+  const double gram_bytes = (P.nb + 1.0) * in * in * 2.0 * (P.split ? 2.0 : 1.0);
+  if (p->algo == AR_ALGO_GRAM)
+    P.algo = AR_ALGO_GRAM;
+  else if (p->algo == AR_ALGO_DIRECT)
+    P.algo = AR_ALGO_DIRECT;
+  else
+    P.algo = (P.iters > 0 && gram < direct && gram_bytes <= kGramMaxBytes) ? AR_ALGO_GRAM : AR_ALGO_DIRECT;
+  // N tiles of 256: a 128x128x16 MMA reads as many operand bytes from shared
+  // memory per clock as the SM can deliver, 128x256 reads three quarters of that.
+  P.bn_upd = 256;
+  P.bn_gram = 256;
+  P.bn_fin = 256;
+  P.nparts_res = cdiv(P.B, P.bn_res);
+  P.nparts_upd = cdiv(in, P.bn_upd);
+  P.nparts_fin = P.algo == AR_ALGO_GRAM ? cdiv(in, P.bn_fin) : cdiv(n, P.bn_fin);
+  return P;
+}
+
+// Workspace layout (offsets in bytes from the workspace base).
+struct Layout {
+  size_t status, Xt, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
+      part0, part1, rowloss, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum, total;
+};
+
+Layout make_layout(const Plan& P) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 1024);
+    return o;
+  };
+  const size_t elems = static_cast<size_t>(P.out) * P.in;
+  const size_t groups = static_cast<size_t>(P.out) * P.G;
+  const bool gram = P.algo == AR_ALGO_GRAM;
+  const int64_t nparts = std::max(std::max(P.nparts_res, P.nparts_upd), P.nparts_fin);
+  L.status = take(256);
+  L.Xt = take(static_cast<size_t>(P.in) * P.n * 2);
+  L.D_hi = take(elems * 2);
+  L.D_lo = take(elems * 2);
+  // The Gram form reads D_t and writes D_{t+1} in the same launch: two buffers.
+  L.D_hi1 = gram ? take(elems * 2) : L.D_hi;
+  L.D_lo1 = gram ? take(elems * 2) : L.D_lo;
+  L.V0 = take(elems * 4);
+  L.V1 = gram ? take(elems * 4) : L.V0;
+  L.a0 = take(groups * 4);
+  L.b0 = take(groups * 4);
+  L.a1 = gram ? take(groups * 4) : L.a0;
+  L.b1 = gram ? take(groups * 4) : L.b0;
+  L.V_best = take(elems * 4);
+  L.alpha_best = take(groups * 4);
+  L.beta_best = take(groups * 4);
+  L.best0 = take(static_cast<size_t>(P.out) * 4);
+  L.best1 = take(static_cast<size_t>(P.out) * 4);
+  L.wmin = take(groups * 4);
+  L.wmax = take(groups * 4);
+  L.part0 = take(static_cast<size_t>(P.out) * nparts * 4);
+  L.part1 = gram ? take(static_cast<size_t>(P.out) * nparts * 4) : L.part0;
+  L.rowloss = take(static_cast<size_t>(P.out) * std::max<int64_t>(P.iters, 1) * 4);
+  if (gram) {
+    const size_t h = static_cast<size_t>(P.in) * P.in * 2;
+    L.H_hi = take(h * P.nb);
+    L.H_lo = P.split ? take(h * P.nb) : L.H_hi;
+    L.Hs_hi = take(h);
+    L.Hs_lo = P.split ? take(h) : L.Hs_hi;
+    L.Hdiag = take(static_cast<size_t>(P.nb) * P.in * 4);
+    L.Hdsum = take(static_cast<size_t>(P.in) * 4);
+  } else {
+    L.Rt_hi = take(static_cast<size_t>(P.out) * P.B * 2);
+    L.Rt_lo = P.split ? take(static_cast<size_t>(P.out) * P.B * 2) : L.Rt_hi;
+  }
+  L.total = off;
+  return L;
+}
+
+void fill_grid(GemmArgs& a, int64_t M, int64_t N, int64_t K, int bn, int num_seg) {
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.num_m_blk = static_cast<int>(cdiv(M, kBM));
+  a.num_n_blk = static_cast<int>(cdiv(N, bn));
+  a.num_k_blk = static_cast<int>(cdiv(K, kBK));
+  a.num_tiles = a.num_m_blk * a.num_n_blk;
+  a.num_seg = num_seg;
+}
+
+// Events around the contractions of a timed call: ev[2t] before step t's first
+// contraction, ev[2t+1] between the two (DIRECT), ev[2t+2] after the update.
+struct EventTimer {
+  std::vector<cudaEvent_t> ev;
+  cudaEvent_t start = nullptr, stop = nullptr;
+  int launches = 0;
+  int algo = 0;
+  bool create(int iters) {
+    ev.assign(static_cast<size_t>(2 * iters + 1), nullptr);
+    for (auto& e : ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return false;
+    return cudaEventCreate(&start) == cudaSuccess && cudaEventCreate(&stop) == cudaSuccess;
+  }
+  ~EventTimer() {
+    for (auto e : ev)
+      if (e) cudaEventDestroy(e);
+    if (start) cudaEventDestroy(start);
+    if (stop) cudaEventDestroy(stop);
+  }
+};
+
+ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X, int64_t n_rows,
+                    const ar_tune_params* p, ar_tune_state* state, void* workspace, size_t ws_bytes,
+                    uint8_t* codes, float* scale, int32_t* zp, float* loss_trace, double* final_mse,
+                    void* stream, EventTimer* timer) {
+  const ar_status chk = check_tune_args(out, in, n_rows, p);
+  if (chk != AR_OK) return chk;
+  if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
+  if (out == 0 || in == 0) return AR_OK;
+  if (!W || !X || !workspace || !codes || !scale || !zp) return AR_EINVAL;
+  if (!aligned(W, 16) || !aligned(X, 16) || !aligned(workspace, 256)) return AR_EINVAL;
+  if (state) {
+    const void* ptrs[7] = {state->V,      state->alpha,      state->beta,     state->best_loss,
+                           state->V_best, state->alpha_best, state->beta_best};
+    for (const void* q : ptrs)
+      if (!q || !aligned(q, 16)) return AR_EINVAL;
+  }
+
+  const Plan P = make_plan(out, in, n_rows, p);
+  const Layout L = make_layout(P);
+  if (ws_bytes < L.total) return AR_ENOMEM;
+  const bool gram = P.algo == AR_ALGO_GRAM;
+  const int64_t B = P.B;
+  const int iters = p->iters;
+
+  int dev = 0, sms = 0, major = 0;
+  AR_CUDA_TRY(cudaGetDevice(&dev));
+  AR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  AR_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (major != 10) return AR_EUNSUPPORTED;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  auto H = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  uint16_t* Xt = reinterpret_cast<uint16_t*>(ws + L.Xt);
+  __nv_bfloat16* D_hi = H(L.D_hi);
+  __nv_bfloat16* D_lo = H(L.D_lo);
+  __nv_bfloat16* Dh[2] = {D_hi, H(L.D_hi1)};
+  __nv_bfloat16* Dl[2] = {D_lo, H(L.D_lo1)};
+  float* wmin = F(L.wmin);
+  float* wmax = F(L.wmax);
+  float* part[2] = {F(L.part0), F(L.part1)};
+  float* rowloss = F(L.rowloss);
+  // Live state: buffer 0 is the caller's state (or the workspace's); the Gram
+  // form double-buffers V, alpha, beta because its keep-best check of a step runs
+  // one step later.
+  float* Vb[2];
+  float* ab[2];
+  float* bb[2];
+  float *best_loss, *V_best, *alpha_best, *beta_best;
+  if (state) {
+    Vb[0] = state->V;
+    ab[0] = state->alpha;
+    bb[0] = state->beta;
+    best_loss = state->best_loss;
+    V_best = state->V_best;
+    alpha_best = state->alpha_best;
+    beta_best = state->beta_best;
+  } else {
+    Vb[0] = F(L.V0);
+    ab[0] = F(L.a0);
+    bb[0] = F(L.b0);
+    best_loss = F(L.best0);
+    V_best = F(L.V_best);
+    alpha_best = F(L.alpha_best);
+    beta_best = F(L.beta_best);
+  }
+  Vb[1] = gram ? F(L.V1) : Vb[0];
+  ab[1] = gram ? F(L.a1) : ab[0];
+  bb[1] = gram ? F(L.b1) : bb[0];
+  float* best_alt = F(L.best1);
+  const bool init_state = !state || !state->initialized;
+  const size_t elems = static_cast<size_t>(out) * in;
+  const size_t groups = static_cast<size_t>(out) * P.G;
+
+  int launches = 0;
+  if (timer) {
+    timer->algo = P.algo;
+    AR_CUDA_TRY(cudaEventRecord(timer->start, st));
+  }
+  AR_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  if (init_state) {
+    AR_CUDA_TRY(cudaMemsetAsync(Vb[0], 0, elems * 4, st));
+    AR_CUDA_TRY(cudaMemsetAsync(V_best, 0, elems * 4, st));
+    AR_CUDA_TRY(launch_fill_f32(ab[0], groups, p->minmax_shrink, st));
+    AR_CUDA_TRY(launch_fill_f32(bb[0], groups, p->minmax_shrink, st));
+    AR_CUDA_TRY(launch_fill_f32(alpha_best, groups, p->minmax_shrink, st));
+    AR_CUDA_TRY(launch_fill_f32(beta_best, groups, p->minmax_shrink, st));
+    AR_CUDA_TRY(launch_fill_f32(best_loss, out, INFINITY, st));
+    launches += 5;
+  }
+
+  // Group statistics of W and the first step's D = W' - W.
+  GroupQuantArgs prep;
+  prep.W = W;
+  prep.w_bf16 = w_dtype == AR_BF16;
+  prep.out = out;
+  prep.in = in;
+  prep.g = static_cast<int>(P.g);
+  prep.G = static_cast<int>(P.G);
+  prep.bits = p->bits;
+  prep.sym = p->sym != 0;
+  prep.wmin_out = wmin;
+  prep.wmax_out = wmax;
+  prep.V = Vb[0];
+  prep.alpha = ab[0];
+  prep.beta = bb[0];
+  prep.D_hi = D_hi;
+  prep.D_lo = P.split ? D_lo : nullptr;
+  AR_CUDA_TRY(launch_group_quant(prep, st));
+  ++launches;
+
+  const uint64_t timeout_ns = 1000000000ull;
+  const float mlr = p->minmax_lr < 0.0f ? p->lr : p->minmax_lr;
+  const int nseg_d = P.split ? 2 : 1;
+  const int nseg_g = P.split ? 3 : 1;
+  const std::vector<int64_t> sched = block_schedule(P.nb, p->start_step, iters, p->seed);
+  const bool need_xt = iters > 0 || (gram && final_mse);
+
+  if (need_xt) {
+    AR_CUDA_TRY(launch_transpose_bf16(X, n_rows, in, Xt, st));
+    ++launches;
+  }
+
+  // The update epilogue's common arguments.
+  GemmArgs u;
+  u.timeout_ns = timeout_ns;
+  u.status = status;
+  u.W = W;
+  u.w_bf16 = w_dtype == AR_BF16;
+  u.wmin = wmin;
+  u.wmax = wmax;
+  u.D_hi = D_hi;
+  u.D_lo = P.split ? D_lo : nullptr;
+  u.V_best = V_best;
+  u.alpha_best = alpha_best;
+  u.beta_best = beta_best;
+  u.inv_batch = 1.0f / static_cast<float>(B);
+  u.g = static_cast<int>(P.g);
+  u.G = static_cast<int>(P.G);
+  u.bits = p->bits;
+  u.sym = p->sym != 0;
+  u.keep_best = p->keep_best != 0;
+  u.lr = p->lr;
+  u.mlr = mlr;
+
+  float* best_cur = best_loss;
+  float* best_next = best_alt;
+  int live = 0;  // buffer holding the live state
+
+  if (gram) {
+    // ---------------------------------------------------------- Gram form
+    __nv_bfloat16* Hh = H(L.H_hi);
+    __nv_bfloat16* Hl = H(L.H_lo);
+    {  // H_b = X_b^T X_b for every block, as a bf16 pair, rows b*in .. b*in + in
+      GemmMaps m{};
+      AR_CUDA_TRY(make_tmap_bf16(&m.a0, Xt, in, n_rows, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m.b0, Xt, in, n_rows, P.bn_gram));
+      m.a1 = m.a0;
+      m.b1 = m.b0;
+      GemmArgs h;
+      fill_grid(h, in, in, B, P.bn_gram, 1);
+      h.timeout_ns = timeout_ns;
+      h.status = status;
+      h.C_hi = Hh;
+      h.C_lo = P.split ? Hl : nullptr;
+      h.ldc = in;
+      h.diag_out = F(L.Hdiag);
+      for (int64_t b = 0; b < P.nb; ++b) {
+        h.a_k_off = static_cast<int>(b * B);
+        h.b_k_off = static_cast<int>(b * B);
+        h.c_row_off = b * in;
+        AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_gram, m, h, sms, st));
+        ++launches;
+      }
+    }
+    GemmMaps m[2]{};  // per parity of t: A = D_t
+    for (int q = 0; q < 2; ++q) {
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].a0, Dh[q], out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].a1, Dl[q], out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].b0, Hh, P.nb * in, in, P.bn_upd));
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].b1, Hl, P.nb * in, in, P.bn_upd));
+    }
+    fill_grid(u, out, in, in, P.bn_upd, nseg_g);
+    // (D_hi + D_lo)(H_hi + H_lo) ~ D_hi H_hi + D_lo H_hi + D_hi H_lo
+    u.seg_a[0] = 0, u.seg_b[0] = 0;
+    u.seg_a[1] = 1, u.seg_b[1] = 0;
+    u.seg_a[2] = 0, u.seg_b[2] = 1;
+    u.part_ld = static_cast<int>(P.nparts_upd);
+    u.nparts = static_cast<int>(P.nparts_upd);
+    u.snap_prev = 1;
+    for (int t = 0; t < iters; ++t) {
+      const int cur = t & 1, nxt = (t + 1) & 1;
+      u.b_row_off = static_cast<int>(sched[t] * in);
+      u.diag_in = F(L.Hdiag) + sched[t] * in;
+      u.V_in = Vb[cur];
+      u.V_out = Vb[nxt];
+      u.alpha_in = ab[cur];
+      u.alpha_out = ab[nxt];
+      u.beta_in = bb[cur];
+      u.beta_out = bb[nxt];
+      u.D_hi = Dh[nxt];
+      u.D_lo = P.split ? Dl[nxt] : nullptr;
+      u.part_out = part[cur];
+      u.part_in = t > 0 ? part[nxt] : nullptr;  // the previous step's partials
+      u.rowloss = t > 0 ? rowloss + static_cast<int64_t>(t - 1) * out : nullptr;
+      u.best_in = best_cur;
+      u.best_out = best_next;
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
+      AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
+      if (timer) {
+        AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
+        AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
+      }
+      ++launches;
+      if (t > 0) std::swap(best_cur, best_next);
+    }
+    if (iters > 0) {
+      const int last = (iters - 1) & 1;
+      FinalizeBestArgs f;
+      f.part = part[last];
+      f.nparts = static_cast<int>(P.nparts_upd);
+      f.out = out;
+      f.in = in;
+      f.G = static_cast<int>(P.G);
+      f.inv_batch = 1.0f / static_cast<float>(B);
+      f.keep_best = p->keep_best != 0;
+      f.best_in = best_cur;
+      f.best_out = best_next;
+      f.rowloss = rowloss + static_cast<int64_t>(iters - 1) * out;
+      f.V_last = Vb[last];
+      f.alpha_last = ab[last];
+      f.beta_last = bb[last];
+      f.V_best = V_best;
+      f.alpha_best = alpha_best;
+      f.beta_best = beta_best;
+      AR_CUDA_TRY(launch_finalize_best(f, st));
+      ++launches;
+      std::swap(best_cur, best_next);
+      live = iters & 1;
+    }
+  } else if (iters > 0) {
+    // ---------------------------------------------------------- direct form
+    __nv_bfloat16* Rh = H(L.Rt_hi);
+    __nv_bfloat16* Rl = H(L.Rt_lo);
+    GemmMaps mr{}, mu{};
+    AR_CUDA_TRY(make_tmap_bf16(&mr.a0, D_hi, out, in, kBM));
+    AR_CUDA_TRY(make_tmap_bf16(&mr.a1, D_lo, out, in, kBM));
+    AR_CUDA_TRY(make_tmap_bf16(&mr.b0, X, n_rows, in, P.bn_res));
+    mr.b1 = mr.b0;
+    AR_CUDA_TRY(make_tmap_bf16(&mu.a0, Rh, out, B, kBM));
+    AR_CUDA_TRY(make_tmap_bf16(&mu.a1, Rl, out, B, kBM));
+    AR_CUDA_TRY(make_tmap_bf16(&mu.b0, Xt, in, n_rows, P.bn_upd));
+    mu.b1 = mu.b0;
+
+    GemmArgs r;  // residual: R^T = D X_b^T, (D_hi + D_lo) X_b^T
+    fill_grid(r, out, B, in, P.bn_res, nseg_d);
+    r.seg_a[1] = 1;
+    r.timeout_ns = timeout_ns;
+    r.status = status;
+    r.C_hi = Rh;
+    r.C_lo = P.split ? Rl : nullptr;
+    r.ldc = B;
+    r.part = part[0];
+    r.part_ld = static_cast<int>(P.nparts_res);
+
+    fill_grid(u, out, in, B, P.bn_upd, nseg_d);  // update: G = (R_hi + R_lo)^T X_b
+    u.seg_a[1] = 1;
+    u.V_in = Vb[0];
+    u.V_out = Vb[0];
+    u.alpha_in = ab[0];
+    u.alpha_out = ab[0];
+    u.beta_in = bb[0];
+    u.beta_out = bb[0];
+    u.part_in = part[0];
+    u.nparts = static_cast<int>(P.nparts_res);
+    u.snap_prev = 0;
+    u.part_out = nullptr;
+    for (int t = 0; t < iters; ++t) {
+      const int64_t b0 = sched[t] * B;
+      r.b_row_off = static_cast<int>(b0);
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
+      AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
+      u.b_k_off = static_cast<int>(b0);
+      u.best_in = best_cur;
+      u.best_out = best_next;
+      u.rowloss = rowloss + static_cast<int64_t>(t) * out;
+      AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, mu, u, sms, st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
+      launches += 2;
+      std::swap(best_cur, best_next);
+    }
+  }
+
+  if (iters > 0) {
+    if (p->keep_best && best_cur != best_loss)
+      AR_CUDA_TRY(cudaMemcpyAsync(best_loss, best_cur, static_cast<size_t>(out) * 4, cudaMemcpyDeviceToDevice, st));
+    if (live != 0) {  // hand the live state back in buffer 0
+      AR_CUDA_TRY(cudaMemcpyAsync(Vb[0], Vb[live], elems * 4, cudaMemcpyDeviceToDevice, st));
+      AR_CUDA_TRY(cudaMemcpyAsync(ab[0], ab[live], groups * 4, cudaMemcpyDeviceToDevice, st));
+      AR_CUDA_TRY(cudaMemcpyAsync(bb[0], bb[live], groups * 4, cudaMemcpyDeviceToDevice, st));
+    }
+    if (loss_trace) {
+      AR_CUDA_TRY(launch_loss_trace(rowloss, out, iters, B, loss_trace, st));
+      ++launches;
+    }
+  }
+
+  // Codes, scales and zero-points of the applied state, and its D for the MSE.
+  GroupQuantArgs fin;
+  fin.W = W;
+  fin.w_bf16 = w_dtype == AR_BF16;
+  fin.out = out;
+  fin.in = in;
+  fin.g = static_cast<int>(P.g);
+  fin.G = static_cast<int>(P.G);
+  fin.bits = p->bits;
+  fin.sym = p->sym != 0;
+  fin.wmin_in = wmin;
+  fin.wmax_in = wmax;
+  fin.V = p->keep_best ? V_best : Vb[0];
+  fin.alpha = p->keep_best ? alpha_best : ab[0];
+  fin.beta = p->keep_best ? beta_best : bb[0];
+  fin.codes = codes;
+  fin.scale = scale;
+  fin.zp = zp;
+  fin.D_hi = final_mse ? D_hi : nullptr;
+  fin.D_lo = final_mse && P.split ? D_lo : nullptr;
+  AR_CUDA_TRY(launch_group_quant(fin, st));
+  ++launches;
+
+  if (final_mse) {
+    GemmMaps m{};
+    GemmArgs f;
+    f.timeout_ns = timeout_ns;
+    f.status = status;
+    f.part = part[0];
+    if (gram) {
+      // sum_j D_j (sum_b H_b) D_j^T over all calibration rows
+      AR_CUDA_TRY(launch_gram_sum(H(L.H_hi), P.split ? H(L.H_lo) : nullptr, static_cast<int>(P.nb),
+                                  in * in, H(L.Hs_hi), P.split ? H(L.Hs_lo) : nullptr, st));
+      AR_CUDA_TRY(launch_diag_sum(F(L.Hdiag), static_cast<int>(P.nb), in, F(L.Hdsum), st));
+      launches += 1;
+      AR_CUDA_TRY(make_tmap_bf16(&m.a0, D_hi, out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m.a1, D_lo, out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m.b0, H(L.Hs_hi), in, in, P.bn_fin));
+      AR_CUDA_TRY(make_tmap_bf16(&m.b1, H(L.Hs_lo), in, in, P.bn_fin));
+      fill_grid(f, out, in, in, P.bn_fin, nseg_g);
+      f.seg_a[1] = 1;
+      f.seg_b[2] = 1;
+      f.Dd_hi = D_hi;
+      f.Dd_lo = P.split ? D_lo : nullptr;
+      f.diag_in = F(L.Hdsum);
+      f.part_ld = f.num_n_blk;
+      AR_CUDA_TRY(launch_gemm(kEpiDotD, P.bn_fin, m, f, sms, st));
+      launches += 2;
+    } else {
+      AR_CUDA_TRY(make_tmap_bf16(&m.a0, D_hi, out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m.a1, D_lo, out, in, kBM));
+      AR_CUDA_TRY(make_tmap_bf16(&m.b0, X, n_rows, in, P.bn_fin));
+      m.b1 = m.b0;
+      fill_grid(f, out, n_rows, in, P.bn_fin, nseg_d);
+      f.seg_a[1] = 1;
+      f.part_ld = f.num_n_blk;
+      AR_CUDA_TRY(launch_gemm(kEpiSumSq, P.bn_fin, m, f, sms, st));
+      ++launches;
+    }
+    AR_CUDA_TRY(launch_sum_to_double(part[0], out * f.part_ld, static_cast<double>(n_rows) * out, final_mse, st));
+    ++launches;
+  }
+  if (timer) {
+    AR_CUDA_TRY(cudaEventRecord(timer->stop, st));
+    timer->launches = launches;
+  }
   return AR_OK;
 }
 
@@ -179,7 +665,7 @@ using namespace ar;
 
 extern "C" {
 
-const char* ar_version(void) { return "ar 0.1.0 sm_100a"; }
+const char* ar_version(void) { return "ar 0.2.0 sm_100a"; }
 
 const char* ar_status_string(ar_status s) {
   switch (s) {
@@ -243,270 +729,8 @@ ar_status ar_pack(const uint8_t* codes, int64_t rows, int64_t cols, int32_t bits
 size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, const ar_tune_params* p) {
   if (check_tune_args(out, in, n_rows, p) != AR_OK) return 0;
   if (out == 0 || in == 0) return 256;
-  const int64_t g = group_of(in, p->group_size);
-  return make_layout(out, in, n_rows, p->batch_rows, in / g, p->iters).total;
+  return make_layout(make_plan(out, in, n_rows, p)).total;
 }
-
-}  // extern "C"
-
-namespace ar {
-namespace {
-
-// Events around the contractions of a timed call: ev[2t] before the residual
-// GEMM of step t, ev[2t+1] between the two GEMMs, ev[2t+2] after the update GEMM.
-struct EventTimer {
-  std::vector<cudaEvent_t> ev;
-  cudaEvent_t start = nullptr, stop = nullptr;
-  int launches = 0;
-  bool create(int iters) {
-    ev.assign(static_cast<size_t>(2 * iters + 1), nullptr);
-    for (auto& e : ev)
-      if (cudaEventCreate(&e) != cudaSuccess) return false;
-    return cudaEventCreate(&start) == cudaSuccess && cudaEventCreate(&stop) == cudaSuccess;
-  }
-  ~EventTimer() {
-    for (auto e : ev)
-      if (e) cudaEventDestroy(e);
-    if (start) cudaEventDestroy(start);
-    if (stop) cudaEventDestroy(stop);
-  }
-};
-
-ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X, int64_t n_rows,
-                    const ar_tune_params* p, ar_tune_state* state, void* workspace, size_t ws_bytes,
-                    uint8_t* codes, float* scale, int32_t* zp, float* loss_trace, double* final_mse,
-                    void* stream, EventTimer* timer) {
-  const ar_status chk = check_tune_args(out, in, n_rows, p);
-  if (chk != AR_OK) return chk;
-  if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
-  if (out == 0 || in == 0) return AR_OK;
-  if (!W || !X || !workspace || !codes || !scale || !zp) return AR_EINVAL;
-  if (!aligned(W, 16) || !aligned(X, 16) || !aligned(workspace, 256)) return AR_EINVAL;
-  if (state) {
-    const void* ptrs[7] = {state->V, state->alpha, state->beta, state->best_loss,
-                           state->V_best, state->alpha_best, state->beta_best};
-    for (const void* q : ptrs)
-      if (!q || !aligned(q, 16)) return AR_EINVAL;
-  }
-
-  const int64_t B = p->batch_rows;
-  const int64_t g = group_of(in, p->group_size);
-  const int64_t G = in / g;
-  const int iters = p->iters;
-  const Layout L = make_layout(out, in, n_rows, B, G, iters);
-  if (ws_bytes < L.total) return AR_ENOMEM;
-
-  int dev = 0, sms = 0, major = 0;
-  AR_CUDA_TRY(cudaGetDevice(&dev));
-  AR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  AR_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
-  if (major != 10) return AR_EUNSUPPORTED;
-
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int* status = reinterpret_cast<int*>(ws + L.status);
-  uint16_t* Xt = reinterpret_cast<uint16_t*>(ws + L.Xt);
-  __nv_bfloat16* Rt = reinterpret_cast<__nv_bfloat16*>(ws + L.Rt);
-  __nv_bfloat16* D = reinterpret_cast<__nv_bfloat16*>(ws + L.D);
-  float* wmin = reinterpret_cast<float*>(ws + L.wmin);
-  float* wmax = reinterpret_cast<float*>(ws + L.wmax);
-  float* part = reinterpret_cast<float*>(ws + L.part);
-  float* rowloss = reinterpret_cast<float*>(ws + L.rowloss);
-  float* best_alt = reinterpret_cast<float*>(ws + L.best_alt);
-  float *V, *alpha, *beta, *best_loss, *V_best, *alpha_best, *beta_best;
-  if (state) {
-    V = state->V;
-    alpha = state->alpha;
-    beta = state->beta;
-    best_loss = state->best_loss;
-    V_best = state->V_best;
-    alpha_best = state->alpha_best;
-    beta_best = state->beta_best;
-  } else {
-    V = reinterpret_cast<float*>(ws + L.V);
-    alpha = reinterpret_cast<float*>(ws + L.alpha);
-    beta = reinterpret_cast<float*>(ws + L.beta);
-    best_loss = reinterpret_cast<float*>(ws + L.best_loss);
-    V_best = reinterpret_cast<float*>(ws + L.V_best);
-    alpha_best = reinterpret_cast<float*>(ws + L.alpha_best);
-    beta_best = reinterpret_cast<float*>(ws + L.beta_best);
-  }
-  const bool init_state = !state || !state->initialized;
-  const size_t elems = static_cast<size_t>(out) * in;
-  const size_t groups = static_cast<size_t>(out) * G;
-
-  int launches = 0;
-  if (timer) AR_CUDA_TRY(cudaEventRecord(timer->start, st));
-  AR_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
-  if (init_state) {
-    AR_CUDA_TRY(cudaMemsetAsync(V, 0, elems * 4, st));
-    AR_CUDA_TRY(cudaMemsetAsync(V_best, 0, elems * 4, st));
-    AR_CUDA_TRY(launch_fill_f32(alpha, groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(beta, groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(alpha_best, groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(beta_best, groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(best_loss, out, INFINITY, st));
-    launches += 5;
-  }
-
-  // Group statistics of W and the first step's D = bf16(W' - W).
-  GroupQuantArgs prep;
-  prep.W = W;
-  prep.w_bf16 = w_dtype == AR_BF16;
-  prep.out = out;
-  prep.in = in;
-  prep.g = static_cast<int>(g);
-  prep.G = static_cast<int>(G);
-  prep.bits = p->bits;
-  prep.sym = p->sym != 0;
-  prep.wmin_out = wmin;
-  prep.wmax_out = wmax;
-  prep.V = V;
-  prep.alpha = alpha;
-  prep.beta = beta;
-  prep.D = D;
-  AR_CUDA_TRY(launch_group_quant(prep, st));
-  ++launches;
-
-  const uint64_t timeout_ns = 1000000000ull;
-  const float mlr = p->minmax_lr < 0.0f ? p->lr : p->minmax_lr;
-  const int64_t nparts = cdiv(B, kBN);
-
-  if (iters > 0) {
-    AR_CUDA_TRY(launch_transpose_bf16(X, n_rows, in, Xt, st));
-    ++launches;
-    CUtensorMap tmD, tmX, tmRt, tmXt;
-    AR_CUDA_TRY(make_tmap_bf16(&tmD, D, out, in, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&tmX, X, n_rows, in, kBN));
-    AR_CUDA_TRY(make_tmap_bf16(&tmRt, Rt, out, B, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&tmXt, Xt, in, n_rows, kBN));
-
-    GemmArgs r;  // residual: R^T = D X_b^T
-    r.M = static_cast<int>(out);
-    r.N = static_cast<int>(B);
-    r.K = static_cast<int>(in);
-    r.num_m_blk = static_cast<int>(cdiv(out, kBM));
-    r.num_n_blk = static_cast<int>(cdiv(B, kBN));
-    r.num_k_blk = static_cast<int>(cdiv(in, kBK));
-    r.num_tiles = r.num_m_blk * r.num_n_blk;
-    r.timeout_ns = timeout_ns;
-    r.status = status;
-    r.Rt = Rt;
-    r.ldr = B;
-    r.part = part;
-    r.part_ld = static_cast<int>(nparts);
-
-    GemmArgs u;  // update: G = R^T X_b
-    u.M = static_cast<int>(out);
-    u.N = static_cast<int>(in);
-    u.K = static_cast<int>(B);
-    u.num_m_blk = static_cast<int>(cdiv(out, kBM));
-    u.num_n_blk = static_cast<int>(cdiv(in, kBN));
-    u.num_k_blk = static_cast<int>(cdiv(B, kBK));
-    u.num_tiles = u.num_m_blk * u.num_n_blk;
-    u.timeout_ns = timeout_ns;
-    u.status = status;
-    u.W = W;
-    u.w_bf16 = w_dtype == AR_BF16;
-    u.V = V;
-    u.alpha = alpha;
-    u.beta = beta;
-    u.wmin = wmin;
-    u.wmax = wmax;
-    u.D = D;
-    u.V_best = V_best;
-    u.alpha_best = alpha_best;
-    u.beta_best = beta_best;
-    u.part_in = part;
-    u.nparts = static_cast<int>(nparts);
-    u.inv_batch = 1.0f / static_cast<float>(B);
-    u.g = static_cast<int>(g);
-    u.G = static_cast<int>(G);
-    u.bits = p->bits;
-    u.sym = p->sym != 0;
-    u.keep_best = p->keep_best != 0;
-    u.lr = p->lr;
-    u.mlr = mlr;
-
-    const std::vector<int64_t> sched = block_schedule(n_rows / B, p->start_step, iters, p->seed);
-    float* best_cur = best_loss;
-    float* best_next = best_alt;
-    for (int t = 0; t < iters; ++t) {
-      const int64_t b0 = sched[t] * B;
-      r.b_row_off = static_cast<int>(b0);
-      if (timer && t == 0) AR_CUDA_TRY(cudaEventRecord(timer->ev[0], st));
-      AR_CUDA_TRY(launch_gemm(kEpiResidual, tmD, tmX, r, sms, st));
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
-      u.b_k_off = static_cast<int>(b0);
-      u.best_in = best_cur;
-      u.best_out = best_next;
-      u.rowloss = rowloss + static_cast<int64_t>(t) * out;
-      AR_CUDA_TRY(launch_gemm(kEpiUpdate, tmRt, tmXt, u, sms, st));
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
-      launches += 2;
-      std::swap(best_cur, best_next);
-    }
-    if (p->keep_best && best_cur != best_loss)
-      AR_CUDA_TRY(cudaMemcpyAsync(best_loss, best_cur, static_cast<size_t>(out) * 4, cudaMemcpyDeviceToDevice, st));
-    if (loss_trace) {
-      AR_CUDA_TRY(launch_loss_trace(rowloss, out, iters, B, loss_trace, st));
-      ++launches;
-    }
-  }
-
-  // Codes, scales and zero-points of the applied state, and its D for the MSE.
-  GroupQuantArgs fin;
-  fin.W = W;
-  fin.w_bf16 = w_dtype == AR_BF16;
-  fin.out = out;
-  fin.in = in;
-  fin.g = static_cast<int>(g);
-  fin.G = static_cast<int>(G);
-  fin.bits = p->bits;
-  fin.sym = p->sym != 0;
-  fin.wmin_in = wmin;
-  fin.wmax_in = wmax;
-  fin.V = p->keep_best ? V_best : V;
-  fin.alpha = p->keep_best ? alpha_best : alpha;
-  fin.beta = p->keep_best ? beta_best : beta;
-  fin.codes = codes;
-  fin.scale = scale;
-  fin.zp = zp;
-  fin.D = final_mse ? D : nullptr;
-  AR_CUDA_TRY(launch_group_quant(fin, st));
-  ++launches;
-
-  if (final_mse) {
-    CUtensorMap tmD, tmX;
-    AR_CUDA_TRY(make_tmap_bf16(&tmD, D, out, in, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&tmX, X, n_rows, in, kBN));
-    GemmArgs f;
-    f.M = static_cast<int>(out);
-    f.N = static_cast<int>(n_rows);
-    f.K = static_cast<int>(in);
-    f.num_m_blk = static_cast<int>(cdiv(out, kBM));
-    f.num_n_blk = static_cast<int>(cdiv(n_rows, kBN));
-    f.num_k_blk = static_cast<int>(cdiv(in, kBK));
-    f.num_tiles = f.num_m_blk * f.num_n_blk;
-    f.timeout_ns = timeout_ns;
-    f.status = status;
-    f.part = part;
-    f.part_ld = f.num_n_blk;
-    AR_CUDA_TRY(launch_gemm(kEpiLoss, tmD, tmX, f, sms, st));
-    AR_CUDA_TRY(launch_sum_to_double(part, out * f.num_n_blk, static_cast<double>(n_rows) * out, final_mse, st));
-    launches += 2;
-  }
-  if (timer) {
-    AR_CUDA_TRY(cudaEventRecord(timer->stop, st));
-    timer->launches = launches;
-  }
-  return AR_OK;
-}
-
-}  // namespace
-}  // namespace ar
-
-extern "C" {
 
 ar_status ar_tune_layer(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
                         int64_t n_rows, const ar_tune_params* p, ar_tune_state* state, void* workspace,
@@ -534,14 +758,20 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
   float ms = 0.f;
   for (int t = 0; t < p->iters; ++t) {
     if (cudaEventElapsedTime(&ms, timer.ev[2 * t], timer.ev[2 * t + 1]) != cudaSuccess) return AR_ECUDA;
-    timing->residual_ms += ms;
+    if (timer.algo == AR_ALGO_DIRECT) timing->residual_ms += ms;
+    else timing->update_ms += ms;
     if (cudaEventElapsedTime(&ms, timer.ev[2 * t + 1], timer.ev[2 * t + 2]) != cudaSuccess) return AR_ECUDA;
     timing->update_ms += ms;
+  }
+  if (p->iters > 0) {
+    if (cudaEventElapsedTime(&ms, timer.start, timer.ev[0]) != cudaSuccess) return AR_ECUDA;
+    timing->setup_ms = ms;
   }
   if (cudaEventElapsedTime(&ms, timer.start, timer.stop) != cudaSuccess) return AR_ECUDA;
   timing->total_ms = ms;
   timing->gemm_launches = p->iters;
   timing->kernel_launches = timer.launches;
+  timing->algo = timer.algo;
   return AR_OK;
 }
 

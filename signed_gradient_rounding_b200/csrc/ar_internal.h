@@ -27,7 +27,8 @@ struct GroupQuantArgs {
   float* scale = nullptr;          // [out, G]
   int32_t* zp = nullptr;           // [out, G]
   float* Wq = nullptr;             // [out, in] fp32 s*(q - zp)
-  __nv_bfloat16* D = nullptr;      // [out, in] bf16(s*(q - zp) - W)
+  __nv_bfloat16* D_hi = nullptr;   // [out, in] D = s*(q - zp) - W as hi = bf16(D) ...
+  __nv_bfloat16* D_lo = nullptr;   // ... and lo = bf16(D - hi) (may be null)
 };
 
 cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream);
@@ -44,60 +45,116 @@ cudaError_t launch_sum_to_double(const float* parts, int64_t count, double denom
                                  cudaStream_t stream);
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t stream);
 
+// Keep-best check of the last step of a Gram-form run (its loss is complete only
+// after the step's launch): per row j, L = sum of part[j, 0 .. nparts) in order,
+// rowloss[j] = L; if keep_best and L/B < best_in[j], snapshot the state rows.
+struct FinalizeBestArgs {
+  const float* part = nullptr;
+  int nparts = 0;
+  int64_t out = 0, in = 0;
+  int G = 0;
+  float inv_batch = 1.f;
+  int keep_best = 1;
+  const float* best_in = nullptr;
+  float* best_out = nullptr;
+  float* rowloss = nullptr;
+  const float* V_last = nullptr;
+  const float* alpha_last = nullptr;
+  const float* beta_last = nullptr;
+  float* V_best = nullptr;
+  float* alpha_best = nullptr;
+  float* beta_best = nullptr;
+};
+cudaError_t launch_finalize_best(const FinalizeBestArgs& a, cudaStream_t stream);
+
+// Hs = sum over nb blocks of (H_hi[b] + H_lo[b]) in fp32, returned as a bf16 pair,
+// and dsum[k] = sum over blocks of diag[b*in + k] (the exact diagonals).
+cudaError_t launch_gram_sum(const __nv_bfloat16* H_hi, const __nv_bfloat16* H_lo, int nb, int64_t count,
+                            __nv_bfloat16* Hs_hi, __nv_bfloat16* Hs_lo, cudaStream_t stream);
+cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream);
+
 // ---------------------------------------------------------------------------
-// Persistent tcgen05 GEMM, C[M, N] = A[M, K] * B[N, K]^T, both operands K-major
-// bf16 loaded by TMA, fp32 accumulators in tensor memory, fused epilogues.
+// Persistent tcgen05 GEMM: C[M, N] = sum over K segments of A_s[M, K] B_s[N, K]^T,
+// operands bf16 K-major loaded by TMA, fp32 accumulators in tensor memory, fused
+// epilogues (see gemm_sm100.cu).
 // ---------------------------------------------------------------------------
 
 enum EpiKind : int {
-  kEpiResidual = 0,  // C = R^T tile of one step: store bf16, per-(row, n-tile) sums of R^2
-  kEpiUpdate = 1,    // C = G tile: straight-through sign updates of V, alpha, beta; next D
-  kEpiLoss = 2       // C = R^T tile: per-(row, n-tile) sums of R^2 only
+  kEpiStore = 0,   // C as a bf16 (hi, lo) pair; optional per-(row, n-tile) sums of C^2
+  kEpiSumSq = 1,   // per-(row, n-tile) sums of C^2
+  kEpiUpdate = 2,  // C = G: the SignSGD step (sign updates, keep-best, next D, Gram-form loss)
+  kEpiDotD = 3     // per-(row, n-tile) sums of D * C
+};
+
+// Operand maps: segment s reads A from a{seg_a[s]} and B from b{seg_b[s]}.
+struct GemmMaps {
+  CUtensorMap a0, a1, b0, b1;
 };
 
 struct GemmArgs {
-  int M = 0, N = 0, K = 0;
+  int M = 0, N = 0, K = 0;  // K: per segment
   int num_m_blk = 0, num_n_blk = 0, num_k_blk = 0, num_tiles = 0;
-  int b_row_off = 0;  // added to B's row coordinate (first calibration row of the block)
+  int num_seg = 1;
+  int seg_a[3] = {0, 0, 0};
+  int seg_b[3] = {0, 0, 0};
+  int a_k_off = 0;    // added to A's K coordinate
+  int b_row_off = 0;  // added to B's row coordinate
   int b_k_off = 0;    // added to B's K coordinate
   uint64_t timeout_ns = 1000000000ull;
   int* status = nullptr;
 
-  // kEpiResidual / kEpiLoss
-  __nv_bfloat16* Rt = nullptr;  // [M, ldr]
-  int64_t ldr = 0;
-  float* part = nullptr;        // [M, part_ld] row sums of R^2 per n-tile
+  // kEpiStore: C rows j go to row c_row_off + j of [*, ldc]
+  __nv_bfloat16* C_hi = nullptr;
+  __nv_bfloat16* C_lo = nullptr;  // may be null
+  int64_t ldc = 0;
+  int64_t c_row_off = 0;
+  // kEpiStore / kEpiSumSq / kEpiDotD / kEpiUpdate (Gram loss): per-(row, n-tile) sums
+  float* part = nullptr;  // [M, part_ld] (kEpiUpdate: part_out)
   int part_ld = 0;
+  // kEpiStore: when set, the diagonal (column == row j) is written here in fp32,
+  // at [c_row_off + j], and stored as 0 in the bf16 pair
+  float* diag_out = nullptr;
+  // kEpiUpdate / kEpiDotD: when set, C_jk += D_jk * diag_in[k] in fp32 (the exact
+  // diagonal of a Gram matrix whose bf16 pair holds only the off-diagonal part)
+  const float* diag_in = nullptr;
+  // kEpiDotD
+  const __nv_bfloat16* Dd_hi = nullptr;  // [M, N]
+  const __nv_bfloat16* Dd_lo = nullptr;
 
   // kEpiUpdate
   const void* W = nullptr;
   int w_bf16 = 0;
-  float* V = nullptr;
-  float* alpha = nullptr;
-  float* beta = nullptr;
+  const float* V_in = nullptr;   // state of this step
+  float* V_out = nullptr;        // state of the next step (== V_in: in place)
+  const float* alpha_in = nullptr;
+  float* alpha_out = nullptr;
+  const float* beta_in = nullptr;
+  float* beta_out = nullptr;
   const float* wmin = nullptr;
   const float* wmax = nullptr;
-  __nv_bfloat16* D = nullptr;
+  __nv_bfloat16* D_hi = nullptr;  // next step's W' - W
+  __nv_bfloat16* D_lo = nullptr;  // may be null (single bf16)
   float* V_best = nullptr;
   float* alpha_best = nullptr;
   float* beta_best = nullptr;
-  const float* best_in = nullptr;   // [M] best loss before this step
-  float* best_out = nullptr;        // [M] best loss after this step
-  float* rowloss = nullptr;         // [M] this step's per-row sum of R^2
-  const float* part_in = nullptr;   // [M, nparts] from the residual GEMM
+  const float* best_in = nullptr;  // [M] best mean loss so far
+  float* best_out = nullptr;       // [M]
+  float* rowloss = nullptr;        // [M] sum of R^2 of the judged step
+  const float* part_in = nullptr;  // [M, nparts] partials of the judged step (null: none)
   int nparts = 0;
+  int snap_prev = 0;      // 0: judge this step (snapshot V_in); 1: judge the previous one (snapshot V_out)
+  float* part_out = nullptr;  // [M, part_ld] this step's sum_k D G partials (Gram form), or null
   float inv_batch = 1.0f;
   int g = 0, G = 0, bits = 4, sym = 0, keep_best = 1;
   float lr = 0.f, mlr = 0.f;
 };
 
-// Tile sizes of the GEMM.
+// Tile sizes: M and K tiles fixed, N tile 128 or 256 per launch.
 constexpr int kBM = 128;
-constexpr int kBN = 256;
 constexpr int kBK = 64;
 
-cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                        int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
+                        cudaStream_t stream);
 
 // TMA descriptor for a row-major bf16 matrix [rows, cols], box [box_rows, 64]
 // with 128-byte swizzle; zero fill outside the matrix.

@@ -1,33 +1,40 @@
 // Persistent warp-specialised bf16 GEMM for sm_100a with fused epilogues.
 //
-//   C[M, N] = A[M, K] * B[N, K]^T      (A, B bf16 K-major; C fp32 in tensor memory)
+//   C[M, N] = sum over segments s of  A_s[M, K] * B_s[N, K]^T
+//
+// A and B are bf16, K-major, loaded by TMA; C is fp32 in tensor memory.  A
+// "segment" is one pass over K with its own pair of operand maps, so an operand
+// kept as an exact bf16 pair x = hi + lo (hi = bf16(x), lo = bf16(x - hi), about
+// 16 significant bits) is multiplied as extra segments of the same accumulation:
+// (hi_a + lo_a)(hi_b + lo_b) ~ hi_a hi_b + lo_a hi_b + hi_a lo_b.
 //
 // Roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: 128x64 A tile + 256x64 B tile per stage, 4 stages,
-//               128-byte swizzle, completion counted on the stage's mbarrier.
-//   warp 1      MMA issuer: four tcgen05.mma (M=128, N=256, K=16) per stage into
-//               one of two 256-column fp32 accumulators in tensor memory;
-//               tcgen05.commit frees the stage and, after the last K block,
-//               hands the accumulator to the epilogue.
-//   warps 2..5  epilogue: each thread owns one accumulator row (its warp's
-//               32-lane slice of tensor memory) and walks the tile's 256 columns
-//               32 at a time with tcgen05.ld, while the MMA warp fills the other
-//               accumulator with the next tile.
+//   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage, 128-byte
+//               swizzle, completion counted on the stage's mbarrier.
+//   warp 1      MMA issuer: four tcgen05.mma (M=128, N=BN, K=16) per stage into one
+//               of two BN-column fp32 accumulators in tensor memory;
+//               tcgen05.commit frees the stage and, after the last K block, hands
+//               the accumulator to the epilogue.
+//   warps 2..5  epilogue: each thread owns one accumulator row (its warp's 32-lane
+//               slice of tensor memory) and walks the tile's columns 32 at a time
+//               with tcgen05.ld, while the MMA warp fills the other accumulator.
 //
-// Epilogues (the two contractions of one SignSGD step of the AutoRound loop,
+// Epilogues (the contractions of the AutoRound SignSGD loop,
 // "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END"):
-//   kEpiResidual  A = D = bf16(W' - W) [out, in], B = X_b [B, in]: C = R^T = (Y' - Y)^T.
-//                 Stores R^T in bf16 and per-(row, n-tile) sums of R^2.
-//   kEpiUpdate    A = R^T [out, B], B = X_b^T [in, B]: C = G = R^T X_b = dL/dW' * B*out/2.
-//                 Straight-through sign updates of V (per element) and of alpha,
-//                 beta (per group: a group lies inside one thread's 256 columns),
-//                 the per-row keep-best snapshot, and the next step's D, so the
-//                 gradient never goes to memory.
-//   kEpiLoss      as kEpiResidual without storing R (final MSE over all rows).
+//   kEpiStore   C as a bf16 pair (hi, lo) into [rows, ldc], optionally with the row
+//               sums of C^2 per n-tile: the residual R^T = D X_b^T of one step, or a
+//               calibration block's Gram matrix H_b = X_b^T X_b.
+//   kEpiSumSq   row sums of C^2 per n-tile only (final MSE over all rows).
+//   kEpiUpdate  C = G = dL/dW' up to a positive factor: straight-through sign
+//               updates of V (per element) and of alpha, beta (per group: a group
+//               lies inside one thread's columns), the per-row keep-best snapshot,
+//               the next step's D = W' - W as a bf16 pair, and (Gram form) the row
+//               loss sum_k D_jk G_jk -- the gradient never reaches memory.
+//   kEpiDotD    row sums of D * C per n-tile (the Gram form of the final MSE).
 //
 // Every mbarrier wait is bounded (GemmArgs::timeout_ns); a role that gives up
-// records the timeout in *status and the CTA drains its in-flight copies and
-// MMAs before it frees tensor memory and exits.
+// records the timeout in *status and the CTA drains its in-flight copies and MMAs
+// before it frees tensor memory and exits.
 #include "ar_device.cuh"
 #include "ar_internal.h"
 
@@ -35,19 +42,23 @@ namespace ar {
 
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kThreads = 192;
-constexpr int kTileABytes = kBM * kBK * 2;   // 16 KB
-constexpr int kTileBBytes = kBN * kBK * 2;   // 32 KB
-constexpr int kStageBytes = kTileABytes + kTileBBytes;
-constexpr int kTmemCols = 2 * kBN;           // two accumulators
-constexpr int kBarOffset = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOffset + 1024 /* barriers etc. */ + 1024 /* alignment slack */;
-constexpr uint32_t kIdesc = umma_idesc_bf16(kBM, kBN);
+constexpr int kTileABytes = kBM * kBK * 2;  // 16 KB
+
+template <int kBN>
+struct Cfg {
+  static constexpr int kTileBBytes = kBN * kBK * 2;
+  static constexpr int kStageBytes = kTileABytes + kTileBBytes;
+  static constexpr int kStages = (kBN == 256) ? 4 : 6;
+  static constexpr int kTmemCols = 2 * kBN;
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;
+  static constexpr uint32_t kIdesc = umma_idesc_bf16(kBM, kBN);
+};
 
 struct Smem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[8];
+  uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -83,6 +94,11 @@ __device__ __forceinline__ void load_w32(const void* W, int w_bf16, int64_t idx,
   }
 }
 
+// 32 consecutive bf16 values as fp32.
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&v)[32]) {
+  load_w32(p, 1, 0, v);
+}
+
 __device__ __forceinline__ void load_f32x32(const float* p, float (&v)[32]) {
   const float4* q4 = reinterpret_cast<const float4*>(p);
 #pragma unroll
@@ -106,14 +122,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi) (x - hi is exact in fp32).
+__device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
+  hi = __bfloat162float(__float2bfloat16_rn(x));
+  lo = __fsub_rn(x, hi);
+}
+
+// Store 8 values (a multiple-of-8 column chunk) as hi and, if wanted, lo bf16.
+__device__ __forceinline__ void store_pair8(const float* x, __nv_bfloat16* hi_dst, __nv_bfloat16* lo_dst) {
+  float h[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) split_bf16(x[i], h[i], l[i]);
+  *reinterpret_cast<uint4*>(hi_dst) =
+      make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+  if (lo_dst)
+    *reinterpret_cast<uint4*>(lo_dst) = make_uint4(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]),
+                                                   pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
+}
+
 // ---------------------------------------------------------------------------
 // epilogues
 // ---------------------------------------------------------------------------
 
-// R^T tile: optional bf16 store, per-row sum of squares over the valid columns.
-template <bool kStore>
-__device__ __forceinline__ void epi_residual(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk) {
-  float sumsq = 0.0f;
+// kEpiStore / kEpiSumSq / kEpiDotD: one pass over the tile's columns.
+template <int kKind, int kBN>
+__device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk) {
+  float acc = 0.0f;
   const bool row_ok = j < a.M;
 #pragma unroll 1
   for (int c = 0; c < kBN / 32; ++c) {
@@ -123,43 +157,68 @@ __device__ __forceinline__ void epi_residual(const GemmArgs& a, uint32_t t_row, 
     __syncwarp();
     tmem_ld_32cols(t_row + c * 32, r);
     tmem_ld_wait();
-    if (row_ok) {
-      const int nvalid = min(32, a.N - col0);
+    if (!row_ok) continue;  // nothing warp-collective follows in this iteration
+    const int nvalid = min(32, a.N - col0);  // a multiple of 8
+    float x[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float v = __uint_as_float(r[i]);
-        if (i < nvalid) sumsq = fmaf(v, v, sumsq);
+    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+    if (kKind == kEpiStore || kKind == kEpiSumSq) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nvalid) acc = fmaf(x[i], x[i], acc);
+    }
+    if (kKind == kEpiDotD) {
+      const int64_t e = static_cast<int64_t>(j) * a.N + col0;
+      float dh[32], dl[32];
+      load_bf16x32(a.Dd_hi + e, dh);
+      if (a.Dd_lo) {
+        load_bf16x32(a.Dd_lo + e, dl);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dh[i] += dl[i];
       }
-      if (kStore) {
-        __nv_bfloat16* dst = a.Rt + static_cast<int64_t>(j) * a.ldr + col0;
+      if (a.diag_in) {
+        float dg[32];
+        load_f32x32(a.diag_in + col0, dg);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (q * 8 < nvalid) {  // nvalid is a multiple of 8
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(r[q * 8 + 0]), __uint_as_float(r[q * 8 + 1]));
-            pk.y = pack_bf16x2(__uint_as_float(r[q * 8 + 2]), __uint_as_float(r[q * 8 + 3]));
-            pk.z = pack_bf16x2(__uint_as_float(r[q * 8 + 4]), __uint_as_float(r[q * 8 + 5]));
-            pk.w = pack_bf16x2(__uint_as_float(r[q * 8 + 6]), __uint_as_float(r[q * 8 + 7]));
-            reinterpret_cast<uint4*>(dst)[q] = pk;
-          }
+        for (int i = 0; i < 32; ++i) x[i] = fmaf(dh[i], dg[i], x[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc = fmaf(dh[i], x[i], acc);
+    }
+    if (kKind == kEpiStore && a.diag_out && j >= col0 && j < col0 + 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i == j) {
+          a.diag_out[a.c_row_off + j] = x[i];
+          x[i] = 0.0f;
         }
-      }
+    }
+    if (kKind == kEpiStore) {
+      const int64_t off = (a.c_row_off + j) * a.ldc + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
     }
   }
-  if (row_ok) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk] = sumsq;
+  if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk] = acc;
 }
 
-// G tile: the SignSGD update of one step for the rows x columns of this tile.
+// kEpiUpdate: one SignSGD step for the rows x columns of this G tile.
+template <int kBN>
 __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk) {
   const bool row_ok = j < a.M;
   const float Q = qmaxf(a.bits);
   const bool sym = a.sym != 0;
   const int64_t row_base = static_cast<int64_t>(j) * a.N;
 
-  // Per-row batch loss of this step (sum over the residual GEMM's n-tiles, fixed
-  // order) and the keep-best decision; identical in every n-tile of the row.
+  // Keep-best: the row's batch loss (sum of the per-n-tile partials in a fixed
+  // order, so every n-tile of the row reaches the same decision) against the best
+  // so far.  Direct form: the loss of this step (computed by the residual GEMM),
+  // snapshot of the state read now.  Gram form: the loss of the previous step
+  // (computed by the previous launch), snapshot of the previous state, which still
+  // sits in the output buffers until this epilogue overwrites it.
   bool better = false;
-  if (row_ok) {
+  if (row_ok && a.part_in) {
     float L = 0.0f;
     const float* p = a.part_in + static_cast<int64_t>(j) * a.nparts;
     for (int q = 0; q < a.nparts; ++q) L += p[q];
@@ -170,9 +229,12 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
     }
     if (n_blk == 0) a.rowloss[j] = L;
   }
+  const bool snap_now = better && !a.snap_prev;
+  const bool snap_old = better && a.snap_prev;
 
-  const int groups_in_tile = max(1, kBN / a.g);  // g divides 256, or g == N <= 256
+  const int groups_in_tile = max(1, kBN / a.g);  // g divides kBN, or g == N <= kBN
   const int chunks_per_group = a.g / 32;
+  float loss_acc = 0.0f;
 #pragma unroll 1
   for (int gl = 0; gl < groups_in_tile; ++gl) {
     const int gcol0 = n0 + gl * a.g;
@@ -183,8 +245,8 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
     if (row_ok) {
       wmn = a.wmin[gidx];
       wmx = a.wmax[gidx];
-      al = a.alpha[gidx];
-      be = a.beta[gidx];
+      al = a.alpha_in[gidx];
+      be = a.beta_in[gidx];
     }
     const GroupScale gs = group_scale(wmn, wmx, al, be, a.bits, sym);
     // Straight-through derivatives of s and zp with respect to alpha and beta.
@@ -211,22 +273,30 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       __syncwarp();
       tmem_ld_32cols(t_row + tcol, r);
       tmem_ld_wait();
-      if (!row_ok) continue;  // no warp-collective instruction follows in this iteration
+      if (!row_ok) continue;  // nothing warp-collective follows in this iteration
       const int64_t e0 = row_base + n0 + tcol;
-      float w[32], v[32], vn[32];
+      float w[32], v[32], vn[32], dg[32];
       load_w32(a.W, a.w_bf16, e0, w);
-      load_f32x32(a.V + e0, v);
+      load_f32x32(a.V_in + e0, v);
+      if (a.diag_in) load_f32x32(a.diag_in + n0 + tcol, dg);
+      if (snap_old) {
+        float vo[32];
+        load_f32x32(a.V_out + e0, vo);
+        store_f32x32(a.V_best + e0, vo);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float G = __uint_as_float(r[i]);
         const ElemQuant e = quant_elem(w[i], v[i], gs, Q);
+        const float d = __fsub_rn(e.wq, w[i]);
+        const float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
+        loss_acc = fmaf(d, G, loss_acc);
         const float sg = e.m ? sgnf(G) : 0.0f;
         vn[i] = fminf(fmaxf(__fsub_rn(v[i], __fmul_rn(a.lr, sg)), -0.5f), 0.5f);
         float dwa, dwb;
         if (e.m) {
-          const float d = e.r - e.u;
-          dwa = ds_a * d;
-          dwb = ds_b * d;
+          const float ru = e.r - e.u;
+          dwa = ds_a * ru;
+          dwb = ds_b * ru;
         } else {
           const float qz = e.q - gs.zp;
           dwa = ds_a * qz - gs.s * dzp_a;
@@ -235,60 +305,62 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
         dal = fmaf(G, dwa, dal);
         dbe = fmaf(G, dwb, dbe);
       }
-      store_f32x32(a.V + e0, vn);
-      if (better) store_f32x32(a.V_best + e0, v);
+      store_f32x32(a.V_out + e0, vn);
+      if (snap_now) store_f32x32(a.V_best + e0, v);
     }
     if (!row_ok) continue;
 
     const float al_n = fminf(fmaxf(__fsub_rn(al, __fmul_rn(a.mlr, sgnf(dal))), 0.5f), 1.0f);
     const float be_n = sym ? be : fminf(fmaxf(__fsub_rn(be, __fmul_rn(a.mlr, sgnf(dbe))), 0.5f), 1.0f);
-    a.alpha[gidx] = al_n;
-    a.beta[gidx] = be_n;
-    if (better) {
+    if (snap_now) {
       a.alpha_best[gidx] = al;
       a.beta_best[gidx] = be;
     }
+    if (snap_old) {
+      a.alpha_best[gidx] = a.alpha_out[gidx];
+      a.beta_best[gidx] = a.beta_out[gidx];
+    }
+    a.alpha_out[gidx] = al_n;
+    a.beta_out[gidx] = be_n;
 
-    // D for the next step from the updated state.
+    // D = W' - W of the next step, from the updated state, as a bf16 pair.
     const GroupScale gn = group_scale(wmn, wmx, al_n, be_n, a.bits, sym);
 #pragma unroll 1
     for (int cc = 0; cc < chunks_per_group; ++cc) {
       const int64_t e0 = row_base + gcol0 + cc * 32;
-      float w[32], v[32];
+      float w[32], v[32], d[32];
       load_w32(a.W, a.w_bf16, e0, w);
-      load_f32x32(a.V + e0, v);
-      uint32_t pk[16];
+      load_f32x32(a.V_out + e0, v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const ElemQuant e0q = quant_elem(w[2 * i], v[2 * i], gn, Q);
-        const ElemQuant e1q = quant_elem(w[2 * i + 1], v[2 * i + 1], gn, Q);
-        pk[i] = pack_bf16x2(__fsub_rn(e0q.wq, w[2 * i]), __fsub_rn(e1q.wq, w[2 * i + 1]));
-      }
-      uint4* dst = reinterpret_cast<uint4*>(a.D + e0);
+      for (int i = 0; i < 32; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q).wq, w[i]);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      for (int q = 0; q < 4; ++q)
+        store_pair8(d + q * 8, a.D_hi + e0 + q * 8, a.D_lo ? a.D_lo + e0 + q * 8 : nullptr);
     }
   }
+  if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk] = loss_acc;
 }
 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
 
-template <int kKind>
+template <int kKind, int kBN>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                 const __grid_constant__ GemmArgs args) {
+  using C = Cfg<kBN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Smem* sm = reinterpret_cast<Smem*>(smem + kBarOffset);
+  Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
   volatile int* abort_flag = &sm->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (warp == 1 && lane == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
     }
@@ -301,17 +373,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&sm->tmem_base, kTmemCols);
+    tmem_alloc(&sm->tmem_base, C::kTmemCols);
     tmem_relinquish();
     if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
+      tma_prefetch_desc(&tmA0);
+      tma_prefetch_desc(&tmB0);
+      if (args.num_seg > 1) {
+        tma_prefetch_desc(&tmA1);
+        tma_prefetch_desc(&tmB1);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm->tmem_base;
+  const int k_blocks = args.num_seg * args.num_k_blk;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -323,19 +400,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
         const int m_blk = tile % args.num_m_blk;
         const int n_blk = tile / args.num_m_blk;
-        for (int kb = 0; kb < args.num_k_blk; ++kb) {
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          const int seg = kb / args.num_k_blk;
+          const int kk = kb - seg * args.num_k_blk;
+          const CUtensorMap* mA = args.seg_a[seg] ? &tmA1 : &tmA0;
+          const CUtensorMap* mB = args.seg_b[seg] ? &tmB1 : &tmB0;
           if (!mbar_wait(&sm->empty[stage], phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
             ok = false;
             break;
           }
-          uint8_t* sA = smem + stage * kStageBytes;
+          uint8_t* sA = smem + stage * C::kStageBytes;
           uint8_t* sB = sA + kTileABytes;
-          mbar_arrive_expect_tx(&sm->full[stage], kStageBytes);
-          tma_load_2d(sA, &tmA, kb * kBK, m_blk * kBM, &sm->full[stage]);
-          tma_load_2d(sB, &tmB, kb * kBK + args.b_k_off, n_blk * kBN + args.b_row_off, &sm->full[stage]);
+          mbar_arrive_expect_tx(&sm->full[stage], C::kStageBytes);
+          tma_load_2d(sA, mA, kk * kBK + args.a_k_off, m_blk * kBM, &sm->full[stage]);
+          tma_load_2d(sB, mB, kk * kBK + args.b_k_off, n_blk * kBN + args.b_row_off, &sm->full[stage]);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
+          if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
@@ -343,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // Let the copies already issued land before the CTA exits.
-        for (int s = 0; s < kStages; ++s)
+        for (int s = 0; s < C::kStages; ++s)
           if (issued_mask & (1u << s)) mbar_wait_drain(&sm->full[s], (issued_parity >> s) & 1u, args.timeout_ns);
       }
     }
@@ -362,20 +443,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
-        for (int kb = 0; kb < args.num_k_blk; ++kb) {
+        for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm->full[stage], phase, abort_flag, args.status, args.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
           const uint64_t a_desc = umma_desc_sw128(a_addr);
           const uint64_t b_desc = umma_desc_sw128(a_addr + kTileABytes);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&sm->empty[stage]);
-          if (++stage == kStages) {
+          if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
@@ -403,9 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       const int j = m_blk * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
-      if (kKind == kEpiResidual) epi_residual<true>(args, t_row, j, n0, n_blk);
-      if (kKind == kEpiLoss) epi_residual<false>(args, t_row, j, n0, n_blk);
-      if (kKind == kEpiUpdate) epi_update(args, t_row, j, n0, n_blk);
+      if (kKind == kEpiUpdate)
+        epi_update<kBN>(args, t_row, j, n0, n_blk);
+      else
+        epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk);
       tc_fence_before();
       mbar_arrive(&sm->tempty[acc]);
       acc ^= 1;
@@ -418,37 +500,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 0) {
     __syncwarp();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int kKind>
-cudaError_t launch_kind(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args, int num_sms,
-                        cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+template <int kKind, int kBN>
+cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
+  using C = Cfg<kBN>;
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kKind, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int grid = args.num_tiles < num_sms ? args.num_tiles : num_sms;
   if (grid <= 0) return cudaSuccess;
-  gemm_kernel<kKind><<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, args);
+  gemm_kernel<kKind, kBN><<<grid, kThreads, C::kSmemBytes, stream>>>(m.a0, m.a1, m.b0, m.b1, args);
   return cudaGetLastError();
+}
+
+template <int kBN>
+cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
+  switch (kind) {
+    case kEpiStore:
+      return launch_kind<kEpiStore, kBN>(m, args, num_sms, stream);
+    case kEpiSumSq:
+      return launch_kind<kEpiSumSq, kBN>(m, args, num_sms, stream);
+    case kEpiUpdate:
+      return launch_kind<kEpiUpdate, kBN>(m, args, num_sms, stream);
+    case kEpiDotD:
+      return launch_kind<kEpiDotD, kBN>(m, args, num_sms, stream);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(EpiKind kind, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                        int num_sms, cudaStream_t stream) {
-  switch (kind) {
-    case kEpiResidual:
-      return launch_kind<kEpiResidual>(tmA, tmB, args, num_sms, stream);
-    case kEpiUpdate:
-      return launch_kind<kEpiUpdate>(tmA, tmB, args, num_sms, stream);
-    case kEpiLoss:
-      return launch_kind<kEpiLoss>(tmA, tmB, args, num_sms, stream);
-  }
+cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
+                        cudaStream_t stream) {
+  if (args.num_seg < 1 || args.num_seg > 3) return cudaErrorInvalidValue;
+  if (bn == 256) return launch_bn<256>(kind, maps, args, num_sms, stream);
+  if (bn == 128) return launch_bn<128>(kind, maps, args, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -56,7 +56,7 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
     if (a.scale) a.scale[warp] = gs.s;
     if (a.zp) a.zp[warp] = static_cast<int32_t>(gs.zp);
   }
-  if (!a.codes && !a.Wq && !a.D) return;
+  if (!a.codes && !a.Wq && !a.D_hi) return;
   const float Q = qmaxf(a.bits);
   for (int k = lane; k < a.g; k += 32) {
     const float w = load_w(a.W, a.w_bf16, base + k);
@@ -64,7 +64,12 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
     const ElemQuant e = quant_elem(w, v, gs, Q);
     if (a.codes) a.codes[base + k] = static_cast<uint8_t>(e.q);
     if (a.Wq) a.Wq[base + k] = e.wq;
-    if (a.D) a.D[base + k] = __float2bfloat16_rn(__fsub_rn(e.wq, w));
+    if (a.D_hi) {
+      const float d = __fsub_rn(e.wq, w);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(d);
+      a.D_hi[base + k] = hi;
+      if (a.D_lo) a.D_lo[base + k] = __float2bfloat16_rn(__fsub_rn(d, __bfloat162float(hi)));
+    }
   }
 }
 
@@ -166,7 +171,78 @@ __global__ void timeout_selftest_kernel(int32_t* status, uint64_t timeout_ns) {
   __syncthreads();
 }
 
+// One warp per row.
+__global__ void finalize_best_kernel(FinalizeBestArgs a) {
+  const int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (j >= a.out) return;
+  float L = 0.0f;
+  const float* p = a.part + j * a.nparts;
+  for (int q = 0; q < a.nparts; ++q) L += p[q];  // same order as the update epilogue
+  bool better = false;
+  if (a.keep_best) {
+    const float mean = L * a.inv_batch;
+    better = mean < a.best_in[j];
+    if (lane == 0) a.best_out[j] = better ? mean : a.best_in[j];
+  }
+  if (lane == 0) a.rowloss[j] = L;
+  if (!better) return;
+  for (int64_t k = lane; k < a.in; k += 32) a.V_best[j * a.in + k] = a.V_last[j * a.in + k];
+  for (int64_t k = lane; k < a.G; k += 32) {
+    a.alpha_best[j * a.G + k] = a.alpha_last[j * a.G + k];
+    a.beta_best[j * a.G + k] = a.beta_last[j * a.G + k];
+  }
+}
+
+__global__ void gram_sum_kernel(const __nv_bfloat16* __restrict__ H_hi, const __nv_bfloat16* __restrict__ H_lo,
+                                int nb, int64_t count, __nv_bfloat16* __restrict__ Hs_hi,
+                                __nv_bfloat16* __restrict__ Hs_lo) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.0f;
+    for (int b = 0; b < nb; ++b) {
+      s += __bfloat162float(H_hi[b * count + i]);
+      if (H_lo) s += __bfloat162float(H_lo[b * count + i]);
+    }
+    const __nv_bfloat16 hi = __float2bfloat16_rn(s);
+    Hs_hi[i] = hi;
+    if (Hs_lo) Hs_lo[i] = __float2bfloat16_rn(s - __bfloat162float(hi));
+  }
+}
+
+__global__ void diag_sum_kernel(const float* __restrict__ diag, int nb, int64_t in, float* __restrict__ dsum) {
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < in;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.0f;
+    for (int b = 0; b < nb; ++b) s += diag[b * in + k];
+    dsum[k] = s;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream) {
+  if (in == 0) return cudaSuccess;
+  diag_sum_kernel<<<static_cast<unsigned>((in + 255) / 256), 256, 0, stream>>>(diag, nb, in, dsum);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_best(const FinalizeBestArgs& a, cudaStream_t stream) {
+  if (a.out == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (a.out * 32 + threads - 1) / threads;
+  finalize_best_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_sum(const __nv_bfloat16* H_hi, const __nv_bfloat16* H_lo, int nb, int64_t count,
+                            __nv_bfloat16* Hs_hi, __nv_bfloat16* Hs_lo, cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  int64_t blocks = (count + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  gram_sum_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(H_hi, H_lo, nb, count, Hs_hi, Hs_lo);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream) {
   const int64_t groups = a.out * a.G;
