@@ -218,6 +218,33 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
 ar_status ar_block_schedule(int64_t n_blocks, int64_t first, int64_t count, uint64_t seed,
                             int64_t* blocks);
 
+/* Size of the fixed device scratch array used by ar_tune_layer_static (64 MiB). */
+#define AR_STATIC_SCRATCH_BYTES (64ull << 20)
+
+/* ar_tune_layer for callers that cannot allocate device memory at call time --
+ * code that runs where cudaMalloc is not allowed or not wanted (inside a region
+ * whose memory is owned by another allocator, or a path that must not trigger the
+ * device synchronisation an allocation can cause).  The pages have no counterpart
+ * of this entry point; it is a property of this library.
+ * Same arguments, results and errors as ar_tune_layer with state = NULL, minus the
+ * workspace: the scratch is one array of AR_STATIC_SCRATCH_BYTES in device memory,
+ * created when the library's device code is loaded on a GPU and held by every GPU
+ * that loads the library until the process exits.  The call makes no device
+ * allocation (no cudaMalloc/cudaFree or other allocator); its host side uses the
+ * C++ heap only for the step schedule.
+ *   AR_ENOMEM: the layer needs more scratch than AR_STATIC_SCRATCH_BYTES
+ *              (ar_tune_workspace_bytes() tells how much it needs); nothing is enqueued.
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * All calls share the one array, and it keeps the last call's contents; every call
+ * initialises what it reads.  Calls that overlap on the device (other streams,
+ * other threads) race on the array: serialise them.  ar_tune_status() is not
+ * available for this entry point (the status word is in the shared array). */
+ar_status ar_tune_layer_static(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
+                               const uint16_t* X, int64_t n_rows, const ar_tune_params* params,
+                               uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
+                               double* final_mse, void* stream);
+
 /* Device status of the last ar_tune_layer call that used `workspace`: synchronises
  * `stream`, then returns AR_OK, or AR_ETIMEOUT if a kernel's bounded wait ran out
  * (its results are then invalid), or AR_ECUDA if the stream reports an error. */

@@ -28,7 +28,7 @@ ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
-           "ar_tune_status", "ar_selftest_timeout")
+           "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static")
 
 
 class ArError(RuntimeError):
@@ -83,6 +83,9 @@ def _load() -> ctypes.CDLL:
     lib.ar_tune_layer_timed.argtypes = lib.ar_tune_layer.argtypes + [ctypes.POINTER(TuneTiming)]
     lib.ar_block_schedule.restype = ctypes.c_int
     lib.ar_block_schedule.argtypes = [I64, I64, I64, U64, P]
+    lib.ar_tune_layer_static.restype = ctypes.c_int
+    lib.ar_tune_layer_static.argtypes = [P, ctypes.c_int, I64, I64, P, I64, ctypes.POINTER(TuneParams),
+                                         P, P, P, P, P, P]
     lib.ar_tune_status.restype = ctypes.c_int
     lib.ar_tune_status.argtypes = [P, P]
     lib.ar_selftest_timeout.restype = ctypes.c_int
@@ -96,6 +99,11 @@ lib = _lib
 
 def version() -> str:
     return _lib.ar_version().decode()
+
+
+def lib_static_scratch_bytes() -> int:
+    """Size of the fixed device scratch of ar_tune_layer_static (AR_STATIC_SCRATCH_BYTES)."""
+    return 64 << 20
 
 
 def _check(status: int, what: str) -> None:

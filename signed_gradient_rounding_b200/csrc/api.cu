@@ -797,4 +797,42 @@ ar_status ar_selftest_timeout(int32_t* status, uint64_t timeout_ns, void* stream
   return from_cuda(launch_timeout_selftest(status, timeout_ns, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------------------
+// ar_tune_layer_static: tuning without any device-memory allocation.
+//
+// The scratch lives in one fixed array in device memory, created when the
+// library's device code is loaded on a GPU and held until the process exits.  In
+// host code `g_static_scratch` names a host-side stand-in, not the device array,
+// so its device address is looked up (cudaGetSymbolAddress) once per device, with
+// that device current, on the first call there, and cached.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) uint8_t g_static_scratch[AR_STATIC_SCRATCH_BYTES];
+
+static std::mutex g_static_mu;
+static void* g_static_ptr[256];
+
+ar_status ar_tune_layer_static(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
+                               int64_t n_rows, const ar_tune_params* p, uint8_t* codes, float* scale, int32_t* zp,
+                               float* loss_trace, double* final_mse, void* stream) {
+  const ar_status chk = check_tune_args(out, in, n_rows, p);
+  if (chk != AR_OK) return chk;
+  if (out == 0 || in == 0) return AR_OK;
+  if (make_layout(make_plan(out, in, n_rows, p)).total > AR_STATIC_SCRATCH_BYTES) return AR_ENOMEM;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return AR_ECUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return AR_ECUDA;
+      g_static_ptr[dev] = ptr;
+    }
+    scratch = g_static_ptr[dev];
+  }
+  return tune_impl(W, w_dtype, out, in, X, n_rows, p, nullptr, scratch, AR_STATIC_SCRATCH_BYTES, codes, scale, zp,
+                   loss_trace, final_mse, stream, nullptr);
+}
+
 }  // extern "C"
