@@ -32,9 +32,11 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import DOWN_7B, DOWN_72B, Q_PROJ_7B, TINY, make_activations, make_activations_cuda, make_weight  # noqa: E402
+from workloads import (DOWN_7B, DOWN_72B, Q_PROJ_7B, Q_PROJ_7B_2BLK, TINY, make_activations,  # noqa: E402
+                       make_activations_cuda, make_weight)
 
-WORKLOADS = {"q_proj": Q_PROJ_7B, "tiny": TINY, "down_7b": DOWN_7B, "down_72b": DOWN_72B}
+WORKLOADS = {"q_proj": Q_PROJ_7B, "q_proj_2blk": Q_PROJ_7B_2BLK, "tiny": TINY, "down_7b": DOWN_7B,
+             "down_72b": DOWN_72B}
 METRIC = "signsgd_steps_per_sec"
 UNIT = "steps/s"
 
@@ -98,6 +100,23 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def _recorded_traffic(key: str):
+    """DRAM bytes per launch from profiles/traffic.txt, if the GEMM source is unchanged."""
+    import hashlib
+    try:
+        rec = {}
+        for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
+            parts = line.split()
+            if len(parts) == 2 and not line.startswith("#"):
+                rec[parts[0]] = parts[1]
+        src = open(os.path.join(ROOT, "signed_gradient_rounding_b200", "csrc", "gemm_sm100.cu"), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != rec.get("gemm_source_sha256_16"):
+            return None
+        return int(rec[key]) if key in rec else None
+    except (OSError, ValueError):
+        return None
 
 
 def _dist():
@@ -218,8 +237,10 @@ def run_ours(args):
     upd_ms = sum(t.update_ms for t in timings) / n_launch
     if res_ms > upd_ms:
         dom_name, dom_ms, dom_flops = "residual (kEpiStore)", res_ms, flops_res
+        traffic = _recorded_traffic("direct_residual_bytes")
     else:
         dom_name, dom_ms, dom_flops = "update (kEpiUpdate)", upd_ms, flops_upd
+        traffic = _recorded_traffic(f"{algo}_update_bytes")
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     layer_s = ms_max / args.steps / 1e3
     step_ms = res_ms + upd_ms
@@ -257,7 +278,8 @@ def run_ours(args):
         "final_mse": mse,
         "roofline": {"bound": "tensor", "kernel": f"gemm_kernel {algo} {dom_name}", "achieved": achieved,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                     "traffic_unit": "bytes per launch (ncu, profiles/traffic.txt)",
                      "peak_source": peaks["source"] + " sustained bf16",
                      "per_launch_ms": {"residual": res_ms, "update": upd_ms}},
         "gpu_launches": launches,

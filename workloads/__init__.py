@@ -86,6 +86,10 @@ TINY = LayerWorkload("tiny 256x256 W4 g64", 256, 256, 512, 512, 4, 64, False, 50
                      0.005, 0.005, 0.02, "f32", "tiny")
 Q_PROJ_7B = LayerWorkload("llama7b q_proj 4096x4096 W4 g128", 4096, 4096, 262144, 16384,
                           4, 128, False, 200, 0.005, 0.005, 0.02, "bf16", "llm")
+# The q_proj layer with only 2 calibration blocks: the same per-step kernel shapes
+# on about 1 GB of device memory (for profiler captures that replay kernels).
+Q_PROJ_7B_2BLK = LayerWorkload("llama7b q_proj 4096x4096 W4 g128, 2 calibration blocks", 4096, 4096,
+                               32768, 16384, 4, 128, False, 200, 0.005, 0.005, 0.02, "bf16", "llm")
 DOWN_7B = LayerWorkload("llama7b down_proj 4096x11008 W2 g128", 4096, 11008, 262144, 16384,
                         2, 128, False, 200, 0.005, 0.005, 0.02, "bf16", "llm")
 DOWN_72B = LayerWorkload("qwen2.5-72b down_proj 8192x29568 W2 g128", 8192, 29568, 262144, 16384,
