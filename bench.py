@@ -32,11 +32,11 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import (DOWN_7B, DOWN_72B, Q_PROJ_7B, Q_PROJ_7B_2BLK, TINY, make_activations,  # noqa: E402
-                       make_activations_cuda, make_weight)
+from workloads import (BLOCK_7B, BLOCK_7B_LAYERS, DOWN_7B, DOWN_72B, Q_PROJ_7B, Q_PROJ_7B_2BLK,  # noqa: E402
+                       TINY, make_activations, make_activations_cuda, make_weight)
 
 WORKLOADS = {"q_proj": Q_PROJ_7B, "q_proj_2blk": Q_PROJ_7B_2BLK, "tiny": TINY, "down_7b": DOWN_7B,
-             "down_72b": DOWN_72B}
+             "down_72b": DOWN_72B, "block_7b": BLOCK_7B}
 METRIC = "signsgd_steps_per_sec"
 UNIT = "steps/s"
 
@@ -124,6 +124,66 @@ def _dist():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def run_block(args):
+    """The LLaMA-7B decoder block tuned layer by layer, each layer on the quantised
+    block's activations; one bench step = the whole block (7 x 200 SignSGD steps)."""
+    import torch
+
+    import signed_gradient_rounding_b200 as ar
+    from signed_gradient_rounding_b200.block import block_workspace_bytes, tune_block
+
+    world, rank, local = _dist()
+    if world > 1:
+        raise SystemExit("block_7b runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    c = BLOCK_7B
+    weights = {name: torch.from_numpy(make_weight(o, i, c.w_std, c.w_dtype, seed=10 + j)).to(torch.bfloat16).to(dev)
+               for j, (name, o, i) in enumerate(BLOCK_7B_LAYERS)}
+    x0 = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
+                       split=bool(args.split))
+    ws = torch.empty(block_workspace_bytes(weights, c.n_rows, p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        tune_block(x0, weights, p, workspace=ws)
+    torch.cuda.synchronize()
+    timings = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            tune_block(x0, weights, p, workspace=ws, timings=timings)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if ar.tune_status(ws) != ar.AR_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    peaks = _peaks()
+    steps_total = len(BLOCK_7B_LAYERS) * c.iters * args.steps
+    flops = 0.0
+    for (name, o, i), t in zip(BLOCK_7B_LAYERS * args.steps, timings):
+        pieces = (3 if t.algo == ar.AR_ALGO_GRAM else 2) if args.split else 1
+        flops += c.iters * (pieces * 2.0 * o * i * i if t.algo == ar.AR_ALGO_GRAM
+                            else 2 * pieces * 2.0 * c.batch_rows * o * i)
+    step_ms = sum(t.residual_ms + t.update_ms for t in timings)
+    return {"metric": METRIC, "value": steps_total / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": c.name, "layers": [list(x) for x in BLOCK_7B_LAYERS], "n_rows": c.n_rows,
+                       "batch_rows": c.batch_rows, "iters_per_layer": c.iters, "bits": c.bits,
+                       "group_size": c.group_size, "sym": c.sym, "bench_step": "one whole block (7 layers)",
+                       "l2": "inputs larger than L2 (activations 2.1-5.8 GB)"},
+            "block_tune_s": ms / args.steps / 1e3,
+            "algos": sorted({("gram" if t.algo == ar.AR_ALGO_GRAM else "direct") for t in timings}),
+            "fused_step_tflops": flops / (step_ms * 1e-3) / 1e12,
+            "tensor_peak_frac": flops / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+            "gpu_launches": sum(t.kernel_launches for t in timings) + 5 * args.steps,
+            "clocks": clk.summary(), "e2e": None}
 
 
 def run_ours(args):
@@ -384,7 +444,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        line = run_reference(args)
+    elif args.workload == "block_7b":
+        line = run_block(args)
+    else:
+        line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

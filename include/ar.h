@@ -218,6 +218,39 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
 ar_status ar_block_schedule(int64_t n_blocks, int64_t first, int64_t count, uint64_t seed,
                             int64_t* blocks);
 
+/* ---------------------------------------------------------------------------
+ * Layer chain ("[llm-compressor] AutoRound ...", "enable_quanted_input 모드": with
+ * quant-aware calibration each layer is tuned on the output of the already
+ * quantised layers before it; the per-layer loop ends by replacing the layer's
+ * weight with the fake-quantised W' = s*(q - zp) -- "최종 양자화 적용").
+ * ------------------------------------------------------------------------- */
+
+/* W' = s*(q - zp) per element (one fp32 operation after the exact q - zp).
+ *   codes [out, in] uint8, scale/zp [out, G] (G = in / group_size; -1: whole row).
+ *   Wq_hi [out, in] bf16 bits out: bf16(W'); Wq_lo [out, in] bf16 bits out (may be
+ *   NULL): bf16(W' - bf16(W')), so hi + lo carries ~16 significant bits;
+ *   Wq [out, in] fp32 out (may be NULL).
+ * AR_EINVAL: bad group_size, NULL codes/scale/zp/Wq_hi.  out == 0 or in == 0: no-op. */
+ar_status ar_dequant(const uint8_t* codes, const float* scale, const int32_t* zp, int64_t out,
+                     int64_t in, int32_t group_size, uint16_t* Wq_hi, uint16_t* Wq_lo,
+                     float* Wq, void* stream);
+
+/* Y = bf16(X (Wq_hi + Wq_lo)^T + add): the linear layer with the quantised weight,
+ * on the tensor cores (fp32 accumulation), rounded once to bf16.
+ *   X [n, in] bf16 bits, Wq_hi/Wq_lo [out, in] bf16 bits (Wq_lo may be NULL),
+ *   add [n, out] bf16 bits or NULL (a residual added in fp32 before rounding),
+ *   Y [n, out] bf16 bits out.  All 16-byte aligned; in and out multiples of 8.
+ *   status: device int32 or NULL; a bounded wait in the kernel that runs out sets
+ *   it to AR_ETIMEOUT (Y is then invalid).  The caller zeroes it beforehand.
+ * AR_EINVAL: NULL or misaligned pointers, in or out not a multiple of 8.  n == 0: no-op. */
+ar_status ar_linear(const uint16_t* X, int64_t n, int64_t in, const uint16_t* Wq_hi,
+                    const uint16_t* Wq_lo, int64_t out, const uint16_t* add, uint16_t* Y,
+                    int32_t* status, void* stream);
+
+/* y = bf16(silu(a) * b), silu(a) = a / (1 + exp(-a)), in fp32 (the gated MLP input
+ * of a LLaMA-style down projection).  a, b, y: count bf16 bits. */
+ar_status ar_silu_mul(const uint16_t* a, const uint16_t* b, int64_t count, uint16_t* y, void* stream);
+
 /* Size of the fixed device scratch array used by ar_tune_layer_static (64 MiB). */
 #define AR_STATIC_SCRATCH_BYTES (64ull << 20)
 

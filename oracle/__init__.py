@@ -53,3 +53,4 @@ from .autoround import (  # noqa: F401
 )
 from .pack import pack_codes, unpack_codes  # noqa: F401
 from .schedule import block_schedule, splitmix64_stream  # noqa: F401
+from . import chain  # noqa: F401

@@ -28,7 +28,8 @@ ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
-           "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static")
+           "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static", "ar_dequant", "ar_linear",
+           "ar_silu_mul")
 
 
 class ArError(RuntimeError):
@@ -86,6 +87,12 @@ def _load() -> ctypes.CDLL:
     lib.ar_tune_layer_static.restype = ctypes.c_int
     lib.ar_tune_layer_static.argtypes = [P, ctypes.c_int, I64, I64, P, I64, ctypes.POINTER(TuneParams),
                                          P, P, P, P, P, P]
+    lib.ar_dequant.restype = ctypes.c_int
+    lib.ar_dequant.argtypes = [P, P, P, I64, I64, I32, P, P, P, P]
+    lib.ar_linear.restype = ctypes.c_int
+    lib.ar_linear.argtypes = [P, I64, I64, P, P, I64, P, P, P, P]
+    lib.ar_silu_mul.restype = ctypes.c_int
+    lib.ar_silu_mul.argtypes = [P, P, I64, P, P]
     lib.ar_tune_status.restype = ctypes.c_int
     lib.ar_tune_status.argtypes = [P, P]
     lib.ar_selftest_timeout.restype = ctypes.c_int
@@ -181,6 +188,42 @@ def pack(codes: torch.Tensor, bits: int, stream=None) -> torch.Tensor:
     packed = torch.empty((rows, cols * bits // 32), dtype=torch.int32, device=codes.device)
     _check(_lib.ar_pack(_ptr(codes), rows, cols, bits, _ptr(packed), _stream(stream)), "ar_pack")
     return packed
+
+
+def dequant(codes: torch.Tensor, scale: torch.Tensor, zp: torch.Tensor, group_size: int, want_lo: bool = True,
+            want_f32: bool = False, stream=None):
+    """W' = s*(q - zp): (bf16 hi, bf16 lo or None, fp32 or None), each [out, in]."""
+    _dev(codes, "codes", torch.uint8)
+    out, inn = codes.shape
+    hi = torch.empty((out, inn), dtype=torch.bfloat16, device=codes.device)
+    lo = torch.empty_like(hi) if want_lo else None
+    f32 = torch.empty((out, inn), dtype=torch.float32, device=codes.device) if want_f32 else None
+    _check(_lib.ar_dequant(_ptr(codes), _ptr(scale), _ptr(zp), out, inn, group_size, _ptr(hi), _ptr(lo),
+                           _ptr(f32), _stream(stream)), "ar_dequant")
+    return hi, lo, f32
+
+
+def linear(X: torch.Tensor, Wq_hi: torch.Tensor, Wq_lo: torch.Tensor | None = None,
+           add: torch.Tensor | None = None, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """bf16(X (Wq_hi + Wq_lo)^T + add) on the tensor cores: X [n, in] bf16, Wq [out, in] bf16."""
+    _dev(X, "X", torch.bfloat16)
+    _dev(Wq_hi, "Wq_hi", torch.bfloat16)
+    n, inn = X.shape
+    o = Wq_hi.shape[0]
+    Y = out if out is not None else torch.empty((n, o), dtype=torch.bfloat16, device=X.device)
+    _check(_lib.ar_linear(_ptr(X), n, inn, _ptr(Wq_hi), _ptr(Wq_lo), o, _ptr(add), _ptr(Y), _ptr(status),
+                          _stream(stream)), "ar_linear")
+    return Y
+
+
+def silu_mul(a: torch.Tensor, b: torch.Tensor, stream=None) -> torch.Tensor:
+    """bf16(silu(a) * b) elementwise on bf16 tensors."""
+    _dev(a, "a", torch.bfloat16)
+    _dev(b, "b", torch.bfloat16)
+    y = torch.empty_like(a)
+    _check(_lib.ar_silu_mul(_ptr(a), _ptr(b), a.numel(), _ptr(y), _stream(stream)), "ar_silu_mul")
+    return y
 
 
 def make_params(bits=4, group_size=128, sym=False, iters=200, lr=0.005, minmax_lr=-1.0, minmax_shrink=1.0,

@@ -797,6 +797,59 @@ ar_status ar_selftest_timeout(int32_t* status, uint64_t timeout_ns, void* stream
   return from_cuda(launch_timeout_selftest(status, timeout_ns, static_cast<cudaStream_t>(stream)));
 }
 
+ar_status ar_dequant(const uint8_t* codes, const float* scale, const int32_t* zp, int64_t out, int64_t in,
+                     int32_t group_size, uint16_t* Wq_hi, uint16_t* Wq_lo, float* Wq, void* stream) {
+  if (out < 0 || in < 0) return AR_EINVAL;
+  if (out == 0 || in == 0) return AR_OK;
+  if (!group_ok(in, group_size) || !codes || !scale || !zp || !Wq_hi) return AR_EINVAL;
+  return from_cuda(launch_dequant(codes, scale, zp, out, in, static_cast<int>(group_of(in, group_size)),
+                                  reinterpret_cast<__nv_bfloat16*>(Wq_hi), reinterpret_cast<__nv_bfloat16*>(Wq_lo),
+                                  Wq, static_cast<cudaStream_t>(stream)));
+}
+
+// Where ar_linear's bounded waits report when the caller passes no status word.
+static __device__ int g_linear_status;
+
+ar_status ar_linear(const uint16_t* X, int64_t n, int64_t in, const uint16_t* Wq_hi, const uint16_t* Wq_lo,
+                    int64_t out, const uint16_t* add, uint16_t* Y, int32_t* status, void* stream) {
+  if (n < 0 || in <= 0 || out <= 0 || in % 8 != 0 || out % 8 != 0) return AR_EINVAL;
+  if (n >= (1ll << 31) || in >= (1ll << 31) || out >= (1ll << 31)) return AR_EUNSUPPORTED;
+  if (n == 0) return AR_OK;
+  if (!X || !Wq_hi || !Y || !aligned(X, 16) || !aligned(Wq_hi, 16) || !aligned(Y, 16)) return AR_EINVAL;
+  if ((Wq_lo && !aligned(Wq_lo, 16)) || (add && !aligned(add, 16))) return AR_EINVAL;
+  int dev = 0, sms = 0, major = 0;
+  AR_CUDA_TRY(cudaGetDevice(&dev));
+  AR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  AR_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (major != 10) return AR_EUNSUPPORTED;
+  const int bn = 256;
+  GemmMaps m{};
+  AR_CUDA_TRY(make_tmap_bf16(&m.a0, X, n, in, kBM));
+  AR_CUDA_TRY(make_tmap_bf16(&m.b0, Wq_hi, out, in, bn));
+  m.a1 = m.a0;
+  if (Wq_lo)
+    AR_CUDA_TRY(make_tmap_bf16(&m.b1, Wq_lo, out, in, bn));
+  else
+    m.b1 = m.b0;
+  GemmArgs a;
+  fill_grid(a, n, out, in, bn, Wq_lo ? 2 : 1);
+  a.seg_b[1] = 1;  // X Wq_hi^T + X Wq_lo^T
+  a.C_hi = reinterpret_cast<__nv_bfloat16*>(Y);
+  a.C_add = reinterpret_cast<const __nv_bfloat16*>(add);
+  a.ldc = out;
+  if (!status) AR_CUDA_TRY(cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_linear_status));
+  a.status = status;
+  return from_cuda(launch_gemm(kEpiStore, bn, m, a, sms, static_cast<cudaStream_t>(stream)));
+}
+
+ar_status ar_silu_mul(const uint16_t* a, const uint16_t* b, int64_t count, uint16_t* y, void* stream) {
+  if (count < 0) return AR_EINVAL;
+  if (count == 0) return AR_OK;
+  if (!a || !b || !y) return AR_EINVAL;
+  return from_cuda(launch_silu_mul(reinterpret_cast<const __nv_bfloat16*>(a), reinterpret_cast<const __nv_bfloat16*>(b),
+                                   count, reinterpret_cast<__nv_bfloat16*>(y), static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------------------
 // ar_tune_layer_static: tuning without any device-memory allocation.
 //

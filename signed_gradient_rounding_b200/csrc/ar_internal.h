@@ -71,6 +71,10 @@ cudaError_t launch_finalize_best(const FinalizeBestArgs& a, cudaStream_t stream)
 // and dsum[k] = sum over blocks of diag[b*in + k] (the exact diagonals).
 cudaError_t launch_gram_sum(const __nv_bfloat16* H_hi, const __nv_bfloat16* H_lo, int nb, int64_t count,
                             __nv_bfloat16* Hs_hi, __nv_bfloat16* Hs_lo, cudaStream_t stream);
+cudaError_t launch_dequant(const uint8_t* codes, const float* scale, const int32_t* zp, int64_t out, int64_t in,
+                           int g, __nv_bfloat16* Wq_hi, __nv_bfloat16* Wq_lo, float* Wq, cudaStream_t stream);
+cudaError_t launch_silu_mul(const __nv_bfloat16* a, const __nv_bfloat16* b, int64_t count, __nv_bfloat16* y,
+                            cudaStream_t stream);
 cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
@@ -106,6 +110,7 @@ struct GemmArgs {
   // kEpiStore: C rows j go to row c_row_off + j of [*, ldc]
   __nv_bfloat16* C_hi = nullptr;
   __nv_bfloat16* C_lo = nullptr;  // may be null
+  const __nv_bfloat16* C_add = nullptr;  // may be null: [*, ldc] added in fp32 before the store
   int64_t ldc = 0;
   int64_t c_row_off = 0;
   // kEpiStore / kEpiSumSq / kEpiDotD / kEpiUpdate (Gram loss): per-(row, n-tile) sums
@@ -155,6 +160,7 @@ constexpr int kBK = 64;
 
 cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
                         cudaStream_t stream);
+
 
 // TMA descriptor for a row-major bf16 matrix [rows, cols], box [box_rows, 64]
 // with 128-byte swizzle; zero fill outside the matrix.

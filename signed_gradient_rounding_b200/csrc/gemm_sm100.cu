@@ -195,6 +195,12 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
     }
     if (kKind == kEpiStore) {
       const int64_t off = (a.c_row_off + j) * a.ldc + col0;
+      if (a.C_add) {
+        float ad[32];
+        load_bf16x32(a.C_add + off, ad);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] += ad[i];
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);

@@ -219,7 +219,55 @@ __global__ void diag_sum_kernel(const float* __restrict__ diag, int nb, int64_t 
   }
 }
 
+// W' = s * (q - zp), one element per thread.
+__global__ void dequant_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ scale,
+                               const int32_t* __restrict__ zp, int64_t out, int64_t in, int g,
+                               __nv_bfloat16* __restrict__ Wq_hi, __nv_bfloat16* __restrict__ Wq_lo,
+                               float* __restrict__ Wq) {
+  const int64_t total = out * in;
+  const int64_t G = in / g;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / in;
+    const int64_t gi = row * G + (i - row * in) / g;
+    const float w = __fmul_rn(scale[gi], __fsub_rn(static_cast<float>(codes[i]), static_cast<float>(zp[gi])));
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    Wq_hi[i] = hi;
+    if (Wq_lo) Wq_lo[i] = __float2bfloat16_rn(__fsub_rn(w, __bfloat162float(hi)));
+    if (Wq) Wq[i] = w;
+  }
+}
+
+__global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                                int64_t count, __nv_bfloat16* __restrict__ y) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float x = __bfloat162float(a[i]);
+    const float s = x / (1.0f + expf(-x));
+    y[i] = __float2bfloat16_rn(s * __bfloat162float(b[i]));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dequant(const uint8_t* codes, const float* scale, const int32_t* zp, int64_t out, int64_t in,
+                           int g, __nv_bfloat16* Wq_hi, __nv_bfloat16* Wq_lo, float* Wq, cudaStream_t stream) {
+  const int64_t total = out * in;
+  if (total == 0) return cudaSuccess;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(codes, scale, zp, out, in, g, Wq_hi, Wq_lo, Wq);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_silu_mul(const __nv_bfloat16* a, const __nv_bfloat16* b, int64_t count, __nv_bfloat16* y,
+                            cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  int64_t blocks = (count + 255) / 256;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  silu_mul_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a, b, count, y);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream) {
   if (in == 0) return cudaSuccess;

@@ -15,8 +15,8 @@ import torch
 
 import oracle
 from oracle import autoround as oar
-from workloads import (Q_PROJ_7B, TINY, bf16_round, make_activations, make_activations_cuda,
-                       make_weight)
+from workloads import (DOWN_7B, DOWN_72B, Q_PROJ_7B, TINY, bf16_round, make_activations,
+                       make_activations_cuda, make_weight)
 
 pytestmark = pytest.mark.gpu
 
@@ -290,6 +290,52 @@ def test_rejects_unsupported(ar):
     with pytest.raises(ar.ArError) as e:
         ar.tune_layer(W, X, ar.make_params(group_size=16, batch_rows=512))
     assert e.value.status in (ar.AR_EUNSUPPORTED, ar.AR_EINVAL)
+
+
+def _full_size_case(c, n_sample):
+    """A full-size workload on the device and the oracle replaying sampled rows."""
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0)
+    rows = np.sort(np.random.default_rng(0).choice(c.out, n_sample, replace=False))
+    Xh = _x_bits(Xd)
+    ref = oracle.tune_layer(W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr,
+                            c.batch_rows, 0, want_final_mse=False)
+    return c, W, Xd, Xh, rows, ref
+
+
+def _check_full_size(ar, case, algo, mse_rows=65536):
+    c, W, Xd, Xh, rows, ref = case
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
+                       batch_rows=c.batch_rows, seed=0, algo=algo)
+    res = ar.tune_layer(_w_dev(W, "bf16"), Xd, p, want_final_mse=False)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    del res.workspace
+    codes = _np(res.codes)[rows]
+    frac = float(np.mean(codes != ref.codes))
+    # MSE of the GPU's sampled rows, evaluated by the oracle's own fp64 loss
+    s = _np(res.scale)[rows]
+    z = _np(res.zero_point)[rows].astype(np.float32)
+    Wq_gpu = np.repeat(s, c.group_size, 1) * (codes.astype(np.float32) - np.repeat(z, c.group_size, 1))
+    mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:mse_rows])
+    mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:mse_rows])
+    print(f"{c.name} {algo}: {frac:.3%} of sampled codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
+    assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
+    assert frac <= CHAOS_CODE_BOUND, f"{frac:.4%} of sampled codes differ"
+    _, _, _, Wrtn = oracle.rtn(W[rows], c.bits, c.group_size, c.sym)
+    assert mse_gpu < oar.layer_mse(W[rows], Wrtn, Xh[:mse_rows])
+
+
+@pytest.mark.parametrize("algo", ["auto"])
+def test_down_7b_full_size_sampled_rows(ar, algo):
+    """LLaMA-7B down_proj, 4096 x 11008 W2 g128, 262144 x 11008 activations, 200 steps."""
+    _check_full_size(ar, _full_size_case(DOWN_7B, 64), algo, mse_rows=32768)
+
+
+@pytest.mark.parametrize("algo", ["auto"])
+def test_down_72b_full_size_sampled_rows(ar, algo):
+    """Qwen2.5-72B down_proj, 8192 x 29568 W2 g128, 262144 x 29568 activations (15.5 GB),
+    200 steps; the oracle replays 32 sampled rows."""
+    _check_full_size(ar, _full_size_case(DOWN_72B, 32), algo, mse_rows=16384)
 
 
 @pytest.fixture(scope="module")

@@ -396,3 +396,49 @@ def test_pack_matches_bitstream_and_round_trips(bits):
     decoded = (stream.reshape(5, 96, bits) * weights).sum(-1)
     assert np.array_equal(decoded, codes)
     assert np.array_equal(oracle.unpack_codes(packed, bits, 96), codes)
+
+
+# ---------------------------------------------------------------- layer chain
+
+def _bf16_neighbours(x64):
+    x32 = x64.astype(np.float32)
+    b = x32.view(np.uint32).astype(np.uint64)
+    lo = ((b >> 16) << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    hi = (((b >> 16) + 1) << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    return lo, hi
+
+
+def test_chain_bf16_rounding_is_nearest():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(20000) * 10.0 ** rng.uniform(-3, 3, 20000)
+    r = oracle.chain._bf16_round(x).astype(np.float64)
+    lo, hi = _bf16_neighbours(x)
+    best = np.minimum(np.abs(x - lo), np.abs(hi - x))
+    assert np.all(np.abs(r - x) <= best)
+    x32 = rng.standard_normal(20000).astype(np.float32)          # fp32 inputs: plain RNE
+    assert np.array_equal(oracle.chain._bf16_round(x32.astype(np.float64)), bf16_round(x32))
+
+
+def test_chain_dequant_reconstructs_grid_example():
+    d = json.load(open(os.path.join(GOLDEN, "rtn_grid_example.json")))
+    codes = np.array([d["codes"]], dtype=np.uint8)
+    W = oracle.chain.dequant(codes, np.array([[d["scale"]]], np.float32), np.array([[d["zero_point"]]]), 16)
+    assert np.array_equal(W[0], np.array(d["w"], np.float32))
+
+
+def test_chain_linear_and_silu_match_torch():
+    rng = np.random.default_rng(6)
+    X = bf16_round(rng.standard_normal((64, 96)).astype(np.float32))
+    Wq = (rng.standard_normal((40, 96)) * 0.02).astype(np.float32)
+    add = bf16_round(rng.standard_normal((64, 40)).astype(np.float32))
+    Y = oracle.chain.linear(X, Wq, add).astype(np.float64)
+    ref = (torch.nn.functional.linear(torch.from_numpy(X.astype(np.float64)),
+                                      torch.from_numpy(Wq.astype(np.float64))) + torch.from_numpy(add.astype(np.float64))).numpy()
+    lo, hi = _bf16_neighbours(ref)
+    assert np.all(np.abs(Y - ref) <= np.minimum(np.abs(ref - lo), np.abs(hi - ref)))
+    a = bf16_round(rng.standard_normal(5000).astype(np.float32) * 4)
+    b = bf16_round(rng.standard_normal(5000).astype(np.float32))
+    y = oracle.chain.silu_mul(a, b).astype(np.float64)
+    ref = (torch.nn.functional.silu(torch.from_numpy(a.astype(np.float64))) * torch.from_numpy(b.astype(np.float64))).numpy()
+    lo, hi = _bf16_neighbours(ref)
+    assert np.all(np.abs(y - ref) <= np.minimum(np.abs(ref - lo), np.abs(hi - ref)))

@@ -95,7 +95,10 @@ DOWN_7B = LayerWorkload("llama7b down_proj 4096x11008 W2 g128", 4096, 11008, 262
 DOWN_72B = LayerWorkload("qwen2.5-72b down_proj 8192x29568 W2 g128", 8192, 29568, 262144, 16384,
                          2, 128, False, 200, 0.005, 0.005, 0.015, "bf16", "llm")
 
-# The LLaMA-7B decoder block, tuned layer by layer (W3, g128, symmetric).
+# The LLaMA-7B decoder block, tuned layer by layer (W3, g128, symmetric), each layer on
+# the quantised block's activations at its input width (262144 calibration rows).
+BLOCK_7B = LayerWorkload("llama7b decoder block (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008) W3 g128 sym",
+                         4096, 4096, 262144, 16384, 3, 128, True, 200, 0.005, 0.005, 0.02, "bf16", "llm")
 BLOCK_7B_LAYERS = [
     ("q_proj", 4096, 4096), ("k_proj", 4096, 4096), ("v_proj", 4096, 4096),
     ("o_proj", 4096, 4096), ("gate_proj", 11008, 4096), ("up_proj", 11008, 4096),
