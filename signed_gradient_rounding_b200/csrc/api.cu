@@ -442,6 +442,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       m.b1 = m.b0;
       GemmArgs h;
       fill_grid(h, in, in, B, P.bn_gram, 1);
+      h.symmetric = 1;  // H_b = X_b^T X_b: compute the tiles reaching the upper triangle
+      h.num_tiles = 0;
+      for (int n = 0; n < h.num_n_blk; ++n)
+        h.num_tiles += static_cast<int>(std::min<int64_t>(h.num_m_blk, cdiv((n + 1) * int64_t(P.bn_gram), kBM)));
       h.timeout_ns = timeout_ns;
       h.status = status;
       h.C_hi = Hh;

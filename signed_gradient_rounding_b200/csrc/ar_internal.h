@@ -112,6 +112,10 @@ struct GemmArgs {
   __nv_bfloat16* C_lo = nullptr;  // may be null
   const __nv_bfloat16* C_add = nullptr;  // may be null: [*, ldc] added in fp32 before the store
   int64_t ldc = 0;
+  // kEpiStore of a symmetric C (M == N, A == B): only tiles that reach the upper
+  // triangle run (num_tiles counts them); each writes its upper elements in place and
+  // its strictly upper ones again transposed, so every element is written once.
+  int symmetric = 0;
   int64_t c_row_off = 0;
   // kEpiStore / kEpiSumSq / kEpiDotD / kEpiUpdate (Gram loss): per-(row, n-tile) sums
   float* part = nullptr;  // [M, part_ld] (kEpiUpdate: part_out)

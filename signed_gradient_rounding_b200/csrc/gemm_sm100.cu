@@ -140,6 +140,23 @@ __device__ __forceinline__ void store_pair8(const float* x, __nv_bfloat16* hi_ds
                                                    pack_bf16x2(l[4], l[5]), pack_bf16x2(l[6], l[7]));
 }
 
+// Tile t of the launch -> (m_blk, n_blk).  Plain: m fastest.  Symmetric: only the
+// tiles with some column >= row, n-major, ceil((n + 1) * BN / BM) of them per n.
+template <int kBN>
+__device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, int& n_blk) {
+  if (!a.symmetric) {
+    m_blk = t % a.num_m_blk;
+    n_blk = t / a.num_m_blk;
+    return;
+  }
+  for (n_blk = 0; n_blk < a.num_n_blk; ++n_blk) {
+    const int cnt = min(a.num_m_blk, ((n_blk + 1) * kBN + kBM - 1) / kBM);
+    if (t < cnt) break;
+    t -= cnt;
+  }
+  m_blk = t;
+}
+
 // ---------------------------------------------------------------------------
 // epilogues
 // ---------------------------------------------------------------------------
@@ -201,9 +218,41 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] += ad[i];
       }
+      if (!a.symmetric) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
+        for (int q = 0; q < 4; ++q)
+          if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
+      } else {
+        // upper elements (col >= row) in place, strictly upper ones also at [col, row]
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c8 = col0 + q * 8;
+          if (q * 8 >= nvalid || c8 + 7 < j) continue;
+          if (c8 >= j) {
+            store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (c8 + i >= j) {
+                float h, l;
+                split_bf16(x[q * 8 + i], h, l);
+                a.C_hi[off + q * 8 + i] = __float2bfloat16_rn(h);
+                if (a.C_lo) a.C_lo[off + q * 8 + i] = __float2bfloat16_rn(l);
+              }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = col0 + i;
+          if (i < nvalid && col > j) {
+            float h, l;
+            split_bf16(x[i], h, l);
+            const int64_t mo = (a.c_row_off + col) * a.ldc + j;
+            a.C_hi[mo] = __float2bfloat16_rn(h);
+            if (a.C_lo) a.C_lo[mo] = __float2bfloat16_rn(l);
+          }
+        }
+      }
     }
   }
   if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk] = acc;
@@ -404,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        const int m_blk = tile % args.num_m_blk;
-        const int n_blk = tile / args.num_m_blk;
+        int m_blk, n_blk;
+        tile_pos<kBN>(args, tile, m_blk, n_blk);
         for (int kb = 0; kb < k_blocks; ++kb) {
           const int seg = kb / args.num_k_blk;
           const int kk = kb - seg * args.num_k_blk;
@@ -483,8 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
-      const int m_blk = tile % args.num_m_blk;
-      const int n_blk = tile / args.num_m_blk;
+      int m_blk, n_blk;
+      tile_pos<kBN>(args, tile, m_blk, n_blk);
       if (!mbar_wait(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;

@@ -104,12 +104,35 @@ __global__ void fill_f32_kernel(float* p, int64_t n, float v) {
     p[i] = v;
 }
 
-// 64 x 64 tiles through shared memory; 256 threads, each moving 16 elements.
+// 64 x 64 tiles through shared memory; 256 threads.  Full tiles move 16-byte
+// vectors both ways (rows and cols multiples of 8 keep them aligned); the tile's
+// ragged edges fall back to single elements.
 __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
                                       uint16_t* __restrict__ Xt) {
-  __shared__ uint16_t tile[64][66];
+  __shared__ __align__(16) uint16_t tile[64][72];
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 64;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const bool full = (r0 + 64 <= rows) && (c0 + 64 <= cols) && (rows % 8 == 0) && (cols % 8 == 0);
+  if (full) {
+    for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 rows x 8 vectors
+      const int r = v >> 3, c8 = (v & 7) * 8;
+      *reinterpret_cast<uint4*>(&tile[r][c8]) = *reinterpret_cast<const uint4*>(X + (r0 + r) * cols + c0 + c8);
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 output rows (cols of X) x 8 vectors
+      const int c = v >> 3, r8 = (v & 7) * 8;
+      uint16_t e[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) e[k] = tile[r8 + k][c];
+      uint4 o;
+      o.x = e[0] | (uint32_t(e[1]) << 16);
+      o.y = e[2] | (uint32_t(e[3]) << 16);
+      o.z = e[4] | (uint32_t(e[5]) << 16);
+      o.w = e[6] | (uint32_t(e[7]) << 16);
+      *reinterpret_cast<uint4*>(Xt + (c0 + c) * rows + r0 + r8) = o;
+    }
+    return;
+  }
   const int tx = threadIdx.x & 63;
   const int ty = threadIdx.x >> 6;  // 0..3
   for (int i = ty; i < 64; i += 4) {
