@@ -153,6 +153,9 @@ struct Plan {
   int bn_gram = 128;  // Gram matrices (N = in)
   int bn_fin = 256;   // final-MSE GEMM
   int64_t nparts_res = 0, nparts_upd = 0, nparts_fin = 0;
+  // Gram-form update GEMM on 2-SM pair tiles (256 x 256, tcgen05 cta_group::2):
+  // each SM stages 32 KB per K block instead of 48 KB, so six stages fit.
+  bool pair_upd = true;
 };
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
@@ -184,9 +187,10 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p) {
   P.bn_upd = 256;
   P.bn_gram = 256;
   P.bn_fin = 256;
-  P.nparts_res = cdiv(P.B, P.bn_res);
-  P.nparts_upd = cdiv(in, P.bn_upd);
-  P.nparts_fin = P.algo == AR_ALGO_GRAM ? cdiv(in, P.bn_fin) : cdiv(n, P.bn_fin);
+  // Row partial sums: kEpiHalves per n-tile (one per epilogue column half).
+  P.nparts_res = cdiv(P.B, P.bn_res) * kEpiHalves;
+  P.nparts_upd = cdiv(in, P.bn_upd) * kEpiHalves;
+  P.nparts_fin = (P.algo == AR_ALGO_GRAM ? cdiv(in, P.bn_fin) : cdiv(n, P.bn_fin)) * kEpiHalves;
   return P;
 }
 
@@ -247,11 +251,12 @@ Layout make_layout(const Plan& P) {
   return L;
 }
 
-void fill_grid(GemmArgs& a, int64_t M, int64_t N, int64_t K, int bn, int num_seg) {
+void fill_grid(GemmArgs& a, int64_t M, int64_t N, int64_t K, int bn, int num_seg, bool pair = false) {
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.num_m_blk = static_cast<int>(cdiv(M, kBM));
+  a.pair = pair ? 1 : 0;
+  a.num_m_blk = static_cast<int>(cdiv(M, pair ? 2 * kBM : kBM));
   a.num_n_blk = static_cast<int>(cdiv(N, bn));
   a.num_k_blk = static_cast<int>(cdiv(K, kBK));
   a.num_tiles = a.num_m_blk * a.num_n_blk;
@@ -461,13 +466,15 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       }
     }
     GemmMaps m[2]{};  // per parity of t: A = D_t
+    // 2-SM pair tiles: each CTA of a pair stages half of the tile's B rows.
+    const uint32_t b_box = P.pair_upd ? P.bn_upd / 2 : P.bn_upd;
     for (int q = 0; q < 2; ++q) {
       AR_CUDA_TRY(make_tmap_bf16(&m[q].a0, Dh[q], out, in, kBM));
       AR_CUDA_TRY(make_tmap_bf16(&m[q].a1, Dl[q], out, in, kBM));
-      AR_CUDA_TRY(make_tmap_bf16(&m[q].b0, Hh, P.nb * in, in, P.bn_upd));
-      AR_CUDA_TRY(make_tmap_bf16(&m[q].b1, Hl, P.nb * in, in, P.bn_upd));
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].b0, Hh, P.nb * in, in, b_box));
+      AR_CUDA_TRY(make_tmap_bf16(&m[q].b1, Hl, P.nb * in, in, b_box));
     }
-    fill_grid(u, out, in, in, P.bn_upd, nseg_g);
+    fill_grid(u, out, in, in, P.bn_upd, nseg_g, P.pair_upd);
     // (D_hi + D_lo)(H_hi + H_lo) ~ D_hi H_hi + D_lo H_hi + D_hi H_lo
     u.seg_a[0] = 0, u.seg_b[0] = 0;
     u.seg_a[1] = 1, u.seg_b[1] = 0;
@@ -638,7 +645,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       f.Dd_hi = D_hi;
       f.Dd_lo = P.split ? D_lo : nullptr;
       f.diag_in = F(L.Hdsum);
-      f.part_ld = f.num_n_blk;
+      f.part_ld = f.num_n_blk * kEpiHalves;
       AR_CUDA_TRY(launch_gemm(kEpiDotD, P.bn_fin, m, f, sms, st));
       launches += 2;
     } else {
@@ -648,7 +655,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       m.b1 = m.b0;
       fill_grid(f, out, n_rows, in, P.bn_fin, nseg_d);
       f.seg_a[1] = 1;
-      f.part_ld = f.num_n_blk;
+      f.part_ld = f.num_n_blk * kEpiHalves;
       AR_CUDA_TRY(launch_gemm(kEpiSumSq, P.bn_fin, m, f, sms, st));
       ++launches;
     }

@@ -116,9 +116,12 @@ struct GemmArgs {
   // triangle run (num_tiles counts them); each writes its upper elements in place and
   // its strictly upper ones again transposed, so every element is written once.
   int symmetric = 0;
+  // 2-SM pair tiles (tcgen05 cta_group::2, clusters of two CTAs): 256 x 256 tiles,
+  // num_m_blk counts 256-row blocks, B maps use 128-row boxes.
+  int pair = 0;
   int64_t c_row_off = 0;
   // kEpiStore / kEpiSumSq / kEpiDotD / kEpiUpdate (Gram loss): per-(row, n-tile) sums
-  float* part = nullptr;  // [M, part_ld] (kEpiUpdate: part_out)
+  float* part = nullptr;  // [M, part_ld], part_ld >= num_n_blk * kEpiHalves (kEpiUpdate: part_out)
   int part_ld = 0;
   // kEpiStore: when set, the diagonal (column == row j) is written here in fp32,
   // at [c_row_off + j], and stored as 0 in the bf16 pair
@@ -161,6 +164,10 @@ struct GemmArgs {
 // Tile sizes: M and K tiles fixed, N tile 128 or 256 per launch.
 constexpr int kBM = 128;
 constexpr int kBK = 64;
+// Two epilogue warps share each accumulator row, one per column half of the tile;
+// the per-(row, n-tile) partial sums (GemmArgs::part, part_out) therefore hold
+// kEpiHalves entries per n-tile, at n_blk * kEpiHalves + half.
+constexpr int kEpiHalves = 2;
 
 cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
                         cudaStream_t stream);

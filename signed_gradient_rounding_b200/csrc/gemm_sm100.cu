@@ -8,16 +8,19 @@
 // 16 significant bits) is multiplied as extra segments of the same accumulation:
 // (hi_a + lo_a)(hi_b + lo_b) ~ hi_a hi_b + lo_a hi_b + hi_a lo_b.
 //
-// Roles (192 threads, one CTA per SM):
+// Roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage, 128-byte
 //               swizzle, completion counted on the stage's mbarrier.
 //   warp 1      MMA issuer: four tcgen05.mma (M=128, N=BN, K=16) per stage into one
 //               of two BN-column fp32 accumulators in tensor memory;
 //               tcgen05.commit frees the stage and, after the last K block, hands
 //               the accumulator to the epilogue.
-//   warps 2..5  epilogue: each thread owns one accumulator row (its warp's 32-lane
-//               slice of tensor memory) and walks the tile's columns 32 at a time
-//               with tcgen05.ld, while the MMA warp fills the other accumulator.
+//   warps 2..9  epilogue: two warps per 32-lane slice of tensor memory (a warp may
+//               only read the slice warp % 4), one per column half of the tile.
+//               Each thread owns one accumulator row and walks its half's columns
+//               with tcgen05.ld while the MMA warp fills the other accumulator.
+//               The halves never wait for each other: each writes its own row
+//               partial sums (kEpiHalves entries per n-tile).
 //
 // Epilogues (the contractions of the AutoRound SignSGD loop,
 // "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END"):
@@ -42,18 +45,20 @@ namespace ar {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4 * kEpiHalves;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTileABytes = kBM * kBK * 2;  // 16 KB
 
-template <int kBN>
+// Per-CTA operand staging: 128 A rows and kBN (pair: kBN / 2) B rows per stage.
+template <int kBN, bool kPair>
 struct Cfg {
-  static constexpr int kTileBBytes = kBN * kBK * 2;
+  static constexpr int kTileBBytes = (kPair ? kBN / 2 : kBN) * kBK * 2;
   static constexpr int kStageBytes = kTileABytes + kTileBBytes;
-  static constexpr int kStages = (kBN == 256) ? 4 : 6;
+  static constexpr int kStages = (kStageBytes <= 32 * 1024) ? 6 : 4;
   static constexpr int kTmemCols = 2 * kBN;
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;
-  static constexpr uint32_t kIdesc = umma_idesc_bf16(kBM, kBN);
+  static constexpr uint32_t kIdesc = umma_idesc_bf16(kPair ? 2 * kBM : kBM, kBN);
 };
 
 struct Smem {
@@ -111,10 +116,51 @@ __device__ __forceinline__ void load_f32x32(const float* p, float (&v)[32]) {
   }
 }
 
-__device__ __forceinline__ void store_f32x32(float* p, const float (&v)[32]) {
+// 16-column variants for the update epilogue, which keeps two chunks in registers.
+constexpr int kUC = 16;
+
+__device__ __forceinline__ void load_w16(const void* W, int w_bf16, int64_t idx, float (&w)[kUC]) {
+  if (w_bf16) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(W) + idx);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 x = p[q];
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        w[q * 8 + 2 * h] = __uint_as_float(xs[h] << 16);
+        w[q * 8 + 2 * h + 1] = __uint_as_float(xs[h] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(W) + idx);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 x = p[q];
+      w[q * 4 + 0] = x.x;
+      w[q * 4 + 1] = x.y;
+      w[q * 4 + 2] = x.z;
+      w[q * 4 + 3] = x.w;
+    }
+  }
+}
+
+__device__ __forceinline__ void load_f32x16(const float* p, float (&v)[kUC]) {
+  const float4* q4 = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 x = q4[q];
+    v[q * 4 + 0] = x.x;
+    v[q * 4 + 1] = x.y;
+    v[q * 4 + 2] = x.z;
+    v[q * 4 + 3] = x.w;
+  }
+}
+
+__device__ __forceinline__ void store_f32x16(float* p, const float (&v)[kUC]) {
   float4* q4 = reinterpret_cast<float4*>(p);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) q4[q] = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+  for (int q = 0; q < 4; ++q) q4[q] = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -163,11 +209,12 @@ __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, i
 
 // kEpiStore / kEpiSumSq / kEpiDotD: one pass over the tile's columns.
 template <int kKind, int kBN>
-__device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk) {
+__device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
   float acc = 0.0f;
   const bool row_ok = j < a.M;
+  constexpr int kHalfChunks = kBN / 32 / kEpiHalves;
 #pragma unroll 1
-  for (int c = 0; c < kBN / 32; ++c) {
+  for (int c = half * kHalfChunks; c < (half + 1) * kHalfChunks; ++c) {
     const int col0 = n0 + c * 32;
     if (col0 >= a.N) break;  // warp-uniform
     uint32_t r[32];
@@ -255,12 +302,38 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
       }
     }
   }
-  if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk] = acc;
+  if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = acc;
 }
 
 // kEpiUpdate: one SignSGD step for the rows x columns of this G tile.
+//
+// The tile's groups are split between the two column halves (a group wider than
+// half a tile stays with half 0).  Each chunk of kUC columns is processed while
+// the next chunk's W, V and diagonal values are already on their way into
+// registers, so the memory latency of one chunk overlaps the arithmetic of the
+// previous one.
 template <int kBN>
-__device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk) {
+__device__ __forceinline__ void epi_group_range(const GemmArgs& a, int half, int& gl_begin, int& gl_end) {
+  const int gpt = max(1, kBN / a.g);  // g divides kBN, or g == N <= kBN
+  if (a.g <= kBN / kEpiHalves) {
+    gl_begin = half * (gpt / kEpiHalves);
+    gl_end = gl_begin + gpt / kEpiHalves;
+  } else {
+    gl_begin = 0;
+    gl_end = half == 0 ? gpt : 0;
+  }
+}
+
+// W, V and (Gram form) the exact Gram diagonal of one chunk.
+__device__ __forceinline__ void load_upd_chunk(const GemmArgs& a, int64_t e0, int col, float (&w)[kUC],
+                                               float (&v)[kUC], float (&dg)[kUC]) {
+  load_w16(a.W, a.w_bf16, e0, w);
+  load_f32x16(a.V_in + e0, v);
+  if (a.diag_in) load_f32x16(a.diag_in + col, dg);
+}
+
+template <int kBN>
+__device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
   const bool row_ok = j < a.M;
   const float Q = qmaxf(a.bits);
   const bool sym = a.sym != 0;
@@ -280,18 +353,19 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
     if (a.keep_best) {
       const float mean = L * a.inv_batch;
       better = mean < a.best_in[j];
-      if (n_blk == 0) a.best_out[j] = better ? mean : a.best_in[j];
+      if (n_blk == 0 && half == 0) a.best_out[j] = better ? mean : a.best_in[j];
     }
-    if (n_blk == 0) a.rowloss[j] = L;
+    if (n_blk == 0 && half == 0) a.rowloss[j] = L;
   }
   const bool snap_now = better && !a.snap_prev;
   const bool snap_old = better && a.snap_prev;
 
-  const int groups_in_tile = max(1, kBN / a.g);  // g divides kBN, or g == N <= kBN
-  const int chunks_per_group = a.g / 32;
+  int gl_begin, gl_end;
+  epi_group_range<kBN>(a, half, gl_begin, gl_end);
+  const int cpg = a.g / kUC;  // chunks per group
   float loss_acc = 0.0f;
 #pragma unroll 1
-  for (int gl = 0; gl < groups_in_tile; ++gl) {
+  for (int gl = gl_begin; gl < gl_end; ++gl) {
     const int gcol0 = n0 + gl * a.g;
     if (gcol0 >= a.N) break;  // warp-uniform
     const int64_t gidx = static_cast<int64_t>(j) * a.G + gcol0 / a.g;
@@ -320,27 +394,35 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       }
     }
 
+    // Pass 1: sign updates of V, and the group's d alpha, d beta.
     float dal = 0.f, dbe = 0.f;
+    float w_nx[kUC], v_nx[kUC], dg_nx[kUC];
+    if (row_ok) load_upd_chunk(a, row_base + gcol0, gcol0, w_nx, v_nx, dg_nx);
 #pragma unroll 1
-    for (int cc = 0; cc < chunks_per_group; ++cc) {
-      const int tcol = gl * a.g + cc * 32;
-      uint32_t r[32];
+    for (int cc = 0; cc < cpg; ++cc) {
+      const int col = gcol0 + cc * kUC;
+      const int64_t e0 = row_base + col;
+      float w[kUC], v[kUC], dg[kUC];
+#pragma unroll
+      for (int i = 0; i < kUC; ++i) {
+        w[i] = w_nx[i];
+        v[i] = v_nx[i];
+        dg[i] = dg_nx[i];
+      }
+      if (row_ok && cc + 1 < cpg) load_upd_chunk(a, e0 + kUC, col + kUC, w_nx, v_nx, dg_nx);
+      uint32_t r[kUC];
       __syncwarp();
-      tmem_ld_32cols(t_row + tcol, r);
+      tmem_ld_16cols(t_row + (col - n0), r);
       tmem_ld_wait();
       if (!row_ok) continue;  // nothing warp-collective follows in this iteration
-      const int64_t e0 = row_base + n0 + tcol;
-      float w[32], v[32], vn[32], dg[32];
-      load_w32(a.W, a.w_bf16, e0, w);
-      load_f32x32(a.V_in + e0, v);
-      if (a.diag_in) load_f32x32(a.diag_in + n0 + tcol, dg);
       if (snap_old) {
-        float vo[32];
-        load_f32x32(a.V_out + e0, vo);
-        store_f32x32(a.V_best + e0, vo);
+        float vo[kUC];
+        load_f32x16(a.V_out + e0, vo);
+        store_f32x16(a.V_best + e0, vo);
       }
+      float vn[kUC];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < kUC; ++i) {
         const ElemQuant e = quant_elem(w[i], v[i], gs, Q);
         const float d = __fsub_rn(e.wq, w[i]);
         const float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
@@ -360,8 +442,8 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
         dal = fmaf(G, dwa, dal);
         dbe = fmaf(G, dwb, dbe);
       }
-      store_f32x32(a.V_out + e0, vn);
-      if (snap_now) store_f32x32(a.V_best + e0, v);
+      store_f32x16(a.V_out + e0, vn);
+      if (snap_now) store_f32x16(a.V_best + e0, v);
     }
     if (!row_ok) continue;
 
@@ -378,34 +460,67 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
     a.alpha_out[gidx] = al_n;
     a.beta_out[gidx] = be_n;
 
-    // D = W' - W of the next step, from the updated state, as a bf16 pair.
+    // Pass 2: D = W' - W of the next step, from the updated state, as a bf16 pair
+    // (the values were written by this thread in pass 1).
     const GroupScale gn = group_scale(wmn, wmx, al_n, be_n, a.bits, sym);
+    load_w16(a.W, a.w_bf16, row_base + gcol0, w_nx);
+    load_f32x16(a.V_out + row_base + gcol0, v_nx);
 #pragma unroll 1
-    for (int cc = 0; cc < chunks_per_group; ++cc) {
-      const int64_t e0 = row_base + gcol0 + cc * 32;
-      float w[32], v[32], d[32];
-      load_w32(a.W, a.w_bf16, e0, w);
-      load_f32x32(a.V_out + e0, v);
+    for (int cc = 0; cc < cpg; ++cc) {
+      const int64_t e0 = row_base + gcol0 + cc * kUC;
+      float w[kUC], v[kUC], d[kUC];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q).wq, w[i]);
+      for (int i = 0; i < kUC; ++i) {
+        w[i] = w_nx[i];
+        v[i] = v_nx[i];
+      }
+      if (cc + 1 < cpg) {
+        load_w16(a.W, a.w_bf16, e0 + kUC, w_nx);
+        load_f32x16(a.V_out + e0 + kUC, v_nx);
+      }
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int i = 0; i < kUC; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q).wq, w[i]);
+#pragma unroll
+      for (int q = 0; q < kUC / 8; ++q)
         store_pair8(d + q * 8, a.D_hi + e0 + q * 8, a.D_lo ? a.D_lo + e0 + q * 8 : nullptr);
     }
   }
-  if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk] = loss_acc;
+  if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = loss_acc;
+}
+
+// Before waiting for a tile's accumulator, ask L2 for the W and V row segments the
+// update epilogue of that tile will read, so the wait covers their memory latency.
+template <int kBN>
+__device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, int n0, int half) {
+  if (j >= a.M) return;
+  int gl_begin, gl_end;
+  epi_group_range<kBN>(a, half, gl_begin, gl_end);
+  const int c0 = n0 + gl_begin * a.g;
+  const int c1 = min(a.N, n0 + gl_end * a.g);
+  if (c0 >= c1) return;
+  const int64_t e0 = static_cast<int64_t>(j) * a.N + c0;
+  const uint32_t cols = static_cast<uint32_t>(c1 - c0);  // a multiple of 8
+  const int wsz = a.w_bf16 ? 2 : 4;
+  prefetch_l2(static_cast<const uint8_t*>(a.W) + e0 * wsz, cols * wsz);
+  prefetch_l2(a.V_in + e0, cols * 4);
 }
 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
 
-template <int kKind, int kBN>
+// kPair: a cluster of two CTAs computes one 256 x kBN tile with tcgen05
+// cta_group::2.  CTA `rank` loads its 128 A rows and B rows rank * kBN/2 ..
+// + kBN/2 - 1 of the tile; its TMA bytes are counted on the leader's (rank 0)
+// full barrier; the leader's MMA thread alone issues M = 256 MMAs and its commits
+// arrive on both CTAs' barriers; each CTA's epilogue reads its own 128 accumulator
+// rows and releases the accumulator with one arrive per warp on the leader.
+template <int kKind, int kBN, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                 const __grid_constant__ GemmArgs args) {
-  using C = Cfg<kBN>;
+  using C = Cfg<kBN, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
@@ -413,6 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int unit0 = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int unit_stride = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == 1 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -421,15 +539,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm->tfull[b], 1);
-      mbar_init(&sm->tempty[b], 128);
+      // 1-SM: every epilogue thread arrives; pair: one arrive per epilogue warp of
+      // both CTAs, on the leader's barrier.
+      mbar_init(&sm->tempty[b], kPair ? 2 * kEpiWarps : 32 * kEpiWarps);
     }
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&sm->tmem_base, C::kTmemCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&sm->tmem_base, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&sm->tmem_base, C::kTmemCols);
+      tmem_relinquish();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&tmA0);
       tma_prefetch_desc(&tmB0);
@@ -441,6 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = sm->tmem_base;
   const int k_blocks = args.num_seg * args.num_k_blk;
@@ -452,23 +578,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+      for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
         int m_blk, n_blk;
         tile_pos<kBN>(args, tile, m_blk, n_blk);
+        const int a_row = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM;
+        const int b_row = n_blk * kBN + args.b_row_off + (kPair ? static_cast<int>(rank) * (kBN / 2) : 0);
         for (int kb = 0; kb < k_blocks; ++kb) {
           const int seg = kb / args.num_k_blk;
           const int kk = kb - seg * args.num_k_blk;
           const CUtensorMap* mA = args.seg_a[seg] ? &tmA1 : &tmA0;
           const CUtensorMap* mB = args.seg_b[seg] ? &tmB1 : &tmB0;
-          if (!mbar_wait(&sm->empty[stage], phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
+          if (!mbar_wait<kPair>(&sm->empty[stage], phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
             ok = false;
             break;
           }
           uint8_t* sA = smem + stage * C::kStageBytes;
           uint8_t* sB = sA + kTileABytes;
-          mbar_arrive_expect_tx(&sm->full[stage], C::kStageBytes);
-          tma_load_2d(sA, mA, kk * kBK + args.a_k_off, m_blk * kBM, &sm->full[stage]);
-          tma_load_2d(sB, mB, kk * kBK + args.b_k_off, n_blk * kBN + args.b_row_off, &sm->full[stage]);
+          if (kPair) {
+            if (rank == 0) mbar_arrive_expect_tx(&sm->full[stage], 2 * C::kStageBytes);
+            const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
+            tma_load_2d_pair(sA, mA, kk * kBK + args.a_k_off, a_row, leader_full);
+            tma_load_2d_pair(sB, mB, kk * kBK + args.b_k_off, b_row, leader_full);
+          } else {
+            mbar_arrive_expect_tx(&sm->full[stage], C::kStageBytes);
+            tma_load_2d(sA, mA, kk * kBK + args.a_k_off, a_row, &sm->full[stage]);
+            tma_load_2d(sB, mB, kk * kBK + args.b_k_off, b_row, &sm->full[stage]);
+          }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) {
@@ -478,28 +613,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        // Let the copies already issued land before the CTA exits.
-        for (int s = 0; s < C::kStages; ++s)
-          if (issued_mask & (1u << s)) mbar_wait_drain(&sm->full[s], (issued_parity >> s) & 1u, args.timeout_ns);
+        if (kPair) {
+          // The copies' completion is counted on the leader's barriers, which this
+          // CTA cannot wait on: give anything in flight time to land.
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 10000000ull) {
+          }
+        } else {
+          // Let the copies already issued land before the CTA exits.
+          for (int s = 0; s < C::kStages; ++s)
+            if (issued_mask & (1u << s)) mbar_wait_drain(&sm->full[s], (issued_parity >> s) & 1u, args.timeout_ns);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(&sm->tempty[acc], acc_phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
+      for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
+        if (!mbar_wait<kPair>(&sm->tempty[acc], acc_phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
         for (int kb = 0; kb < k_blocks; ++kb) {
-          if (!mbar_wait(&sm->full[stage], phase, abort_flag, args.status, args.timeout_ns)) {
+          if (!mbar_wait<kPair>(&sm->full[stage], phase, abort_flag, args.status, args.timeout_ns)) {
             ok = false;
             break;
           }
@@ -508,43 +651,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t a_desc = umma_desc_sw128(a_addr);
           const uint64_t b_desc = umma_desc_sw128(a_addr + kTileABytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit(&sm->empty[stage]);
+          for (int k = 0; k < kBK / 16; ++k) {
+            if (kPair)
+              umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          if (kPair)
+            umma_commit_pair_both(&sm->empty[stage]);
+          else
+            umma_commit(&sm->empty[stage]);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&sm->tfull[acc]);
+        if (kPair)
+          umma_commit_pair_both(&sm->tfull[acc]);
+        else
+          umma_commit(&sm->tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
       // Every MMA this thread issued has completed once `drain` flips.
-      umma_commit(&sm->drain);
+      if (kPair)
+        umma_commit_pair_local(&sm->drain);
+      else
+        umma_commit(&sm->drain);
       mbar_wait_drain(&sm->drain, 0, args.timeout_ns);
     }
   } else {
     // -------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // tensor-memory lanes this warp may access
+    const int half = (warp - 2) >> 2;  // column half of the tile
     const int row_in_tile = quarter * 32 + lane;
+    // Pair: the leader's accumulator-empty barriers, as shared::cluster addresses.
+    const uint32_t leader_tempty0 = kPair ? mapa_shared(smem_u32(&sm->tempty[0]), 0) : 0u;
+    const uint32_t leader_tempty1 = kPair ? mapa_shared(smem_u32(&sm->tempty[1]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x) {
+    for (int tile = unit0; tile < args.num_tiles; tile += unit_stride) {
       int m_blk, n_blk;
       tile_pos<kBN>(args, tile, m_blk, n_blk);
-      if (!mbar_wait(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns)) break;
+      const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
+      const int n0 = n_blk * kBN;
+      if (kKind == kEpiUpdate) epi_update_prefetch<kBN>(args, j, n0, half);
+      // No early exit on another role's abort: every epilogue warp of the CTA takes
+      // the same decision here (the phase completes for all of them, or for none).
+      if (!mbar_wait<kPair>(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns, false)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
-      const int j = m_blk * kBM + row_in_tile;
-      const int n0 = n_blk * kBN;
       if (kKind == kEpiUpdate)
-        epi_update<kBN>(args, t_row, j, n0, n_blk);
+        epi_update<kBN>(args, t_row, j, n0, n_blk, half);
       else
-        epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk);
+        epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk, half);
       tc_fence_before();
-      mbar_arrive(&sm->tempty[acc]);
+      if (kPair) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
+      } else {
+        mbar_arrive(&sm->tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -552,36 +720,74 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (kPair) cluster_sync_all();  // the leader's MMAs into this CTA's tensor memory are done
   tc_fence_after();
   if (warp == 0) {
     __syncwarp();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if (kPair)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int kKind, int kBN>
+template <int kKind, int kBN, bool kPair>
 cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
-  using C = Cfg<kBN>;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kKind, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  using C = Cfg<kBN, kPair>;
+  auto* fn = gemm_kernel<kKind, kBN, kPair>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int grid = args.num_tiles < num_sms ? args.num_tiles : num_sms;
-  if (grid <= 0) return cudaSuccess;
-  gemm_kernel<kKind, kBN><<<grid, kThreads, C::kSmemBytes, stream>>>(m.a0, m.a1, m.b0, m.b1, args);
+  if (!kPair) {
+    const int grid = args.num_tiles < num_sms ? args.num_tiles : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    fn<<<grid, kThreads, C::kSmemBytes, stream>>>(m.a0, m.a1, m.b0, m.b1, args);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // A persistent grid must not exceed the clusters that can be resident at once
+  // (a pair needs two SMs of one GPC): queried once per device.
+  static int resident[64];  // 0: not yet known
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int max_pairs = (dev >= 0 && dev < 64) ? resident[dev] : 0;
+  if (max_pairs <= 0) {
+    e = cudaOccupancyMaxActiveClusters(&max_pairs, fn, &cfg);
+    if (e != cudaSuccess) return e;
+    if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) resident[dev] = max_pairs;
+  }
+  int pairs = args.num_tiles < num_sms / 2 ? args.num_tiles : num_sms / 2;
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  e = cudaLaunchKernelEx(&cfg, fn, m.a0, m.a1, m.b0, m.b1, args);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int kBN>
+template <int kBN, bool kPair>
 cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
   switch (kind) {
     case kEpiStore:
-      return launch_kind<kEpiStore, kBN>(m, args, num_sms, stream);
+      return launch_kind<kEpiStore, kBN, kPair>(m, args, num_sms, stream);
     case kEpiSumSq:
-      return launch_kind<kEpiSumSq, kBN>(m, args, num_sms, stream);
+      return launch_kind<kEpiSumSq, kBN, kPair>(m, args, num_sms, stream);
     case kEpiUpdate:
-      return launch_kind<kEpiUpdate, kBN>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdate, kBN, kPair>(m, args, num_sms, stream);
     case kEpiDotD:
-      return launch_kind<kEpiDotD, kBN>(m, args, num_sms, stream);
+      return launch_kind<kEpiDotD, kBN, kPair>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -591,8 +797,13 @@ cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int
 cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
                         cudaStream_t stream) {
   if (args.num_seg < 1 || args.num_seg > 3) return cudaErrorInvalidValue;
-  if (bn == 256) return launch_bn<256>(kind, maps, args, num_sms, stream);
-  if (bn == 128) return launch_bn<128>(kind, maps, args, num_sms, stream);
+  if (args.pair) {
+    // Pair tiles: 256 rows x 256 columns; B maps with 128-row boxes; no symmetric mode.
+    if (bn != 256 || args.symmetric) return cudaErrorInvalidValue;
+    return launch_bn<256, true>(kind, maps, args, num_sms, stream);
+  }
+  if (bn == 256) return launch_bn<256, false>(kind, maps, args, num_sms, stream);
+  if (bn == 128) return launch_bn<128, false>(kind, maps, args, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 
