@@ -156,6 +156,9 @@ struct Plan {
   // Gram-form update GEMM on 2-SM pair tiles (256 x 256, tcgen05 cta_group::2):
   // each SM stages 32 KB per K block instead of 48 KB, so six stages fit.
   bool pair_upd = true;
+  // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
+  // one sweep over all rows on the 4096 x 4096 layer.
+  int raster_upd = 8;
 };
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
@@ -475,6 +478,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       AR_CUDA_TRY(make_tmap_bf16(&m[q].b1, Hl, P.nb * in, in, b_box));
     }
     fill_grid(u, out, in, in, P.bn_upd, nseg_g, P.pair_upd);
+    u.raster_m = P.raster_upd;
     // (D_hi + D_lo)(H_hi + H_lo) ~ D_hi H_hi + D_lo H_hi + D_hi H_lo
     u.seg_a[0] = 0, u.seg_b[0] = 0;
     u.seg_a[1] = 1, u.seg_b[1] = 0;

@@ -191,8 +191,17 @@ __device__ __forceinline__ void store_pair8(const float* x, __nv_bfloat16* hi_ds
 template <int kBN>
 __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, int& n_blk) {
   if (!a.symmetric) {
-    m_blk = t % a.num_m_blk;
-    n_blk = t / a.num_m_blk;
+    if (a.raster_m <= 0 || a.raster_m >= a.num_m_blk) {
+      m_blk = t % a.num_m_blk;
+      n_blk = t / a.num_m_blk;
+      return;
+    }
+    const int per_group = a.raster_m * a.num_n_blk;
+    const int grp = t / per_group;
+    const int gm = min(a.raster_m, a.num_m_blk - grp * a.raster_m);  // m-blocks in this group
+    const int ti = t - grp * per_group;
+    m_blk = grp * a.raster_m + ti % gm;
+    n_blk = ti / gm;
     return;
   }
   for (n_blk = 0; n_blk < a.num_n_blk; ++n_blk) {
@@ -347,9 +356,18 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
   // sits in the output buffers until this epilogue overwrites it.
   bool better = false;
   if (row_ok && a.part_in) {
+    // Sum in index order; eight loads are in flight at a time.
     float L = 0.0f;
     const float* p = a.part_in + static_cast<int64_t>(j) * a.nparts;
-    for (int q = 0; q < a.nparts; ++q) L += p[q];
+    int q = 0;
+    for (; q + 8 <= a.nparts; q += 8) {
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = p[q + i];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) L += x[i];
+    }
+    for (; q < a.nparts; ++q) L += p[q];
     if (a.keep_best) {
       const float mean = L * a.inv_batch;
       better = mean < a.best_in[j];
