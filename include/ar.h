@@ -196,7 +196,9 @@ typedef struct {
   int32_t gemm_launches;     /* launches of each timed contraction (= iters) */
   int32_t kernel_launches;   /* every kernel this call launched */
   int32_t algo;              /* the ar_algo the call ran (DIRECT or GRAM) */
-  float setup_ms;            /* device time before the first step (transpose, Gram matrices) */
+  float setup_ms;            /* device time before the first step (group statistics, and the
+                                first block's transpose and Gram matrix; later blocks are
+                                prepared just before their first step) */
 } ar_tune_timing;
 
 /* ar_tune_layer, with CUDA events recorded on `stream` around each contraction;
@@ -207,6 +209,34 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
                               ar_tune_state* state, void* workspace, size_t ws_bytes,
                               uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
                               double* final_mse, void* stream, ar_tune_timing* timing);
+
+/* Device workspace of ar_tune_layer_host, in bytes (0 if the arguments are invalid):
+ * ar_tune_workspace_bytes() plus device copies of W, X and the outputs. */
+size_t ar_tune_host_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,
+                                    const ar_tune_params* params);
+
+/* ar_tune_layer from host buffers to host buffers: the end-to-end call.
+ * Same method, sources, results and errors as ar_tune_layer.  The differences:
+ *   W_host, X_host      host pointers (layouts as for ar_tune_layer); page-locked
+ *                       memory lets the copies overlap the work, pageable memory
+ *                       works but copies synchronously.
+ *   codes_host, scale_host, zp_host, loss_trace_host (may be NULL),
+ *   final_mse_host (may be NULL)   host outputs, written when the call returns.
+ *   workspace           device scratch of at least ar_tune_host_workspace_bytes(),
+ *                       256-byte aligned; owned by the caller.
+ * X goes to the device one calibration block at a time, on a stream of the call's
+ * own, in the order in which the block schedule first needs the blocks.  Each
+ * block's first kernel waits only for that block's copy, so the copy overlaps the
+ * Gram matrices and the first epoch's steps.  The call starts after the work
+ * already queued on `stream` and synchronises `stream` before it returns.  Device
+ * errors (AR_ETIMEOUT) are reported directly, as ar_tune_status would.  Tuning
+ * state is always fresh (no ar_tune_state).  Creates and destroys one stream and
+ * n_rows/batch_rows + 3 events per call; allocates no device memory. */
+ar_status ar_tune_layer_host(const void* W_host, ar_dtype w_dtype, int64_t out, int64_t in,
+                             const uint16_t* X_host, int64_t n_rows, const ar_tune_params* params,
+                             void* workspace, size_t ws_bytes, uint8_t* codes_host, float* scale_host,
+                             int32_t* zp_host, float* loss_trace_host, double* final_mse_host,
+                             void* stream);
 
 /* The calibration-block schedule ar_tune_layer follows (host only, no GPU):
  * blocks[i] = block index of step first + i, i < count, for n_blocks blocks.

@@ -28,6 +28,7 @@ ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
+           "ar_tune_host_workspace_bytes", "ar_tune_layer_host",
            "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static", "ar_dequant", "ar_linear",
            "ar_silu_mul")
 
@@ -82,6 +83,11 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(_TuneStateC), P, SZ, P, P, P, P, P, P]
     lib.ar_tune_layer_timed.restype = ctypes.c_int
     lib.ar_tune_layer_timed.argtypes = lib.ar_tune_layer.argtypes + [ctypes.POINTER(TuneTiming)]
+    lib.ar_tune_host_workspace_bytes.restype = SZ
+    lib.ar_tune_host_workspace_bytes.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.POINTER(TuneParams)]
+    lib.ar_tune_layer_host.restype = ctypes.c_int
+    lib.ar_tune_layer_host.argtypes = [P, ctypes.c_int, I64, I64, P, I64, ctypes.POINTER(TuneParams), P, SZ,
+                                       P, P, P, P, P, P]
     lib.ar_block_schedule.restype = ctypes.c_int
     lib.ar_block_schedule.argtypes = [I64, I64, I64, U64, P]
     lib.ar_tune_layer_static.restype = ctypes.c_int
@@ -330,15 +336,47 @@ def tune_status(workspace: torch.Tensor, stream=None) -> int:
     return int(_lib.ar_tune_status(_ptr(workspace), _stream(stream)))
 
 
-def tune_layer_host(W, X, params: TuneParams, device="cuda", want_final_mse: bool = True):
-    """Host arrays in, host arrays out: copies W and X to the device (from pinned
-    memory when given), tunes, and copies codes, scales, zero-points, the loss
-    trace and the final MSE back.  W: fp32 or bf16 CPU tensor; X: bf16 CPU tensor."""
-    Wd = W.to(device, non_blocking=True)
-    Xd = X.to(device, non_blocking=True)
-    res = tune_layer(Wd, Xd, params, want_final_mse=want_final_mse)
-    out = dict(codes=res.codes.to("cpu"), scale=res.scale.to("cpu"), zero_point=res.zero_point.to("cpu"),
-               loss_trace=res.loss_trace.to("cpu") if res.loss_trace is not None else None,
-               final_mse=float(res.final_mse.item()) if res.final_mse is not None else None)
-    _check(tune_status(res.workspace), "ar_tune_layer (device)")
-    return out
+def tune_layer_host(W, X, params: TuneParams, device="cuda", want_final_mse: bool = True, workspace=None,
+                    stream=None):
+    """Host arrays in, host arrays out, through ar_tune_layer_host: X goes to the
+    device block by block, overlapped with the work.  W: fp32 or bf16 CPU tensor;
+    X: bf16 CPU tensor [n_rows, in] (page-locked memory lets the copies overlap;
+    other memory is pinned here first, which costs a host copy).  ``workspace`` may
+    pass a device uint8 tensor of tune_host_workspace_bytes() bytes to reuse."""
+    if W.device.type != "cpu" or X.device.type != "cpu":
+        raise ValueError("tune_layer_host takes CPU tensors")
+    if X.dtype != torch.bfloat16:
+        raise TypeError("X must be bf16")
+    W = W.contiguous()
+    X = X.contiguous()
+    if not X.is_pinned():
+        X = X.pin_memory()
+    if not W.is_pinned():
+        W = W.pin_memory()
+    out, inn = W.shape
+    n_rows = X.shape[0]
+    if X.shape[1] != inn:
+        raise ValueError("X must be [n_rows, in]")
+    wdt = _wdtype(W)
+    need = tune_host_workspace_bytes(out, inn, n_rows, params, wdt)
+    if need == 0:
+        raise ArError(AR_EINVAL, "ar_tune_host_workspace_bytes")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    G = max(_groups(inn, params.group_size), 1)
+    codes = torch.empty((out, inn), dtype=torch.uint8, pin_memory=True)
+    scale = torch.empty((out, G), dtype=torch.float32, pin_memory=True)
+    zp = torch.empty((out, G), dtype=torch.int32, pin_memory=True)
+    trace = torch.empty((max(params.iters, 1),), dtype=torch.float32, pin_memory=True)
+    mse = torch.empty((1,), dtype=torch.float64, pin_memory=True) if want_final_mse else None
+    with torch.cuda.device(workspace.device):
+        _check(_lib.ar_tune_layer_host(_ptr(W), wdt, out, inn, _ptr(X), n_rows, ctypes.byref(params),
+                                       _ptr(workspace), workspace.numel(), _ptr(codes), _ptr(scale), _ptr(zp),
+                                       _ptr(trace), _ptr(mse), _stream(stream)), "ar_tune_layer_host")
+    return dict(codes=codes, scale=scale, zero_point=zp, loss_trace=trace[:params.iters],
+                final_mse=float(mse.item()) if mse is not None else None)
+
+
+def tune_host_workspace_bytes(out: int, inn: int, n_rows: int, params: TuneParams, w_dtype: int = AR_BF16) -> int:
+    """Device workspace bytes of tune_layer_host (ar_tune_host_workspace_bytes)."""
+    return int(_lib.ar_tune_host_workspace_bytes(out, inn, n_rows, w_dtype, ctypes.byref(params)))

@@ -287,10 +287,12 @@ struct EventTimer {
   }
 };
 
+// block_ready (optional, one event per calibration block): the stream waits for
+// block b's event before the first kernel that reads block b of X.
 ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X, int64_t n_rows,
                     const ar_tune_params* p, ar_tune_state* state, void* workspace, size_t ws_bytes,
                     uint8_t* codes, float* scale, int32_t* zp, float* loss_trace, double* final_mse,
-                    void* stream, EventTimer* timer) {
+                    void* stream, EventTimer* timer, const cudaEvent_t* block_ready = nullptr) {
   const ar_status chk = check_tune_args(out, in, n_rows, p);
   if (chk != AR_OK) return chk;
   if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
@@ -405,12 +407,49 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   const int nseg_d = P.split ? 2 : 1;
   const int nseg_g = P.split ? 3 : 1;
   const std::vector<int64_t> sched = block_schedule(P.nb, p->start_step, iters, p->seed);
-  const bool need_xt = iters > 0 || (gram && final_mse);
-
-  if (need_xt) {
-    AR_CUDA_TRY(launch_transpose_bf16(X, n_rows, in, Xt, st));
-    ++launches;
+  // Gram matrices H_b = X_b^T X_b, as bf16 pairs at rows b*in .. b*in + in.
+  GemmMaps gram_maps{};
+  GemmArgs h;
+  if (gram) {
+    AR_CUDA_TRY(make_tmap_bf16(&gram_maps.a0, Xt, in, n_rows, kBM));
+    AR_CUDA_TRY(make_tmap_bf16(&gram_maps.b0, Xt, in, n_rows, P.bn_gram));
+    gram_maps.a1 = gram_maps.a0;
+    gram_maps.b1 = gram_maps.b0;
+    fill_grid(h, in, in, B, P.bn_gram, 1);
+    h.symmetric = 1;  // H_b = X_b^T X_b: compute the tiles reaching the upper triangle
+    h.num_tiles = 0;
+    for (int nn = 0; nn < h.num_n_blk; ++nn)
+      h.num_tiles += static_cast<int>(std::min<int64_t>(h.num_m_blk, cdiv((nn + 1) * int64_t(P.bn_gram), kBM)));
+    h.timeout_ns = timeout_ns;
+    h.status = status;
+    h.C_hi = H(L.H_hi);
+    h.C_lo = P.split ? H(L.H_lo) : nullptr;
+    h.ldc = in;
+    h.diag_out = F(L.Hdiag);
   }
+  // Each calibration block is transposed into its columns of Xt (and, in the Gram
+  // form, its Gram matrix is made) just before the first step that uses it.  With
+  // block_ready events, the block's copy to the device is awaited first.
+  std::vector<char> have_block(static_cast<size_t>(P.nb), 0), waited_block(static_cast<size_t>(P.nb), 0);
+  auto wait_block = [&](int64_t b) -> cudaError_t {
+    if (!block_ready || waited_block[b]) return cudaSuccess;
+    waited_block[b] = 1;
+    return cudaStreamWaitEvent(st, block_ready[b], 0);
+  };
+  auto ensure_block = [&](int64_t b) -> cudaError_t {
+    if (have_block[b]) return cudaSuccess;
+    have_block[b] = 1;
+    cudaError_t e = wait_block(b);
+    if (e != cudaSuccess) return e;
+    e = launch_transpose_bf16(X + b * B * in, B, in, Xt + b * B, n_rows, st);
+    ++launches;
+    if (e != cudaSuccess || !gram) return e;
+    h.a_k_off = static_cast<int>(b * B);
+    h.b_k_off = static_cast<int>(b * B);
+    h.c_row_off = b * in;
+    ++launches;
+    return launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
+  };
 
   // The update epilogue's common arguments.
   GemmArgs u;
@@ -442,32 +481,6 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     // ---------------------------------------------------------- Gram form
     __nv_bfloat16* Hh = H(L.H_hi);
     __nv_bfloat16* Hl = H(L.H_lo);
-    {  // H_b = X_b^T X_b for every block, as a bf16 pair, rows b*in .. b*in + in
-      GemmMaps m{};
-      AR_CUDA_TRY(make_tmap_bf16(&m.a0, Xt, in, n_rows, kBM));
-      AR_CUDA_TRY(make_tmap_bf16(&m.b0, Xt, in, n_rows, P.bn_gram));
-      m.a1 = m.a0;
-      m.b1 = m.b0;
-      GemmArgs h;
-      fill_grid(h, in, in, B, P.bn_gram, 1);
-      h.symmetric = 1;  // H_b = X_b^T X_b: compute the tiles reaching the upper triangle
-      h.num_tiles = 0;
-      for (int n = 0; n < h.num_n_blk; ++n)
-        h.num_tiles += static_cast<int>(std::min<int64_t>(h.num_m_blk, cdiv((n + 1) * int64_t(P.bn_gram), kBM)));
-      h.timeout_ns = timeout_ns;
-      h.status = status;
-      h.C_hi = Hh;
-      h.C_lo = P.split ? Hl : nullptr;
-      h.ldc = in;
-      h.diag_out = F(L.Hdiag);
-      for (int64_t b = 0; b < P.nb; ++b) {
-        h.a_k_off = static_cast<int>(b * B);
-        h.b_k_off = static_cast<int>(b * B);
-        h.c_row_off = b * in;
-        AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_gram, m, h, sms, st));
-        ++launches;
-      }
-    }
     GemmMaps m[2]{};  // per parity of t: A = D_t
     // 2-SM pair tiles: each CTA of a pair stages half of the tile's B rows.
     const uint32_t b_box = P.pair_upd ? P.bn_upd / 2 : P.bn_upd;
@@ -503,6 +516,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       u.rowloss = t > 0 ? rowloss + static_cast<int64_t>(t - 1) * out : nullptr;
       u.best_in = best_cur;
       u.best_out = best_next;
+      AR_CUDA_TRY(ensure_block(sched[t]));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
       AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
       if (timer) {
@@ -576,6 +590,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     for (int t = 0; t < iters; ++t) {
       const int64_t b0 = sched[t] * B;
       r.b_row_off = static_cast<int>(b0);
+      AR_CUDA_TRY(ensure_block(sched[t]));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
@@ -635,6 +650,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     f.part = part[0];
     if (gram) {
       // sum_j D_j (sum_b H_b) D_j^T over all calibration rows
+      for (int64_t b = 0; b < P.nb; ++b) AR_CUDA_TRY(ensure_block(b));
       AR_CUDA_TRY(launch_gram_sum(H(L.H_hi), P.split ? H(L.H_lo) : nullptr, static_cast<int>(P.nb),
                                   in * in, H(L.Hs_hi), P.split ? H(L.Hs_lo) : nullptr, st));
       AR_CUDA_TRY(launch_diag_sum(F(L.Hdiag), static_cast<int>(P.nb), in, F(L.Hdsum), st));
@@ -653,6 +669,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       AR_CUDA_TRY(launch_gemm(kEpiDotD, P.bn_fin, m, f, sms, st));
       launches += 2;
     } else {
+      for (int64_t b = 0; b < P.nb; ++b) AR_CUDA_TRY(wait_block(b));
       AR_CUDA_TRY(make_tmap_bf16(&m.a0, D_hi, out, in, kBM));
       AR_CUDA_TRY(make_tmap_bf16(&m.a1, D_lo, out, in, kBM));
       AR_CUDA_TRY(make_tmap_bf16(&m.b0, X, n_rows, in, P.bn_fin));
@@ -795,6 +812,142 @@ ar_status ar_block_schedule(int64_t n_blocks, int64_t first, int64_t count, uint
   const std::vector<int64_t> s = block_schedule(n_blocks, first, count, seed);
   for (int64_t i = 0; i < count; ++i) blocks[i] = s[static_cast<size_t>(i)];
   return AR_OK;
+}
+
+// ---------------------------------------------------------------------------
+// ar_tune_layer_host: host buffers in and out, copies overlapped with the work.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// Device workspace of the host entry point: the tuning workspace, then device
+// copies of W, X and the outputs.
+struct HostLayout {
+  size_t tune, W, X, codes, scale, zp, trace, mse, total;
+};
+
+HostLayout make_host_layout(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype, const ar_tune_params* p) {
+  HostLayout H{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  const int64_t G = in / group_of(in, p->group_size);
+  H.tune = take(ar_tune_workspace_bytes(out, in, n_rows, p));
+  H.W = take(static_cast<size_t>(out) * in * (w_dtype == AR_BF16 ? 2 : 4));
+  H.X = take(static_cast<size_t>(n_rows) * in * 2);
+  H.codes = take(static_cast<size_t>(out) * in);
+  H.scale = take(static_cast<size_t>(out) * G * 4);
+  H.zp = take(static_cast<size_t>(out) * G * 4);
+  H.trace = take(static_cast<size_t>(std::max(p->iters, 1)) * 4);
+  H.mse = take(8);
+  H.total = off;
+  return H;
+}
+
+// The copy stream and per-block events of one call; on every exit path the copies
+// still in flight finish before the host buffers are handed back.
+struct CopyPipeline {
+  cudaStream_t copy = nullptr;
+  cudaEvent_t start = nullptr, w_done = nullptr, all_done = nullptr;
+  std::vector<cudaEvent_t> block;
+  bool create(size_t nblocks) {
+    if (cudaStreamCreateWithFlags(&copy, cudaStreamNonBlocking) != cudaSuccess) return false;
+    for (cudaEvent_t* e : {&start, &w_done, &all_done})
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    block.assign(nblocks, nullptr);
+    for (auto& e : block)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~CopyPipeline() {
+    if (copy) {
+      cudaStreamSynchronize(copy);
+      cudaStreamDestroy(copy);
+    }
+    for (cudaEvent_t e : {start, w_done, all_done})
+      if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : block)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+}  // namespace
+
+size_t ar_tune_host_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,
+                                    const ar_tune_params* p) {
+  if (w_dtype != AR_F32 && w_dtype != AR_BF16) return 0;
+  if (ar_tune_workspace_bytes(out, in, n_rows, p) == 0) return 0;
+  return make_host_layout(out, in, n_rows, w_dtype, p).total;
+}
+
+ar_status ar_tune_layer_host(const void* W_host, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X_host,
+                             int64_t n_rows, const ar_tune_params* p, void* workspace, size_t ws_bytes,
+                             uint8_t* codes_host, float* scale_host, int32_t* zp_host, float* loss_trace_host,
+                             double* final_mse_host, void* stream) {
+  const ar_status chk = check_tune_args(out, in, n_rows, p);
+  if (chk != AR_OK) return chk;
+  if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
+  if (out == 0 || in == 0) return AR_OK;
+  if (!W_host || !X_host || !workspace || !codes_host || !scale_host || !zp_host) return AR_EINVAL;
+  if (!aligned(workspace, 256)) return AR_EINVAL;
+  const HostLayout HL = make_host_layout(out, in, n_rows, w_dtype, p);
+  if (ws_bytes < HL.total) return AR_ENOMEM;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t B = p->batch_rows;
+  const int64_t nb = n_rows / B;
+  const int64_t G = in / group_of(in, p->group_size);
+  const size_t w_bytes = static_cast<size_t>(out) * in * (w_dtype == AR_BF16 ? 2 : 4);
+  const size_t block_bytes = static_cast<size_t>(B) * in * 2;
+  uint16_t* Xd = reinterpret_cast<uint16_t*>(ws + HL.X);
+
+  CopyPipeline cp;
+  if (!cp.create(static_cast<size_t>(nb))) return AR_ECUDA;
+  // Copies start after the work already queued on the caller's stream; blocks go
+  // in the order the schedule first needs them.
+  AR_CUDA_TRY(cudaEventRecord(cp.start, st));
+  AR_CUDA_TRY(cudaStreamWaitEvent(cp.copy, cp.start, 0));
+  AR_CUDA_TRY(cudaMemcpyAsync(ws + HL.W, W_host, w_bytes, cudaMemcpyHostToDevice, cp.copy));
+  AR_CUDA_TRY(cudaEventRecord(cp.w_done, cp.copy));
+  std::vector<char> queued(static_cast<size_t>(nb), 0);
+  std::vector<int64_t> order;
+  order.reserve(static_cast<size_t>(nb));
+  for (int64_t b : block_schedule(nb, p->start_step, std::min<int64_t>(p->iters, nb), p->seed))
+    if (!queued[b]) {
+      queued[b] = 1;
+      order.push_back(b);
+    }
+  for (int64_t b = 0; b < nb; ++b)
+    if (!queued[b]) order.push_back(b);
+  for (int64_t b : order) {
+    AR_CUDA_TRY(cudaMemcpyAsync(Xd + b * B * in, X_host + b * B * in, block_bytes, cudaMemcpyHostToDevice,
+                                cp.copy));
+    AR_CUDA_TRY(cudaEventRecord(cp.block[b], cp.copy));
+  }
+  AR_CUDA_TRY(cudaEventRecord(cp.all_done, cp.copy));
+
+  AR_CUDA_TRY(cudaStreamWaitEvent(st, cp.w_done, 0));
+  uint8_t* codes = ws + HL.codes;
+  float* scale = reinterpret_cast<float*>(ws + HL.scale);
+  int32_t* zp = reinterpret_cast<int32_t*>(ws + HL.zp);
+  float* trace = loss_trace_host ? reinterpret_cast<float*>(ws + HL.trace) : nullptr;
+  double* mse = final_mse_host ? reinterpret_cast<double*>(ws + HL.mse) : nullptr;
+  const ar_status s = tune_impl(ws + HL.W, w_dtype, out, in, Xd, n_rows, p, nullptr, ws + HL.tune,
+                                HL.W - HL.tune, codes, scale, zp, trace, mse, stream, nullptr, cp.block.data());
+  if (s != AR_OK) return s;
+  AR_CUDA_TRY(cudaStreamWaitEvent(st, cp.all_done, 0));
+  AR_CUDA_TRY(cudaMemcpyAsync(codes_host, codes, static_cast<size_t>(out) * in, cudaMemcpyDeviceToHost, st));
+  AR_CUDA_TRY(cudaMemcpyAsync(scale_host, scale, static_cast<size_t>(out) * G * 4, cudaMemcpyDeviceToHost, st));
+  AR_CUDA_TRY(cudaMemcpyAsync(zp_host, zp, static_cast<size_t>(out) * G * 4, cudaMemcpyDeviceToHost, st));
+  if (trace && p->iters > 0)
+    AR_CUDA_TRY(cudaMemcpyAsync(loss_trace_host, trace, static_cast<size_t>(p->iters) * 4, cudaMemcpyDeviceToHost,
+                                st));
+  if (mse) AR_CUDA_TRY(cudaMemcpyAsync(final_mse_host, mse, 8, cudaMemcpyDeviceToHost, st));
+  return ar_tune_status(ws + HL.tune, stream);
 }
 
 ar_status ar_tune_status(const void* workspace, void* stream) {

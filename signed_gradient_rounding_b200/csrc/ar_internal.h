@@ -35,7 +35,9 @@ cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream);
 cudaError_t launch_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits, int32_t* packed,
                         cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t stream);
-cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt,
+// Xt[c * ld_t + r] = X[r * cols + c] for r < rows, c < cols (a row block of X
+// into the matching columns of a wider Xt when ld_t > rows).
+cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt, int64_t ld_t,
                                   cudaStream_t stream);
 // loss_trace[t] = sum_j rowloss[t*out + j] / (batch_rows * out), t < iters (fixed order).
 cudaError_t launch_loss_trace(const float* rowloss, int64_t out, int iters, int64_t batch_rows,

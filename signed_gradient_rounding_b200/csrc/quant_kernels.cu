@@ -104,15 +104,16 @@ __global__ void fill_f32_kernel(float* p, int64_t n, float v) {
     p[i] = v;
 }
 
-// 64 x 64 tiles through shared memory; 256 threads.  Full tiles move 16-byte
-// vectors both ways (rows and cols multiples of 8 keep them aligned); the tile's
-// ragged edges fall back to single elements.
+// Xt[c * ld_t + r] = X[r * cols + c].  64 x 64 tiles through shared memory; 256
+// threads.  Full tiles move 16-byte vectors both ways (rows, cols and ld_t
+// multiples of 8 keep them aligned); the tile's ragged edges fall back to single
+// elements.
 __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
-                                      uint16_t* __restrict__ Xt) {
+                                      uint16_t* __restrict__ Xt, int64_t ld_t) {
   __shared__ __align__(16) uint16_t tile[64][72];
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 64;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
-  const bool full = (r0 + 64 <= rows) && (c0 + 64 <= cols) && (rows % 8 == 0) && (cols % 8 == 0);
+  const bool full = (r0 + 64 <= rows) && (c0 + 64 <= cols) && (rows % 8 == 0) && (cols % 8 == 0) && (ld_t % 8 == 0);
   if (full) {
     for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 rows x 8 vectors
       const int r = v >> 3, c8 = (v & 7) * 8;
@@ -129,7 +130,7 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t ro
       o.y = e[2] | (uint32_t(e[3]) << 16);
       o.z = e[4] | (uint32_t(e[5]) << 16);
       o.w = e[6] | (uint32_t(e[7]) << 16);
-      *reinterpret_cast<uint4*>(Xt + (c0 + c) * rows + r0 + r8) = o;
+      *reinterpret_cast<uint4*>(Xt + (c0 + c) * ld_t + r0 + r8) = o;
     }
     return;
   }
@@ -142,7 +143,7 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t ro
   __syncthreads();
   for (int i = ty; i < 64; i += 4) {
     const int64_t c = c0 + i, r = r0 + tx;
-    if (r < rows && c < cols) Xt[c * rows + r] = tile[tx][i];
+    if (r < rows && c < cols) Xt[c * ld_t + r] = tile[tx][i];
   }
 }
 
@@ -343,10 +344,11 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t strea
   return cudaGetLastError();
 }
 
-cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt,
+cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt, int64_t ld_t,
                                   cudaStream_t stream) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>((cols + 63) / 64), static_cast<unsigned>((rows + 63) / 64));
-  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, Xt);
+  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, Xt, ld_t);
   return cudaGetLastError();
 }
 

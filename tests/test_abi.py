@@ -99,3 +99,26 @@ def test_block_schedule_matches_oracle(ar, n_blocks, seed):
     first = min(11, total // 2)
     assert ar.block_schedule(n_blocks, first, total - first, seed) == \
         oracle.block_schedule(n_blocks, total, seed)[first:]
+
+
+def test_host_entry_validation(ar):
+    """ar_tune_layer_host checks its arguments before it creates a stream or copies."""
+    lib = ar.lib
+    dummy = ctypes.c_void_p(4096)
+    p = ar.make_params(batch_rows=512, group_size=64)
+    need = lib.ar_tune_host_workspace_bytes(64, 256, 1024, 1, ctypes.byref(p))
+    assert need > lib.ar_tune_workspace_bytes(64, 256, 1024, ctypes.byref(p)) + 64 * 256 * 2 + 1024 * 256 * 2
+    assert lib.ar_tune_host_workspace_bytes(64, 256, 1024, 7, ctypes.byref(p)) == 0      # bad W dtype
+
+    def call(out, inn, n, ws_bytes=1 << 40, W=dummy, codes=dummy, **kw):
+        q = ar.make_params(**kw)
+        return lib.ar_tune_layer_host(W, 1, out, inn, dummy, n, ctypes.byref(q), dummy, ws_bytes,
+                                      codes, dummy, dummy, None, None, None)
+
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, bits=5) == ar.AR_EINVAL
+    assert call(64, 256, 1000, batch_rows=512, group_size=64) == ar.AR_EINVAL
+    assert call(64, 256, 1024, W=None, batch_rows=512, group_size=64) == ar.AR_EINVAL
+    assert call(64, 256, 1024, codes=None, batch_rows=512, group_size=64) == ar.AR_EINVAL
+    assert call(64, 256, 1024, batch_rows=512, group_size=16) == ar.AR_EUNSUPPORTED
+    assert call(64, 256, 1024, ws_bytes=need - 1, batch_rows=512, group_size=64) == ar.AR_ENOMEM
+    assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK
