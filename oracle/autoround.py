@@ -150,6 +150,44 @@ def rtn(W, bits: int, group_size: int, sym: bool):
     return fq.q.astype(np.uint8), s, zp.astype(np.int32), fq.Wq
 
 
+MSE_GRID = 51   # clip ratios p_i = (100 - i) / 100, i = 0 .. 50: 1.00 down to 0.50
+
+
+def mse_init(W, group_size: int, bits: int, sym: bool):
+    """Initial clip factors by an MSE grid search ("[llm-compressor] AutoRound ...",
+    ``_init_scale_zp``: "Min-Max or MSE").
+
+    The page names the option without spelling it out.  Reading: per group, try a
+    common clip ratio p for both factors (alpha = beta = p; symmetric: alpha = p) on
+    the grid p_i = fp32(100 - i) / fp32(100), i = 0 .. 50, i.e. 1.00 down to 0.50
+    (the clip factors' range), and keep the p whose round-to-nearest weights
+    (V = 0) have the smallest squared error sum_k (W'_k - W_k)^2.  The element
+    arithmetic is the fp32 quantiser's; each square is exact in fp64 and the sum
+    runs in fp64 over k in index order; the first minimum along the grid wins, so
+    a tie keeps the wider range.
+
+    Returns (p fp32 [out, G], err fp64 [out, G]: the squared error at p).
+    """
+    W = _to_f32(W)
+    out, inn = W.shape
+    g = _group(inn, group_size)
+    wmin, wmax = group_minmax(W, g)
+    zeros = np.zeros_like(W)
+    best_p = np.ones(wmin.shape, dtype=F32)
+    best_e = np.full(wmin.shape, np.inf)
+    for i in range(MSE_GRID):
+        p = F32(100 - i) / F32(100)
+        a = np.full(wmin.shape, p, dtype=F32)
+        sc, zp = scale_zero_point(wmin, wmax, a, a, bits, sym)
+        d = fake_quant(W, zeros, sc, zp, g, bits).Wq - W              # fp32
+        d2 = d.astype(F64).reshape(out, inn // g, g) ** 2             # exact squares
+        e = np.cumsum(d2, axis=2)[:, :, -1]                            # sequential sum over k
+        better = e < best_e
+        best_e = np.where(better, e, best_e)
+        best_p = np.where(better, p, best_p).astype(F32)
+    return best_p, best_e
+
+
 # --------------------------------------------------------------------------
 # backward: straight-through derivatives of W' with respect to V, alpha, beta
 # --------------------------------------------------------------------------
@@ -236,7 +274,7 @@ class TuneResult:
 def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
                minmax_lr: float, batch_rows: int, seed: int, minmax_shrink: float = 1.0,
                keep_best: bool = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
-               best0=None, want_final_mse: bool = True) -> TuneResult:
+               best0=None, want_final_mse: bool = True, init: str = "minmax") -> TuneResult:
     """SignSGD tuning of one linear layer.
 
     "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END": per step,
@@ -265,6 +303,10 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     ``start_step`` continues the block schedule of an interrupted run, with the
     live state passed in V0 / alpha0 / beta0 and the best state in
     best0 = (best_loss, V_best, alpha_best, beta_best).
+
+    ``init``: "minmax" starts the clip factors at ``minmax_shrink`` (the page's
+    ``minmax_shrink`` parameter); "mse" starts each group at its ``mse_init``
+    ratio (minmax_shrink is then unused).
     """
     W = _to_f32(W)
     out, inn = W.shape
@@ -280,9 +322,12 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     mlr32 = F32(lr if minmax_lr < 0 else minmax_lr)
 
     wmin, wmax = group_minmax(W, g)
+    if init not in ("minmax", "mse"):
+        raise ValueError("init must be 'minmax' or 'mse'")
+    p0 = mse_init(W, g, bits, sym)[0] if init == "mse" else np.full(wmin.shape, F32(minmax_shrink))
     V = np.zeros_like(W) if V0 is None else _to_f32(V0).copy()
-    alpha = np.full(wmin.shape, F32(minmax_shrink)) if alpha0 is None else _to_f32(alpha0).copy()
-    beta = np.full(wmin.shape, F32(minmax_shrink)) if beta0 is None else _to_f32(beta0).copy()
+    alpha = p0.copy() if alpha0 is None else _to_f32(alpha0).copy()
+    beta = p0.copy() if beta0 is None else _to_f32(beta0).copy()
     if best0 is None:
         best_loss = np.full(out, np.inf)
         V_best, a_best, b_best = V.copy(), alpha.copy(), beta.copy()
