@@ -93,7 +93,21 @@ typedef struct {
                             (hi = bf16(x), lo = bf16(x - hi): ~16 significant bits);
                             0: single bf16 (faster, the tuning trajectory drifts
                             further from an exact evaluation) */
+  int32_t init;          /* ar_init: how alpha and beta start (0: min-max) */
 } ar_tune_params;
+
+/* Initial clip factors ("[llm-compressor] AutoRound ...", "on_event with
+ * SEQUENTIAL_EPOCH_END": _init_scale_zp is "Min-Max or MSE").
+ *   AR_INIT_MINMAX: alpha = beta = minmax_shrink for every group.
+ *   AR_INIT_MSE:    per group, the common ratio p = alpha = beta (symmetric: alpha)
+ *                   on the grid fp32(100 - i) / fp32(100), i = 0 .. 50 (1.00 down to
+ *                   0.50), whose round-to-nearest weights have the smallest squared
+ *                   error sum_k (W'_k - W_k)^2.  The elements use ar_fake_quant's fp32
+ *                   arithmetic; the sum runs in fp64 over the group's columns in
+ *                   order; the first minimum along the grid wins.  minmax_shrink is
+ *                   not used.  (The page names the option; this grid search is the
+ *                   library's reading of it.) */
+typedef enum { AR_INIT_MINMAX = 0, AR_INIT_MSE = 1 } ar_init;
 
 /* Optional caller-owned tuning state (device memory, fp32).  Lets a caller
  * inspect the learned variables, and resume: a run of k steps followed by a run

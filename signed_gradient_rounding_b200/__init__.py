@@ -24,6 +24,8 @@ AR_OK, AR_EINVAL, AR_EUNSUPPORTED, AR_ENOMEM, AR_ECUDA, AR_ETIMEOUT = range(6)
 AR_F32, AR_BF16 = 0, 1
 AR_ALGO_AUTO, AR_ALGO_DIRECT, AR_ALGO_GRAM = 0, 1, 2
 ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
+AR_INIT_MINMAX, AR_INIT_MSE = 0, 1
+INITS = {"minmax": AR_INIT_MINMAX, "mse": AR_INIT_MSE}
 
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
@@ -44,7 +46,7 @@ class TuneParams(ctypes.Structure):
                 ("iters", ctypes.c_int32), ("lr", ctypes.c_float), ("minmax_lr", ctypes.c_float),
                 ("minmax_shrink", ctypes.c_float), ("keep_best", ctypes.c_int32),
                 ("batch_rows", ctypes.c_int64), ("seed", ctypes.c_uint64), ("start_step", ctypes.c_int64),
-                ("algo", ctypes.c_int32), ("split", ctypes.c_int32)]
+                ("algo", ctypes.c_int32), ("split", ctypes.c_int32), ("init", ctypes.c_int32)]
 
 
 class _TuneStateC(ctypes.Structure):
@@ -233,11 +235,13 @@ def silu_mul(a: torch.Tensor, b: torch.Tensor, stream=None) -> torch.Tensor:
 
 
 def make_params(bits=4, group_size=128, sym=False, iters=200, lr=0.005, minmax_lr=-1.0, minmax_shrink=1.0,
-                keep_best=True, batch_rows=16384, seed=0, start_step=0, algo="auto", split=True) -> TuneParams:
-    """ar_tune_params; algo is "auto", "direct" or "gram" (see ar_algo in include/ar.h)."""
+                keep_best=True, batch_rows=16384, seed=0, start_step=0, algo="auto", split=True,
+                init="minmax") -> TuneParams:
+    """ar_tune_params; algo is "auto", "direct" or "gram" (ar_algo in include/ar.h);
+    init is "minmax" or "mse" (ar_init)."""
     return TuneParams(bits, group_size, int(sym), iters, lr, minmax_lr, minmax_shrink, int(keep_best),
                       batch_rows, seed, start_step, ALGOS[algo] if isinstance(algo, str) else int(algo),
-                      int(split))
+                      int(split), INITS[init] if isinstance(init, str) else int(init))
 
 
 def tune_workspace_bytes(out: int, inn: int, n_rows: int, params: TuneParams) -> int:

@@ -132,6 +132,7 @@ ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune
   if (!(p->minmax_shrink > 0.0f) || !isfinite(p->minmax_shrink)) return AR_EINVAL;
   if (p->start_step < 0) return AR_EINVAL;
   if (p->algo < AR_ALGO_AUTO || p->algo > AR_ALGO_GRAM) return AR_EINVAL;
+  if (p->init != AR_INIT_MINMAX && p->init != AR_INIT_MSE) return AR_EINVAL;
   if (out == 0 || in == 0) return AR_OK;
   if (!group_ok(in, p->group_size)) return AR_EINVAL;
   if (p->batch_rows <= 0 || n_rows < p->batch_rows || n_rows % p->batch_rows != 0) return AR_EINVAL;
@@ -374,12 +375,21 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   if (init_state) {
     AR_CUDA_TRY(cudaMemsetAsync(Vb[0], 0, elems * 4, st));
     AR_CUDA_TRY(cudaMemsetAsync(V_best, 0, elems * 4, st));
-    AR_CUDA_TRY(launch_fill_f32(ab[0], groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(bb[0], groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(alpha_best, groups, p->minmax_shrink, st));
-    AR_CUDA_TRY(launch_fill_f32(beta_best, groups, p->minmax_shrink, st));
+    if (p->init == AR_INIT_MSE) {
+      AR_CUDA_TRY(launch_mse_init(W, w_dtype == AR_BF16, out, in, static_cast<int>(P.g), p->bits, p->sym != 0,
+                                  ab[0], bb[0], st));
+      AR_CUDA_TRY(cudaMemcpyAsync(alpha_best, ab[0], groups * 4, cudaMemcpyDeviceToDevice, st));
+      AR_CUDA_TRY(cudaMemcpyAsync(beta_best, bb[0], groups * 4, cudaMemcpyDeviceToDevice, st));
+      launches += 1;
+    } else {
+      AR_CUDA_TRY(launch_fill_f32(ab[0], groups, p->minmax_shrink, st));
+      AR_CUDA_TRY(launch_fill_f32(bb[0], groups, p->minmax_shrink, st));
+      AR_CUDA_TRY(launch_fill_f32(alpha_best, groups, p->minmax_shrink, st));
+      AR_CUDA_TRY(launch_fill_f32(beta_best, groups, p->minmax_shrink, st));
+      launches += 4;
+    }
     AR_CUDA_TRY(launch_fill_f32(best_loss, out, INFINITY, st));
-    launches += 5;
+    launches += 1;
   }
 
   // Group statistics of W and the first step's D = W' - W.
@@ -697,7 +707,7 @@ using namespace ar;
 
 extern "C" {
 
-const char* ar_version(void) { return "ar 0.2.0 sm_100a"; }
+const char* ar_version(void) { return "ar 0.3.0 sm_100a"; }
 
 const char* ar_status_string(ar_status s) {
   switch (s) {

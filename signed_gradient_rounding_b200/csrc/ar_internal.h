@@ -35,6 +35,10 @@ cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream);
 cudaError_t launch_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits, int32_t* packed,
                         cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t stream);
+// AR_INIT_MSE: per group, the clip ratio of the grid 1.00 .. 0.50 with the smallest
+// round-to-nearest squared error, written to alpha and beta [out, in/g].
+cudaError_t launch_mse_init(const void* W, int w_bf16, int64_t out, int64_t in, int g, int bits, bool sym,
+                            float* alpha, float* beta, cudaStream_t stream);
 // Xt[c * ld_t + r] = X[r * cols + c] for r < rows, c < cols (a row block of X
 // into the matching columns of a wider Xt when ld_t > rows).
 cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt, int64_t ld_t,

@@ -147,6 +147,69 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t ro
   }
 }
 
+// AR_INIT_MSE: one warp per group, one lane per grid ratio (two rounds for the 51
+// ratios).  Each lane walks the group's columns in order and sums the squared
+// round-to-nearest error in fp64 (fma(d, d, acc) rounds once, and d*d is exact
+// in fp64, so this is the plain ordered sum of exact squares); the warp then takes
+// the smallest (error, grid index) pair, i.e. the first minimum along the grid.
+constexpr int kMseGrid = 51;
+
+__global__ void mse_init_kernel(const void* __restrict__ W, int w_bf16, int64_t out, int64_t in, int g, int bits,
+                                int sym, float* __restrict__ alpha, float* __restrict__ beta) {
+  const int lane = threadIdx.x & 31;
+  const int64_t G = in / g;
+  const int64_t grp = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (grp >= out * G) return;  // warp-uniform
+  const int64_t e0 = (grp / G) * in + (grp % G) * g;
+  const uint16_t* wb = static_cast<const uint16_t*>(W) + e0;
+  const float* wf = static_cast<const float*>(W) + e0;
+  auto wat = [&](int k) { return w_bf16 ? bf16_bits_to_f32(wb[k]) : wf[k]; };
+
+  float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W) of the group
+  for (int k = lane; k < g; k += 32) {
+    const float w = wat(k);
+    mn = fminf(mn, w);
+    mx = fmaxf(mx, w);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float Q = qmaxf(bits);
+  double best_e = INFINITY;
+  int best_i = kMseGrid;
+  for (int i = lane; i < kMseGrid + 31; i += 32) {  // both rounds run all 32 lanes
+    const bool live = i < kMseGrid;
+    const float p = __fdiv_rn(static_cast<float>(100 - (live ? i : 0)), 100.0f);
+    const GroupScale gs = group_scale(mn, mx, p, p, bits, sym != 0);
+    double acc = 0.0;
+    for (int k = 0; k < g; ++k) {
+      const float w = wat(k);
+      const double d = static_cast<double>(__fsub_rn(quant_elem(w, 0.0f, gs, Q).wq, w));
+      acc = fma(d, d, acc);
+    }
+    if (live && (acc < best_e || (acc == best_e && i < best_i))) {
+      best_e = acc;
+      best_i = i;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double oe = __shfl_xor_sync(0xffffffffu, best_e, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+    if (oe < best_e || (oe == best_e && oi < best_i)) {
+      best_e = oe;
+      best_i = oi;
+    }
+  }
+  if (lane == 0) {
+    const float p = __fdiv_rn(static_cast<float>(100 - best_i), 100.0f);
+    alpha[grp] = p;
+    beta[grp] = p;
+  }
+}
+
 // One block per step; fixed-order fp64 sums.
 __global__ void loss_trace_kernel(const float* __restrict__ rowloss, int64_t out, int64_t batch_rows,
                                   float* __restrict__ loss_trace) {
@@ -349,6 +412,16 @@ cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols,
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>((cols + 63) / 64), static_cast<unsigned>((rows + 63) / 64));
   transpose_bf16_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, Xt, ld_t);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mse_init(const void* W, int w_bf16, int64_t out, int64_t in, int g, int bits, bool sym,
+                            float* alpha, float* beta, cudaStream_t stream) {
+  const int64_t groups = out * (in / g);
+  if (groups <= 0) return cudaSuccess;
+  const int64_t blocks = (groups + 7) / 8;  // 8 warps, one group each
+  mse_init_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(W, w_bf16, out, in, g, bits, sym ? 1 : 0,
+                                                                    alpha, beta);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,7 @@ def test_tune_validation(ar):
     assert call(64, 1024, 1024, batch_rows=512, group_size=512) == ar.AR_EUNSUPPORTED  # g straddles tiles
     assert call(64, 250, 1024, batch_rows=512, group_size=-1) == ar.AR_EUNSUPPORTED   # in % 32
     assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK              # empty layer
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, init=2) == ar.AR_EINVAL  # unknown init
     # too small a workspace
     p = ar.make_params(batch_rows=512, group_size=64)
     assert lib.ar_tune_layer(dummy, 1, 64, 256, dummy, 1024, ctypes.byref(p), None, dummy, 1024,

@@ -1,0 +1,98 @@
+"""GPU parity of the options beyond the base loop: the MSE grid-search start of
+the clip factors (ar_init AR_INIT_MSE) and the full batch per step
+(batch_rows = n_rows, every calibration row in every step, as the page's loop
+over all batches does).
+
+The MSE start is a deterministic integer decision per group made in the same
+fp32/fp64 arithmetic on both sides, so with iters = 0 the codes, scales and
+zero-points must equal the oracle's bit for bit.  Tuned results follow the bars
+of test_gpu_parity.py: at most 0.5% of the codes differ and the final MSE agrees
+within 2% relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import TINY, make_activations, make_weight
+
+pytestmark = pytest.mark.gpu
+
+CODE_TOL = 0.005
+MSE_RTOL = 0.02
+ALGOS = ("direct", "gram")
+
+
+@pytest.fixture(scope="module")
+def ar():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import signed_gradient_rounding_b200 as ar
+    return ar
+
+
+def _w_dev(W, dtype):
+    t = torch.from_numpy(W)
+    return (t.to(torch.bfloat16) if dtype == "bf16" else t).cuda()
+
+
+def _x_dev(X):
+    return torch.from_numpy(X).to(torch.bfloat16).cuda()
+
+
+def _np(t):
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("out,inn,g,bits,sym,wdt", [
+    (512, 1024, 128, 4, False, "bf16"), (300, 256, 64, 2, False, "f32"), (130, 384, 32, 3, True, "bf16"),
+    (64, 256, -1, 8, False, "bf16"), (96, 192, 64, 4, True, "f32")])
+def test_mse_init_bit_exact(ar, out, inn, g, bits, sym, wdt):
+    """iters = 0 applies the initial state: every group's chosen ratio shows in its scale."""
+    W = make_weight(out, inn, 0.02, wdt, seed=11)
+    W[::5, 3] *= 8                                     # outliers: clipping pays off in some groups
+    X = make_activations(512, inn, "llm", seed=11)
+    p = ar.make_params(bits=bits, group_size=g, sym=sym, iters=0, batch_rows=512, init="mse")
+    res = ar.tune_layer(_w_dev(W, wdt), _x_dev(X), p, want_final_mse=False)
+    torch.cuda.synchronize()
+    ref = oracle.tune_layer(W, X, bits, g, sym, 0, 0.005, -1.0, 512, 0, init="mse", want_final_mse=False)
+    assert np.array_equal(_np(res.scale), ref.scale)
+    assert np.array_equal(_np(res.zero_point), ref.zero_point)
+    assert np.array_equal(_np(res.codes), ref.codes)
+    assert np.any(ref.alpha < 1.0)                      # the search did move some groups
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_mse_init_tiny_tuning(ar, algo):
+    c = TINY
+    W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
+    X = make_activations(c.n_rows, c.inn, c.x_kind, seed=0)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, algo=algo, init="mse")
+    res = ar.tune_layer(_w_dev(W, c.w_dtype), _x_dev(X), p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, X, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr, c.batch_rows, 0,
+                            init="mse")
+    frac = float(np.mean(_np(res.codes) != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
+    rtn = oracle.tune_layer(W, X, c.bits, c.group_size, c.sym, 0, c.lr, c.minmax_lr, c.batch_rows, 0)
+    assert ref.final_mse < rtn.final_mse
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_full_batch_per_step(ar, algo):
+    """batch_rows = n_rows: each step's gradient covers every calibration row."""
+    out, inn, n, bits, g = 192, 1024, 8192, 3, 128
+    W = make_weight(out, inn, 0.02, "bf16", seed=12)
+    X = make_activations(n, inn, "llm", seed=12)
+    p = ar.make_params(bits=bits, group_size=g, iters=30, batch_rows=n, algo=algo)
+    res = ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, X, bits, g, False, 30, 0.005, -1.0, n, 0)
+    frac = float(np.mean(_np(res.codes) != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
+    # with one full batch every step's loss is the layer MSE, and keep-best never ends above step 0
+    trace = _np(res.loss_trace).astype(np.float64)
+    np.testing.assert_allclose(trace, ref.loss_trace, rtol=0.05)
+    assert float(res.final_mse.item()) <= trace[0] * (1 + 1e-3)
