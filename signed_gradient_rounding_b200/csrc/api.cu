@@ -160,6 +160,10 @@ struct Plan {
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
+  // Direct-form residual and update GEMMs on pair tiles: measured 3% faster on the
+  // 4096-wide layer, 3-10% slower (more energy per step at the power cap) on the
+  // 29568-wide one, which is where the automatic choice picks the direct form.
+  bool pair_direct = false;
 };
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
@@ -565,17 +569,21 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     __nv_bfloat16* Rh = H(L.Rt_hi);
     __nv_bfloat16* Rl = H(L.Rt_lo);
     GemmMaps mr{}, mu{};
+    // Pair tiles (as for the Gram step): each CTA stages half of a tile's B rows.
+    const uint32_t res_box = P.pair_direct ? P.bn_res / 2 : P.bn_res;
+    const uint32_t upd_box = P.pair_direct ? P.bn_upd / 2 : P.bn_upd;
     AR_CUDA_TRY(make_tmap_bf16(&mr.a0, D_hi, out, in, kBM));
     AR_CUDA_TRY(make_tmap_bf16(&mr.a1, D_lo, out, in, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&mr.b0, X, n_rows, in, P.bn_res));
+    AR_CUDA_TRY(make_tmap_bf16(&mr.b0, X, n_rows, in, res_box));
     mr.b1 = mr.b0;
     AR_CUDA_TRY(make_tmap_bf16(&mu.a0, Rh, out, B, kBM));
     AR_CUDA_TRY(make_tmap_bf16(&mu.a1, Rl, out, B, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&mu.b0, Xt, in, n_rows, P.bn_upd));
+    AR_CUDA_TRY(make_tmap_bf16(&mu.b0, Xt, in, n_rows, upd_box));
     mu.b1 = mu.b0;
 
     GemmArgs r;  // residual: R^T = D X_b^T, (D_hi + D_lo) X_b^T
-    fill_grid(r, out, B, in, P.bn_res, nseg_d);
+    fill_grid(r, out, B, in, P.bn_res, nseg_d, P.pair_direct);
+    r.raster_m = P.raster_upd;
     r.seg_a[1] = 1;
     r.timeout_ns = timeout_ns;
     r.status = status;
@@ -585,7 +593,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     r.part = part[0];
     r.part_ld = static_cast<int>(P.nparts_res);
 
-    fill_grid(u, out, in, B, P.bn_upd, nseg_d);  // update: G = (R_hi + R_lo)^T X_b
+    fill_grid(u, out, in, B, P.bn_upd, nseg_d, P.pair_direct);  // update: G = (R_hi + R_lo)^T X_b
+    u.raster_m = P.raster_upd;
     u.seg_a[1] = 1;
     u.V_in = Vb[0];
     u.V_out = Vb[0];
