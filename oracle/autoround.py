@@ -274,7 +274,7 @@ class TuneResult:
 def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
                minmax_lr: float, batch_rows: int, seed: int, minmax_shrink: float = 1.0,
                keep_best: bool = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
-               best0=None, want_final_mse: bool = True, init: str = "minmax") -> TuneResult:
+               best0=None, want_final_mse: bool = True, init: str = "minmax", X_target=None) -> TuneResult:
     """SignSGD tuning of one linear layer.
 
     "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END": per step,
@@ -307,6 +307,13 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     ``init``: "minmax" starts the clip factors at ``minmax_shrink`` (the page's
     ``minmax_shrink`` parameter); "mse" starts each group at its ``mse_init``
     ratio (minmax_shrink is then unused).
+
+    ``X_target`` ([n, in], bf16-exact, optional): the inputs of the target output.
+    The page's quant-aware mode (``enable_quanted_input``) feeds the layer the
+    output of the already-quantised layers before it, while the target stays the
+    captured full-precision output ``y_true``.  With X_target the batch residual
+    is Y' - Y = X_b W'^T - X_target,b W^T, written out as those two products;
+    without it Y = X_b W^T (the layer's own input on both sides).
     """
     W = _to_f32(W)
     out, inn = W.shape
@@ -346,7 +353,11 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
         Xb = cache[blk]
         s, zp = scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
         Wq = fake_quant(W, V, s, zp, g, bits).Wq
-        R = Xb @ (Wq.astype(F64) - W64).T          # Y' - Y  [B, out]
+        if X_target is None:
+            R = Xb @ (Wq.astype(F64) - W64).T      # Y' - Y  [B, out]
+        else:
+            Xt_b = _rows_f64(X_target, blk * batch_rows, (blk + 1) * batch_rows)
+            R = Xb @ Wq.astype(F64).T - Xt_b @ W64.T
         row_loss = np.sum(R * R, axis=0) / batch_rows
         trace[t] = float(np.sum(row_loss)) / out
         better = row_loss < best_loss
@@ -372,7 +383,10 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
             Xb = cache.get(r0 // batch_rows)
             if Xb is None:
                 Xb = _rows_f64(X, r0, r0 + batch_rows)
-            R = Xb @ D.T
+            if X_target is None:
+                R = Xb @ D.T
+            else:
+                R = Xb @ fq.Wq.astype(F64).T - _rows_f64(X_target, r0, r0 + batch_rows) @ W64.T
             acc += float(np.sum(R * R))
         mse = acc / (n * out)
     return TuneResult(fq.q.astype(np.uint8), s, zp.astype(np.int32), fq.Wq, V, alpha, beta,

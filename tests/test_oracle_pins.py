@@ -151,8 +151,9 @@ def _ste(x):
     return x + (torch.round(x) - x).detach()
 
 
-def _autograd_grads(W, V, alpha, beta, wmin, wmax, X, g, bits, sym):
-    """dL/dV, dL/dalpha, dL/dbeta by torch autograd in fp64, rounding made straight-through."""
+def _autograd_grads(W, V, alpha, beta, wmin, wmax, X, g, bits, sym, X_target=None):
+    """dL/dV, dL/dalpha, dL/dbeta by torch autograd in fp64, rounding made straight-through.
+    With X_target the target output is X_target W^T instead of X W^T."""
     Q = float(2 ** bits - 1)
     Wt = torch.from_numpy(W.astype(np.float64))
     Vt = torch.from_numpy(V.astype(np.float64)).requires_grad_()
@@ -177,7 +178,10 @@ def _autograd_grads(W, V, alpha, beta, wmin, wmax, X, g, bits, sym):
     q = torch.clamp(_ste(Wt / se + Vt) + ze, 0, Q)
     Wq = se * (q - ze)
     Xt = torch.from_numpy(X.astype(np.float64))
-    R = Xt @ (Wq - Wt).T
+    if X_target is None:
+        R = Xt @ (Wq - Wt).T
+    else:
+        R = Xt @ Wq.T - torch.from_numpy(X_target.astype(np.float64)) @ Wt.T
     loss = (R ** 2).sum() / R.numel()
     loss.backward()
     db = np.zeros_like(beta, dtype=np.float64) if bt.grad is None else bt.grad.numpy()
@@ -222,6 +226,58 @@ def test_one_step_from_zero():
     expect = (-F32(lr) * np.sign(dV)).astype(np.float32)
     assert np.array_equal(res.V, expect)
     assert set(np.unique(res.V).tolist()) <= {-F32(lr), 0.0, F32(lr)}
+
+
+def _quant_input(X, seed):
+    """Stand-in for the output of already-quantised layers: X plus small noise, in bf16."""
+    rng = np.random.default_rng(seed)
+    return bf16_round(X + F32(0.05) * rng.standard_normal(X.shape).astype(np.float32) * np.abs(X).mean())
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_fp_target_gradients_match_autograd(sym):
+    """quant-aware input with a full-precision target: one step's moves of V, alpha
+    and beta against autograd of mean((X W'^T - X_fp W^T)^2), from a random state
+    (an exact-tie-free start: V = 0 puts the symmetric group maximum on W/s = 3.5
+    exactly in fp32, which fp64 autograd rounds from the other side)."""
+    out, inn, g, n = 8, 64, 16, 48
+    W = make_weight(out, inn, 0.02, "f32", seed=41)
+    Xf = _tiny_x(n, inn, seed=42)
+    Xq = _quant_input(Xf, 43)
+    lr = 0.005
+    rng = np.random.default_rng(47)
+    V0 = rng.uniform(-0.5, 0.5, W.shape).astype(np.float32)
+    wmin, wmax = oracle.group_minmax(W, g)
+    a0 = rng.uniform(0.6, 0.9, wmin.shape).astype(np.float32)
+    b0 = rng.uniform(0.6, 0.9, wmin.shape).astype(np.float32)
+    res = oracle.tune_layer(W, Xq, 3, g, sym, 1, lr, lr, n, 0, keep_best=False, want_final_mse=False,
+                            V0=V0, alpha0=a0, beta0=b0, X_target=Xf)
+    dV, da, db, R = _autograd_grads(W, V0, a0, b0, wmin, wmax, Xq, g, 3, sym, X_target=Xf)
+    moved = np.abs(dV) > 1e-12
+    expect_V = np.clip(V0 - F32(lr) * np.sign(dV).astype(np.float32), F32(-0.5), F32(0.5))
+    assert np.array_equal(res.V[moved], expect_V[moved])
+    assert np.array_equal(res.V[dV == 0], V0[dV == 0])
+    assert np.array_equal(res.alpha, np.clip(a0 - F32(lr) * np.sign(da).astype(np.float32), F32(0.5), F32(1)))
+    if not sym:
+        assert np.array_equal(res.beta, np.clip(b0 - F32(lr) * np.sign(db).astype(np.float32), F32(0.5), F32(1)))
+    # the step's loss is the batch MSE against the full-precision target (the oracle's W'
+    # is the fp32 one, autograd's the fp64 product of the same factors)
+    assert res.loss_trace[0] == pytest.approx(float(np.mean(R ** 2)), rel=1e-6)
+
+
+def test_fp_target_final_mse_and_same_input():
+    W = make_weight(16, 64, 0.02, "f32", seed=44)
+    Xf = _tiny_x(128, 64, seed=45)
+    Xq = _quant_input(Xf, 46)
+    res = oracle.tune_layer(W, Xq, 4, 32, False, 6, 0.005, 0.005, 64, 0, X_target=Xf)
+    Y = torch.from_numpy(Xf.astype(np.float64)) @ torch.from_numpy(W.astype(np.float64)).T
+    Yq = torch.from_numpy(Xq.astype(np.float64)) @ torch.from_numpy(res.Wq.astype(np.float64)).T
+    assert res.final_mse == pytest.approx(float(((Yq - Y) ** 2).mean()), rel=1e-10)
+    # the target's own input gives the layer's usual loop
+    a = oracle.tune_layer(W, Xf, 4, 32, False, 6, 0.005, 0.005, 64, 0, X_target=Xf)
+    b = oracle.tune_layer(W, Xf, 4, 32, False, 6, 0.005, 0.005, 64, 0)
+    assert np.array_equal(a.codes, b.codes)
+    np.testing.assert_allclose(a.loss_trace, b.loss_trace, rtol=1e-9)
 
 
 # ---------------------------------------------------------------- loop
