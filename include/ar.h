@@ -224,6 +224,39 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
                               uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
                               double* final_mse, void* stream, ar_tune_timing* timing);
 
+/* Workspace of ar_tune_layer_fp_target, in bytes (0 if the arguments are invalid or
+ * ask for the direct form).  On top of ar_tune_workspace_bytes' Gram-form layout:
+ * two copies of one calibration block as a bf16 pair (4 * batch_rows * in * 2
+ * bytes), the in x in pair M_b^T, every block's out x in pair C_b
+ * (n_rows/batch_rows * out * in * 4 bytes), their fp32 sum, and W as a pair when it
+ * is fp32. */
+size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,
+                                         const ar_tune_params* params);
+
+/* ar_tune_layer in the quant-aware mode with a full-precision target
+ * ("[llm-compressor] AutoRound ...", "enable_quanted_input 모드" and the
+ * "AutoRoundModifier" field enable_quanted_input: each layer is fed the output of
+ * the already-quantised layers before it, while the loss compares against the
+ * captured full-precision output).
+ *   X          [n_rows, in] bf16: the layer's input on the quantised path.
+ *   X_target   [n_rows, in] bf16: the input of the full-precision target, Y = X_target W^T.
+ * The batch residual is R = X_b W'^T - X_target,b W^T = X_b D^T + dX_b W^T with
+ * D = W' - W and dX = X - X_target, so with H_b = X_b^T X_b:
+ *   gradient  G = D H_b + W M_b,   M_b = dX_b^T X_b            (in x in)
+ *   row loss  L_j = d_j H_b d_j^T + 2 d_j (W M_b)_j^T + |dX_b w_j^T|^2.
+ * Per calibration block (before its first step) the library forms dX_b as a bf16
+ * pair and computes M_b, C_b = W M_b and e_b = |dX_b w_j^T|^2 on the tensor cores;
+ * the step kernel adds C_b to G and the two loss terms to the row loss.
+ * final_mse = mean((X W'^T - X_target W^T)^2) over all rows.  Gram form only
+ * (params->algo AR_ALGO_AUTO or AR_ALGO_GRAM; AR_ALGO_DIRECT gives
+ * AR_EUNSUPPORTED).  X_target NULL: AR_EINVAL.  Otherwise arguments, results and
+ * errors as ar_tune_layer, with workspace of ar_tune_fp_target_workspace_bytes(). */
+ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
+                                  const uint16_t* X, const uint16_t* X_target, int64_t n_rows,
+                                  const ar_tune_params* params, ar_tune_state* state, void* workspace,
+                                  size_t ws_bytes, uint8_t* codes, float* scale, int32_t* zp,
+                                  float* loss_trace, double* final_mse, void* stream);
+
 /* Device workspace of ar_tune_layer_host, in bytes (0 if the arguments are invalid):
  * ar_tune_workspace_bytes() plus device copies of W, X and the outputs. */
 size_t ar_tune_host_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,

@@ -30,7 +30,8 @@ INITS = {"minmax": AR_INIT_MINMAX, "mse": AR_INIT_MSE}
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
-           "ar_tune_host_workspace_bytes", "ar_tune_layer_host",
+           "ar_tune_host_workspace_bytes", "ar_tune_layer_host", "ar_tune_fp_target_workspace_bytes",
+           "ar_tune_layer_fp_target",
            "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static", "ar_dequant", "ar_linear",
            "ar_silu_mul")
 
@@ -85,6 +86,11 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(_TuneStateC), P, SZ, P, P, P, P, P, P]
     lib.ar_tune_layer_timed.restype = ctypes.c_int
     lib.ar_tune_layer_timed.argtypes = lib.ar_tune_layer.argtypes + [ctypes.POINTER(TuneTiming)]
+    lib.ar_tune_fp_target_workspace_bytes.restype = SZ
+    lib.ar_tune_fp_target_workspace_bytes.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.POINTER(TuneParams)]
+    lib.ar_tune_layer_fp_target.restype = ctypes.c_int
+    lib.ar_tune_layer_fp_target.argtypes = [P, ctypes.c_int, I64, I64, P, P, I64, ctypes.POINTER(TuneParams),
+                                            ctypes.POINTER(_TuneStateC), P, SZ, P, P, P, P, P, P]
     lib.ar_tune_host_workspace_bytes.restype = SZ
     lib.ar_tune_host_workspace_bytes.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.POINTER(TuneParams)]
     lib.ar_tune_layer_host.restype = ctypes.c_int
@@ -333,6 +339,37 @@ def tune_layer(W: torch.Tensor, X: torch.Tensor, params: TuneParams, state: Tune
     if state is not None:
         state.initialized = True
     return TuneResult(codes, scale, zp, trace[:params.iters] if trace is not None else None, mse, workspace)
+
+
+def tune_layer_fp_target(W: torch.Tensor, X: torch.Tensor, X_target: torch.Tensor, params: TuneParams,
+                         workspace: torch.Tensor | None = None, want_final_mse: bool = True,
+                         stream=None) -> TuneResult:
+    """ar_tune_layer_fp_target on device tensors: the layer sees X (its input on the
+    quantised path) and is tuned against the full-precision output X_target W^T."""
+    _dev(W, "W")
+    _dev(X, "X", torch.bfloat16)
+    _dev(X_target, "X_target", torch.bfloat16)
+    out, inn = W.shape
+    n_rows = X.shape[0]
+    if X.shape != (n_rows, inn) or X_target.shape != X.shape:
+        raise ValueError("X and X_target must be [n_rows, in]")
+    wdt = _wdtype(W)
+    need = int(_lib.ar_tune_fp_target_workspace_bytes(out, inn, n_rows, wdt, ctypes.byref(params)))
+    if need == 0:
+        raise ArError(AR_EUNSUPPORTED, "ar_tune_fp_target_workspace_bytes")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    G = max(_groups(inn, params.group_size), 1)
+    codes = torch.empty((out, inn), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((out, G), dtype=torch.float32, device=W.device)
+    zp = torch.empty((out, G), dtype=torch.int32, device=W.device)
+    trace = torch.empty((max(params.iters, 1),), dtype=torch.float32, device=W.device)
+    mse = torch.empty((1,), dtype=torch.float64, device=W.device) if want_final_mse else None
+    _check(_lib.ar_tune_layer_fp_target(_ptr(W), wdt, out, inn, _ptr(X), _ptr(X_target), n_rows,
+                                        ctypes.byref(params), None, _ptr(workspace), workspace.numel(),
+                                        _ptr(codes), _ptr(scale), _ptr(zp), _ptr(trace), _ptr(mse),
+                                        _stream(stream)), "ar_tune_layer_fp_target")
+    return TuneResult(codes, scale, zp, trace[:params.iters], mse, workspace)
 
 
 def tune_status(workspace: torch.Tensor, stream=None) -> int:

@@ -160,6 +160,10 @@ struct Plan {
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
+  // Full-precision-target mode (ar_tune_layer_fp_target; Gram form only), and
+  // whether W is fp32 (then held as a bf16 pair for its contractions).
+  bool fp_target = false;
+  bool w_f32 = false;
   // Direct-form residual and update GEMMs on pair tiles: measured 3% faster on the
   // 4096-wide layer, 3-10% slower (more energy per step at the power cap) on the
   // 29568-wide one, which is where the automatic choice picks the direct form.
@@ -168,8 +172,11 @@ struct Plan {
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
 
-Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p) {
+Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool fp_target = false,
+               bool w_f32 = false) {
   Plan P;
+  P.fp_target = fp_target;
+  P.w_f32 = w_f32;
   P.split = p->split != 0;
   P.out = out;
   P.in = in;
@@ -184,7 +191,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p) {
   const double direct = P.iters * pieces_direct * 4.0 * P.B * out * in + pieces_direct * 2.0 * n * out * in;
   const double gram = P.iters * pieces_gram * 2.0 * out * in * in + 2.0 * n * in * in + pieces_gram * 2.0 * out * in * in;
   const double gram_bytes = (P.nb + 1.0) * in * in * 2.0 * (P.split ? 2.0 : 1.0);
-  if (p->algo == AR_ALGO_GRAM)
+  if (p->algo == AR_ALGO_GRAM || (fp_target && p->algo == AR_ALGO_AUTO))
     P.algo = AR_ALGO_GRAM;
   else if (p->algo == AR_ALGO_DIRECT)
     P.algo = AR_ALGO_DIRECT;
@@ -205,7 +212,12 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p) {
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
   size_t status, Xt, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
-      part0, part1, rowloss, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum, total;
+      part0, part1, rowloss, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
+      // full-precision-target mode: this block's dX = X - X_target (pair, row-major
+      // and transposed), M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b
+      // (pair), their sum Cs (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the
+      // partials of e_b, and W as a pair when it is fp32
+      dX_hi, dX_lo, dXt_hi, dXt_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo, total;
 };
 
 Layout make_layout(const Plan& P) {
@@ -251,6 +263,25 @@ Layout make_layout(const Plan& P) {
     L.Hs_lo = P.split ? take(h) : L.Hs_hi;
     L.Hdiag = take(static_cast<size_t>(P.nb) * P.in * 4);
     L.Hdsum = take(static_cast<size_t>(P.in) * 4);
+    if (P.fp_target) {
+      const size_t blk = static_cast<size_t>(P.B) * P.in * 2;
+      L.dX_hi = take(blk);
+      L.dX_lo = take(blk);
+      L.dXt_hi = take(blk);
+      L.dXt_lo = take(blk);
+      L.Mt_hi = take(h);
+      L.Mt_lo = take(h);
+      L.Cc_hi = take(elems * 2 * P.nb);
+      L.Cc_lo = take(elems * 2 * P.nb);
+      L.Cs = take(elems * 4);
+      L.e = take(static_cast<size_t>(P.nb) * P.out * 4);
+      L.es = take(static_cast<size_t>(P.out) * 4);
+      L.epart = take(static_cast<size_t>(P.out) * cdiv(P.B, 256) * kEpiHalves * 4);
+      if (P.w_f32) {
+        L.Wp_hi = take(elems * 2);
+        L.Wp_lo = take(elems * 2);
+      }
+    }
   } else {
     L.Rt_hi = take(static_cast<size_t>(P.out) * P.B * 2);
     L.Rt_lo = P.split ? take(static_cast<size_t>(P.out) * P.B * 2) : L.Rt_hi;
@@ -297,7 +328,8 @@ struct EventTimer {
 ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X, int64_t n_rows,
                     const ar_tune_params* p, ar_tune_state* state, void* workspace, size_t ws_bytes,
                     uint8_t* codes, float* scale, int32_t* zp, float* loss_trace, double* final_mse,
-                    void* stream, EventTimer* timer, const cudaEvent_t* block_ready = nullptr) {
+                    void* stream, EventTimer* timer, const cudaEvent_t* block_ready = nullptr,
+                    const uint16_t* X_target = nullptr) {
   const ar_status chk = check_tune_args(out, in, n_rows, p);
   if (chk != AR_OK) return chk;
   if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
@@ -311,7 +343,9 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       if (!q || !aligned(q, 16)) return AR_EINVAL;
   }
 
-  const Plan P = make_plan(out, in, n_rows, p);
+  if (X_target && !aligned(X_target, 16)) return AR_EINVAL;
+  const Plan P = make_plan(out, in, n_rows, p, X_target != nullptr, w_dtype == AR_F32);
+  if (P.fp_target && P.algo != AR_ALGO_GRAM) return AR_EUNSUPPORTED;
   const Layout L = make_layout(P);
   if (ws_bytes < L.total) return AR_ENOMEM;
   const bool gram = P.algo == AR_ALGO_GRAM;
@@ -396,6 +430,23 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     launches += 1;
   }
 
+  // Full-precision-target mode: the block sums start at zero; an fp32 W is held as
+  // a bf16 pair for its contractions.
+  const bool fpt = P.fp_target;
+  const __nv_bfloat16* Wa_hi = static_cast<const __nv_bfloat16*>(W);
+  const __nv_bfloat16* Wa_lo = nullptr;
+  if (fpt) {
+    AR_CUDA_TRY(cudaMemsetAsync(F(L.Cs), 0, elems * 4, st));
+    AR_CUDA_TRY(cudaMemsetAsync(F(L.es), 0, static_cast<size_t>(out) * 4, st));
+    if (P.w_f32) {
+      AR_CUDA_TRY(launch_split_pair(static_cast<const float*>(W), static_cast<int64_t>(elems), H(L.Wp_hi),
+                                    H(L.Wp_lo), st));
+      ++launches;
+      Wa_hi = H(L.Wp_hi);
+      Wa_lo = H(L.Wp_lo);
+    }
+  }
+
   // Group statistics of W and the first step's D = W' - W.
   GroupQuantArgs prep;
   prep.W = W;
@@ -441,6 +492,76 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     h.ldc = in;
     h.diag_out = F(L.Hdiag);
   }
+  // Full-precision-target mode, per block b (dX_b = X_b - X_target,b):
+  //   M_b^T = X_b^T dX_b          [in, in]   (pair; A = X_b^T, B = dX_b^T pair)
+  //   C_b   = W M_b               [out, in]  (pair; the step adds it to G)
+  //   e_b[j] = |dX_b w_j^T|^2     (row sums of squares of W dX_b^T)
+  //   Cs += C_b,  es += e_b       (the final MSE over all blocks)
+  GemmMaps mt_maps{}, c_maps{}, e_maps{};
+  GemmArgs mg, cg, eg;
+  if (fpt) {
+    const int nseg_w = P.w_f32 ? 3 : 2;  // W pair x operand pair, or W x operand pair
+    mt_maps.a0 = gram_maps.a0;
+    mt_maps.a1 = gram_maps.a0;
+    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b0, H(L.dXt_hi), in, B, 256));
+    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b1, H(L.dXt_lo), in, B, 256));
+    fill_grid(mg, in, in, B, 256, 2);
+    mg.seg_b[1] = 1;
+    mg.timeout_ns = timeout_ns;
+    mg.status = status;
+    mg.C_hi = H(L.Mt_hi);
+    mg.C_lo = H(L.Mt_lo);
+    mg.ldc = in;
+    for (GemmMaps* m : {&c_maps, &e_maps}) {
+      AR_CUDA_TRY(make_tmap_bf16(&m->a0, Wa_hi, out, in, kBM));
+      if (Wa_lo)
+        AR_CUDA_TRY(make_tmap_bf16(&m->a1, Wa_lo, out, in, kBM));
+      else
+        m->a1 = m->a0;
+    }
+    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b0, H(L.Mt_hi), in, in, 256));
+    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b1, H(L.Mt_lo), in, in, 256));
+    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b0, H(L.dX_hi), B, in, 256));
+    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b1, H(L.dX_lo), B, in, 256));
+    for (GemmArgs* g : {&cg, &eg}) {
+      fill_grid(*g, out, g == &cg ? in : B, in, 256, nseg_w);
+      if (P.w_f32) {  // W_hi X_hi + W_lo X_hi + W_hi X_lo
+        g->seg_a[1] = 1;
+        g->seg_b[2] = 1;
+      } else {        // W X_hi + W X_lo
+        g->seg_b[1] = 1;
+      }
+      g->timeout_ns = timeout_ns;
+      g->status = status;
+    }
+    cg.C_hi = H(L.Cc_hi);
+    cg.C_lo = H(L.Cc_lo);
+    cg.ldc = in;
+    eg.part = F(L.epart);
+    eg.part_ld = eg.num_n_blk * kEpiHalves;
+  }
+  auto fp_target_block = [&](int64_t b) -> cudaError_t {
+    const int64_t blk = B * in;
+    cudaError_t e = launch_diff_pair(X + b * blk, X_target + b * blk, blk, H(L.dX_hi), H(L.dX_lo), st);
+    if (e == cudaSuccess)
+      e = launch_transpose_bf16(reinterpret_cast<const uint16_t*>(H(L.dX_hi)), B, in,
+                                reinterpret_cast<uint16_t*>(H(L.dXt_hi)), B, st);
+    if (e == cudaSuccess)
+      e = launch_transpose_bf16(reinterpret_cast<const uint16_t*>(H(L.dX_lo)), B, in,
+                                reinterpret_cast<uint16_t*>(H(L.dXt_lo)), B, st);
+    mg.a_k_off = static_cast<int>(b * B);
+    if (e == cudaSuccess) e = launch_gemm(kEpiStore, 256, mt_maps, mg, sms, st);
+    cg.c_row_off = b * out;
+    if (e == cudaSuccess) e = launch_gemm(kEpiStore, 256, c_maps, cg, sms, st);
+    if (e == cudaSuccess)
+      e = launch_accum_pair(H(L.Cc_hi) + b * static_cast<int64_t>(elems), H(L.Cc_lo) + b * static_cast<int64_t>(elems),
+                            static_cast<int64_t>(elems), F(L.Cs), st);
+    if (e == cudaSuccess) e = launch_gemm(kEpiSumSq, 256, e_maps, eg, sms, st);
+    if (e == cudaSuccess) e = launch_row_sum(F(L.epart), eg.part_ld, out, F(L.e) + b * out, F(L.es), st);
+    launches += 8;
+    return e;
+  };
+
   // Each calibration block is transposed into its columns of Xt (and, in the Gram
   // form, its Gram matrix is made) just before the first step that uses it.  With
   // block_ready events, the block's copy to the device is awaited first.
@@ -462,7 +583,9 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     h.b_k_off = static_cast<int>(b * B);
     h.c_row_off = b * in;
     ++launches;
-    return launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
+    e = launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
+    if (e != cudaSuccess || !fpt) return e;
+    return fp_target_block(b);
   };
 
   // The update epilogue's common arguments.
@@ -531,8 +654,13 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       u.best_in = best_cur;
       u.best_out = best_next;
       AR_CUDA_TRY(ensure_block(sched[t]));
+      if (fpt) {
+        u.Cc_hi = H(L.Cc_hi) + sched[t] * static_cast<int64_t>(elems);
+        u.Cc_lo = H(L.Cc_lo) + sched[t] * static_cast<int64_t>(elems);
+        u.e_row = F(L.e) + sched[t] * out;
+      }
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
-      AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
+      AR_CUDA_TRY(launch_gemm(fpt ? kEpiUpdateFp : kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
       if (timer) {
         AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
         AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
@@ -684,6 +812,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       f.Dd_hi = D_hi;
       f.Dd_lo = P.split ? D_lo : nullptr;
       f.diag_in = F(L.Hdsum);
+      if (fpt) {
+        f.Cs = F(L.Cs);
+        f.e_row = F(L.es);
+      }
       f.part_ld = f.num_n_blk * kEpiHalves;
       AR_CUDA_TRY(launch_gemm(kEpiDotD, P.bn_fin, m, f, sms, st));
       launches += 2;
@@ -967,6 +1099,29 @@ ar_status ar_tune_layer_host(const void* W_host, ar_dtype w_dtype, int64_t out, 
                                 st));
   if (mse) AR_CUDA_TRY(cudaMemcpyAsync(final_mse_host, mse, 8, cudaMemcpyDeviceToHost, st));
   return ar_tune_status(ws + HL.tune, stream);
+}
+
+size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,
+                                         const ar_tune_params* p) {
+  if (check_tune_args(out, in, n_rows, p) != AR_OK) return 0;
+  if (w_dtype != AR_F32 && w_dtype != AR_BF16) return 0;
+  if (out == 0 || in == 0) return 256;
+  const Plan P = make_plan(out, in, n_rows, p, true, w_dtype == AR_F32);
+  if (P.algo != AR_ALGO_GRAM) return 0;
+  return make_layout(P).total;
+}
+
+ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
+                                  const uint16_t* X_target, int64_t n_rows, const ar_tune_params* p,
+                                  ar_tune_state* state, void* workspace, size_t ws_bytes, uint8_t* codes,
+                                  float* scale, int32_t* zp, float* loss_trace, double* final_mse, void* stream) {
+  const ar_status chk = check_tune_args(out, in, n_rows, p);
+  if (chk != AR_OK) return chk;
+  if (out == 0 || in == 0) return AR_OK;
+  if (!X_target) return AR_EINVAL;
+  if (p->algo == AR_ALGO_DIRECT) return AR_EUNSUPPORTED;
+  return tune_impl(W, w_dtype, out, in, X, n_rows, p, state, workspace, ws_bytes, codes, scale, zp, loss_trace,
+                   final_mse, stream, nullptr, nullptr, X_target);
 }
 
 ar_status ar_tune_status(const void* workspace, void* stream) {

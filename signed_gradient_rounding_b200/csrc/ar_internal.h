@@ -81,6 +81,16 @@ cudaError_t launch_dequant(const uint8_t* codes, const float* scale, const int32
                            int g, __nv_bfloat16* Wq_hi, __nv_bfloat16* Wq_lo, float* Wq, cudaStream_t stream);
 cudaError_t launch_silu_mul(const __nv_bfloat16* a, const __nv_bfloat16* b, int64_t count, __nv_bfloat16* y,
                             cudaStream_t stream);
+// Full-precision-target mode: dX = X - X_target as a bf16 pair; an fp32 array as
+// a bf16 pair; acc += hi + lo; per-row sums of partials (dst) added into total.
+cudaError_t launch_diff_pair(const uint16_t* X, const uint16_t* Xt, int64_t n, __nv_bfloat16* hi,
+                             __nv_bfloat16* lo, cudaStream_t stream);
+cudaError_t launch_split_pair(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                              cudaStream_t stream);
+cudaError_t launch_accum_pair(const __nv_bfloat16* hi, const __nv_bfloat16* lo, int64_t n, float* acc,
+                              cudaStream_t stream);
+cudaError_t launch_row_sum(const float* part, int nparts, int64_t rows, float* dst, float* total,
+                           cudaStream_t stream);
 cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
@@ -93,7 +103,8 @@ enum EpiKind : int {
   kEpiStore = 0,   // C as a bf16 (hi, lo) pair; optional per-(row, n-tile) sums of C^2
   kEpiSumSq = 1,   // per-(row, n-tile) sums of C^2
   kEpiUpdate = 2,  // C = G: the SignSGD step (sign updates, keep-best, next D, Gram-form loss)
-  kEpiDotD = 3     // per-(row, n-tile) sums of D * C
+  kEpiDotD = 3,    // per-(row, n-tile) sums of D * C
+  kEpiUpdateFp = 4 // kEpiUpdate with the full-precision-target terms (Cc_hi, e_row)
 };
 
 // Operand maps: segment s reads A from a{seg_a[s]} and B from b{seg_b[s]}.
@@ -165,6 +176,13 @@ struct GemmArgs {
   int nparts = 0;
   int snap_prev = 0;      // 0: judge this step (snapshot V_in); 1: judge the previous one (snapshot V_out)
   float* part_out = nullptr;  // [M, part_ld] this step's sum_k D G partials (Gram form), or null
+  // Full-precision-target mode (Gram form): G += C (this block's W M_b, a bf16 pair
+  // [M, N]); the row loss gains 2 sum_k D_jk C_jk, and e_row[j] once per row.
+  // kEpiDotD (final MSE): C as fp32 [M, N] (the sum over blocks) via Cs, e via e_row.
+  const __nv_bfloat16* Cc_hi = nullptr;
+  const __nv_bfloat16* Cc_lo = nullptr;
+  const float* Cs = nullptr;
+  const float* e_row = nullptr;
   float inv_batch = 1.0f;
   int g = 0, G = 0, bits = 4, sym = 0, keep_best = 1;
   float lr = 0.f, mlr = 0.f;

@@ -255,6 +255,12 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] = fmaf(dh[i], dg[i], x[i]);
       }
+      if (a.Cs) {  // full-precision target: + 2 D C^T
+        float cs[32];
+        load_f32x32(a.Cs + e, cs);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = fmaf(2.0f, cs[i], x[i]);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc = fmaf(dh[i], x[i], acc);
     }
@@ -311,6 +317,7 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
       }
     }
   }
+  if (kKind == kEpiDotD && row_ok && a.e_row && n_blk == 0 && half == 0) acc += a.e_row[j];
   if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = acc;
 }
 
@@ -341,7 +348,8 @@ __device__ __forceinline__ void load_upd_chunk(const GemmArgs& a, int64_t e0, in
   if (a.diag_in) load_f32x16(a.diag_in + col, dg);
 }
 
-template <int kBN>
+// kFp: the full-precision-target terms (GemmArgs::Cc_hi set) are compiled in.
+template <int kBN, bool kFp>
 __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
   const bool row_ok = j < a.M;
   const float Q = qmaxf(a.bits);
@@ -414,20 +422,36 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
 
     // Pass 1: sign updates of V, and the group's d alpha, d beta.
     float dal = 0.f, dbe = 0.f;
+    // The next chunk's W, V and diagonal are loaded one chunk ahead (the
+    // full-precision-target instance loads this block's C instead, which needs
+    // those registers).
     float w_nx[kUC], v_nx[kUC], dg_nx[kUC];
-    if (row_ok) load_upd_chunk(a, row_base + gcol0, gcol0, w_nx, v_nx, dg_nx);
+    if (!kFp && row_ok) load_upd_chunk(a, row_base + gcol0, gcol0, w_nx, v_nx, dg_nx);
 #pragma unroll 1
     for (int cc = 0; cc < cpg; ++cc) {
       const int col = gcol0 + cc * kUC;
       const int64_t e0 = row_base + col;
       float w[kUC], v[kUC], dg[kUC];
+      if (kFp) {
+        if (row_ok) load_upd_chunk(a, e0, col, w, v, dg);
+      } else {
 #pragma unroll
-      for (int i = 0; i < kUC; ++i) {
-        w[i] = w_nx[i];
-        v[i] = v_nx[i];
-        dg[i] = dg_nx[i];
+        for (int i = 0; i < kUC; ++i) {
+          w[i] = w_nx[i];
+          v[i] = v_nx[i];
+          dg[i] = dg_nx[i];
+        }
+        if (row_ok && cc + 1 < cpg) load_upd_chunk(a, e0 + kUC, col + kUC, w_nx, v_nx, dg_nx);
       }
-      if (row_ok && cc + 1 < cpg) load_upd_chunk(a, e0 + kUC, col + kUC, w_nx, v_nx, dg_nx);
+      // Full-precision target: this block's C = W M_b (a bf16 pair) joins G.
+      float cv[kUC];
+      if (kFp && row_ok) {
+        float clo[kUC];
+        load_w16(a.Cc_hi, 1, e0, cv);
+        load_w16(a.Cc_lo, 1, e0, clo);
+#pragma unroll
+        for (int i = 0; i < kUC; ++i) cv[i] = __fadd_rn(cv[i], clo[i]);
+      }
       uint32_t r[kUC];
       __syncwarp();
       tmem_ld_16cols(t_row + (col - n0), r);
@@ -443,8 +467,14 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       for (int i = 0; i < kUC; ++i) {
         const ElemQuant e = quant_elem(w[i], v[i], gs, Q);
         const float d = __fsub_rn(e.wq, w[i]);
-        const float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
-        loss_acc = fmaf(d, G, loss_acc);
+        float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
+        if (kFp) {
+          // row loss: d H d^T + 2 d C^T (+ e_row once per row, below); gradient D H + C
+          G = __fadd_rn(G, cv[i]);
+          loss_acc = fmaf(d, __fadd_rn(G, cv[i]), loss_acc);
+        } else {
+          loss_acc = fmaf(d, G, loss_acc);
+        }
         const float sg = e.m ? sgnf(G) : 0.0f;
         vn[i] = fminf(fmaxf(__fsub_rn(v[i], __fmul_rn(a.lr, sg)), -0.5f), 0.5f);
         float dwa, dwb;
@@ -503,6 +533,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
         store_pair8(d + q * 8, a.D_hi + e0 + q * 8, a.D_lo ? a.D_lo + e0 + q * 8 : nullptr);
     }
   }
+  if (kFp && row_ok && a.e_row && n_blk == 0 && half == 0) loss_acc += a.e_row[j];
   if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = loss_acc;
 }
 
@@ -521,6 +552,10 @@ __device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, in
   const int wsz = a.w_bf16 ? 2 : 4;
   prefetch_l2(static_cast<const uint8_t*>(a.W) + e0 * wsz, cols * wsz);
   prefetch_l2(a.V_in + e0, cols * 4);
+  if (a.Cc_hi) {
+    prefetch_l2(a.Cc_hi + e0, cols * 2);
+    prefetch_l2(a.Cc_lo + e0, cols * 2);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -714,14 +749,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_pos<kBN>(args, tile, m_blk, n_blk);
       const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
-      if (kKind == kEpiUpdate) epi_update_prefetch<kBN>(args, j, n0, half);
+      if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN>(args, j, n0, half);
       // No early exit on another role's abort: every epilogue warp of the CTA takes
       // the same decision here (the phase completes for all of them, or for none).
       if (!mbar_wait<kPair>(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns, false)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       if (kKind == kEpiUpdate)
-        epi_update<kBN>(args, t_row, j, n0, n_blk, half);
+        epi_update<kBN, false>(args, t_row, j, n0, n_blk, half);
+      else if (kKind == kEpiUpdateFp)
+        epi_update<kBN, true>(args, t_row, j, n0, n_blk, half);
       else
         epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk, half);
       tc_fence_before();
@@ -806,6 +843,8 @@ cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int
       return launch_kind<kEpiUpdate, kBN, kPair>(m, args, num_sms, stream);
     case kEpiDotD:
       return launch_kind<kEpiDotD, kBN, kPair>(m, args, num_sms, stream);
+    case kEpiUpdateFp:
+      return launch_kind<kEpiUpdateFp, kBN, kPair>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

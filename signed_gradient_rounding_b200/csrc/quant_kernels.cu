@@ -210,6 +210,52 @@ __global__ void mse_init_kernel(const void* __restrict__ W, int w_bf16, int64_t 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Helpers of the full-precision-target mode (ar_tune_layer_fp_target).
+// ---------------------------------------------------------------------------
+
+// x = hi + lo as an exact bf16 pair: hi = bf16(x), lo = bf16(x - hi) (x - hi is exact).
+__device__ __forceinline__ void split_pair(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+}
+
+// dX = X - X_target (bf16 inputs; the fp32 difference) as a bf16 pair.
+__global__ void diff_pair_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ Xt, int64_t n,
+                                 __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float d = __fsub_rn(bf16_bits_to_f32(X[i]), bf16_bits_to_f32(Xt[i]));
+    split_pair(d, hi[i], lo[i]);
+  }
+}
+
+__global__ void split_pair_kernel(const float* __restrict__ x, int64_t n, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    split_pair(x[i], hi[i], lo[i]);
+}
+
+// acc += hi + lo (fp32).
+__global__ void accum_pair_kernel(const __nv_bfloat16* __restrict__ hi, const __nv_bfloat16* __restrict__ lo,
+                                  int64_t n, float* __restrict__ acc) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    acc[i] = __fadd_rn(acc[i], __fadd_rn(__bfloat162float(hi[i]), __bfloat162float(lo[i])));
+}
+
+// dst[j] = sum of part[j, 0 .. nparts) in order; total[j] += dst[j].
+__global__ void row_sum_kernel(const float* __restrict__ part, int nparts, int64_t rows, float* __restrict__ dst,
+                               float* __restrict__ total) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= rows) return;
+  float L = 0.0f;
+  for (int q = 0; q < nparts; ++q) L += part[j * nparts + q];
+  dst[j] = L;
+  total[j] = __fadd_rn(total[j], L);
+}
+
 // One block per step; fixed-order fp64 sums.
 __global__ void loss_trace_kernel(const float* __restrict__ rowloss, int64_t out, int64_t batch_rows,
                                   float* __restrict__ loss_trace) {
@@ -422,6 +468,40 @@ cudaError_t launch_mse_init(const void* W, int w_bf16, int64_t out, int64_t in, 
   const int64_t blocks = (groups + 7) / 8;  // 8 warps, one group each
   mse_init_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(W, w_bf16, out, in, g, bits, sym ? 1 : 0,
                                                                     alpha, beta);
+  return cudaGetLastError();
+}
+
+static unsigned grid_for(int64_t n) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  return static_cast<unsigned>(blocks < 1 ? 1 : blocks);
+}
+
+cudaError_t launch_diff_pair(const uint16_t* X, const uint16_t* Xt, int64_t n, __nv_bfloat16* hi,
+                             __nv_bfloat16* lo, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  diff_pair_kernel<<<grid_for(n), 256, 0, stream>>>(X, Xt, n, hi, lo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_pair(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                              cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  split_pair_kernel<<<grid_for(n), 256, 0, stream>>>(x, n, hi, lo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accum_pair(const __nv_bfloat16* hi, const __nv_bfloat16* lo, int64_t n, float* acc,
+                              cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  accum_pair_kernel<<<grid_for(n), 256, 0, stream>>>(hi, lo, n, acc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_sum(const float* part, int nparts, int64_t rows, float* dst, float* total,
+                           cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  row_sum_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(part, nparts, rows, dst, total);
   return cudaGetLastError();
 }
 

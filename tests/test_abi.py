@@ -123,3 +123,21 @@ def test_host_entry_validation(ar):
     assert call(64, 256, 1024, batch_rows=512, group_size=16) == ar.AR_EUNSUPPORTED
     assert call(64, 256, 1024, ws_bytes=need - 1, batch_rows=512, group_size=64) == ar.AR_ENOMEM
     assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK
+
+
+def test_fp_target_validation(ar):
+    lib = ar.lib
+    dummy = ctypes.c_void_p(4096)
+    p = ar.make_params(batch_rows=512, group_size=64)
+    need = lib.ar_tune_fp_target_workspace_bytes(64, 256, 1024, 1, ctypes.byref(p))
+    assert need > lib.ar_tune_workspace_bytes(64, 256, 1024, ctypes.byref(p))
+    q = ar.make_params(batch_rows=512, group_size=64, algo="direct")
+    assert lib.ar_tune_fp_target_workspace_bytes(64, 256, 1024, 1, ctypes.byref(q)) == 0   # Gram form only
+
+    def call(Xt=dummy, params=p):
+        return lib.ar_tune_layer_fp_target(dummy, 1, 64, 256, dummy, Xt, 1024, ctypes.byref(params), None, dummy,
+                                           1 << 40, dummy, dummy, dummy, None, None, None)
+
+    assert call(Xt=None) == ar.AR_EINVAL
+    assert call(params=q) == ar.AR_EUNSUPPORTED
+    assert call(params=ar.make_params(batch_rows=512, group_size=64, bits=5)) == ar.AR_EINVAL

@@ -1,7 +1,9 @@
 """GPU parity of the options beyond the base loop: the MSE grid-search start of
-the clip factors (ar_init AR_INIT_MSE) and the full batch per step
-(batch_rows = n_rows, every calibration row in every step, as the page's loop
-over all batches does).
+the clip factors (ar_init AR_INIT_MSE), the full batch per step (batch_rows =
+n_rows, every calibration row in every step, as the page's loop over all
+batches does), and the quant-aware input with a full-precision target
+(ar_tune_layer_fp_target: the layer sees its input on the quantised path and is
+tuned against the full-precision output).
 
 The MSE start is a deterministic integer decision per group made in the same
 fp32/fp64 arithmetic on both sides, so with iters = 0 the codes, scales and
@@ -96,3 +98,46 @@ def test_full_batch_per_step(ar, algo):
     trace = _np(res.loss_trace).astype(np.float64)
     np.testing.assert_allclose(trace, ref.loss_trace, rtol=0.05)
     assert float(res.final_mse.item()) <= trace[0] * (1 + 1e-3)
+
+
+# ------------------------------------------------ quant-aware input, full-precision target
+
+def _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed):
+    from workloads import make_quantised_path_input
+    W = make_weight(out, inn, 0.02, wdt, seed=seed)
+    Xf = make_activations(n, inn, "llm", seed=seed)
+    Xq = make_quantised_path_input(Xf, 0.05, seed=seed)
+    p = ar.make_params(bits=bits, group_size=g, iters=iters, batch_rows=B, algo="gram")
+    res = ar.tune_layer_fp_target(_w_dev(W, wdt), _x_dev(Xq), _x_dev(Xf), p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, Xq, bits, g, False, iters, 0.005, -1.0, B, 0, X_target=Xf)
+    return res, ref, W, Xq, Xf
+
+
+@pytest.mark.parametrize("case", [(256, 256, 512, 512, 40, 4, 64, "f32"),
+                                  (256, 512, 4096, 1024, 30, 3, 128, "bf16"),
+                                  (200, 384, 2048, 512, 24, 2, 128, "bf16")],
+                         ids=["tiny-f32-full-batch", "multiblock-bf16", "ragged-W2"])
+def test_fp_target_parity(ar, case):
+    out, inn, n, B, iters, bits, g, wdt = case
+    res, ref, *_ = _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed=21)
+    frac = float(np.mean(_np(res.codes) != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
+    trace = _np(res.loss_trace).astype(np.float64)
+    np.testing.assert_allclose(trace[0], ref.loss_trace[0], rtol=5e-3)
+    np.testing.assert_allclose(trace, ref.loss_trace, rtol=0.05)
+
+
+def test_fp_target_with_own_input_is_the_usual_loop(ar):
+    """X_target = X: dX = 0, so every added term is an exact zero and the results
+    equal ar_tune_layer's bit for bit."""
+    W = make_weight(256, 512, 0.02, "bf16", seed=22)
+    X = make_activations(2048, 512, "llm", seed=22)
+    p = ar.make_params(bits=3, group_size=128, iters=20, batch_rows=512, algo="gram")
+    a = ar.tune_layer_fp_target(_w_dev(W, "bf16"), _x_dev(X), _x_dev(X), p)
+    b = ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p)
+    torch.cuda.synchronize()
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.scale, b.scale)
+    assert torch.equal(a.loss_trace, b.loss_trace)
+    assert float(a.final_mse.item()) == float(b.final_mse.item())

@@ -142,6 +142,18 @@ def make_activations(n_rows: int, inn: int, kind: str = "llm", seed: int = 0,
     return bf16_round(z * channel_scale(inn, kind, seed)[None, :])
 
 
+STREAM_QNOISE = 5
+
+
+def make_quantised_path_input(X_fp: np.ndarray, rel: float = 0.05, seed: int = 0) -> np.ndarray:
+    """Stand-in for a layer's input on the quantised path (the output of layers
+    already quantised before it): the full-precision input X_fp with seeded
+    multiplicative noise of relative size ``rel``, rounded to bf16.  Used with
+    X_fp as the target's input in the quant-aware, full-precision-target mode."""
+    z = _rng(seed, STREAM_QNOISE).standard_normal(X_fp.shape, dtype=np.float32)
+    return bf16_round(X_fp * (np.float32(1) + np.float32(rel) * z))
+
+
 def make_activations_cuda(n_rows: int, inn: int, kind: str = "llm", seed: int = 0,
                           stream: int = STREAM_X, device="cuda"):
     """Device-side calibration activations as a torch bf16 tensor [n_rows, inn].
