@@ -20,6 +20,7 @@ bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -183,6 +184,65 @@ def run_block(args):
             "fused_step_tflops": flops / (step_ms * 1e-3) / 1e12,
             "tensor_peak_frac": flops / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
             "gpu_launches": sum(t.kernel_launches for t in timings) + 5 * args.steps,
+            "clocks": clk.summary(), "e2e": None}
+
+
+def run_fp_target(args):
+    """The quant-aware input with a full-precision target (ar_tune_layer_fp_target)
+    on one GPU: the layer's input on the quantised path is the target's input with
+    5% seeded multiplicative noise.  The whole call is timed with CUDA events."""
+    import torch
+
+    import signed_gradient_rounding_b200 as ar
+
+    world, rank, local = _dist()
+    if world > 1:
+        return None if rank else {"metric": METRIC, "unavailable": "--mode fp_target runs on one GPU"}
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    c = WORKLOADS[args.workload]
+    W = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0))
+    Wd = (W.to(torch.bfloat16) if c.w_dtype == "bf16" else W).to(dev)
+    Xt = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    Xq = torch.empty_like(Xt)
+    chunk = max(1, (1 << 27) // c.inn)
+    for r0 in range(0, c.n_rows, chunk):
+        r1 = min(c.n_rows, r0 + chunk)
+        z = torch.randn((r1 - r0, c.inn), generator=gen, device=dev)
+        Xq[r0:r1] = (Xt[r0:r1].float() * (1 + 0.05 * z)).to(torch.bfloat16)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo="gram")
+    ws = torch.empty(int(ar._lib.ar_tune_fp_target_workspace_bytes(c.out, c.inn, c.n_rows,
+                                                                    ar._wdtype(Wd), ctypes.byref(p))),
+                     dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        res = ar.tune_layer_fp_target(Wd, Xq, Xt, p, workspace=ws)
+    torch.cuda.synchronize()
+    if ar.tune_status(ws) != ar.AR_OK:
+        raise RuntimeError("device status not OK after warm-up")
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            res = ar.tune_layer_fp_target(Wd, Xq, Xt, p, workspace=ws)
+            ar.pack(res.codes, c.bits)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if ar.tune_status(ws) != ar.AR_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    return {"metric": METRIC, "value": c.iters * args.steps / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": c.name, "mode": "quant-aware input, full-precision target",
+                       "quantised_path_input": "target input x (1 + 0.05 N(0,1)), bf16", "algo": "gram",
+                       "n_rows": c.n_rows, "batch_rows": c.batch_rows, "iters": c.iters,
+                       "bench_step": "one ar_tune_layer_fp_target call (all iters) + ar_pack"},
+            "layer_tune_s": ms / args.steps / 1e3, "final_mse": float(res.final_mse.item()),
             "clocks": clk.summary(), "e2e": None}
 
 
@@ -441,6 +501,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--algo", choices=["auto", "direct", "gram"], default="auto")
     ap.add_argument("--split", type=int, default=1, help="1: bf16-pair operands (default); 0: single bf16")
+    ap.add_argument("--mode", choices=["layer", "fp_target"], default="layer",
+                    help="fp_target: quant-aware input with a full-precision target")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -448,6 +510,8 @@ def main():
         line = run_reference(args)
     elif args.workload == "block_7b":
         line = run_block(args)
+    elif args.mode == "fp_target":
+        line = run_fp_target(args)
     else:
         line = run_ours(args)
     if line is not None:
