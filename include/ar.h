@@ -365,6 +365,21 @@ ar_status ar_tune_status(const void* workspace, void* stream);
  * status[0] (device int) and exits cleanly.  Returns AR_OK once launched. */
 ar_status ar_selftest_timeout(int32_t* status, uint64_t timeout_ns, void* stream);
 
+/* Test hook for the quantiser's division.  The fake-quantiser forms u = W/s as the
+ * correctly rounded fp32 quotient.  When every weight of a layer is zero or lies
+ * in 2^-100 <= |w| <= 2^20, it gets the quotient from the group's correctly
+ * rounded reciprocal y = 1/s with one fma residual correction (q = RN(W y),
+ * r = s q - W exactly, u = RN(q - r y); P. Markstein, IBM J. Res. Dev. 34(1), 1990),
+ * instead of a full IEEE division.  This hook evaluates both forms for every pair
+ * (a[i], b[j]), i < na, j < nb (device fp32 arrays).  It skips the pairs outside
+ * the fast form's domain: a outside that weight range, b not a positive normal
+ * number at most 2^21 (the scales are positive), or a nonzero a/b that is not a
+ * normal number below 2^64.  It adds the number of pairs whose results differ in
+ * any bit to *mismatches (device uint64), and first_bad[0..1] (device) receive the
+ * first such pair.  Returns AR_OK once launched. */
+ar_status ar_selftest_division(const float* a, int64_t na, const float* b, int64_t nb, uint64_t* mismatches,
+                               float* first_bad, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,7 @@ INITS = {"minmax": AR_INIT_MINMAX, "mse": AR_INIT_MSE}
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
            "ar_tune_host_workspace_bytes", "ar_tune_layer_host", "ar_tune_fp_target_workspace_bytes",
-           "ar_tune_layer_fp_target",
+           "ar_tune_layer_fp_target", "ar_selftest_division",
            "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static", "ar_dequant", "ar_linear",
            "ar_silu_mul")
 
@@ -109,6 +109,8 @@ def _load() -> ctypes.CDLL:
     lib.ar_silu_mul.argtypes = [P, P, I64, P, P]
     lib.ar_tune_status.restype = ctypes.c_int
     lib.ar_tune_status.argtypes = [P, P]
+    lib.ar_selftest_division.restype = ctypes.c_int
+    lib.ar_selftest_division.argtypes = [P, I64, P, I64, P, P, P]
     lib.ar_selftest_timeout.restype = ctypes.c_int
     lib.ar_selftest_timeout.argtypes = [P, U64, P]
     return lib

@@ -302,15 +302,17 @@ void fill_grid(GemmArgs& a, int64_t M, int64_t N, int64_t K, int bn, int num_seg
   a.num_seg = num_seg;
 }
 
-// Events around the contractions of a timed call: ev[2t] before step t's first
-// contraction, ev[2t+1] between the two (DIRECT), ev[2t+2] after the update.
+// Events around the contractions of a timed call, three per step and none shared
+// between steps (work that prepares a block runs between steps): ev[3t] before
+// step t's first contraction, ev[3t+1] after it, ev[3t+2] after the update
+// (DIRECT; the Gram form has one contraction per step and leaves ev[3t+2] unused).
 struct EventTimer {
   std::vector<cudaEvent_t> ev;
   cudaEvent_t start = nullptr, stop = nullptr;
   int launches = 0;
   int algo = 0;
   bool create(int iters) {
-    ev.assign(static_cast<size_t>(2 * iters + 1), nullptr);
+    ev.assign(static_cast<size_t>(3 * iters + 1), nullptr);
     for (auto& e : ev)
       if (cudaEventCreate(&e) != cudaSuccess) return false;
     return cudaEventCreate(&start) == cudaSuccess && cudaEventCreate(&stop) == cudaSuccess;
@@ -363,6 +365,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   auto F = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
   auto H = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
   int* status = reinterpret_cast<int*>(ws + L.status);
+  // Second word of the status block: groups whose weights need the IEEE division.
+  int* div_slow = status + 1;
   uint16_t* Xt = reinterpret_cast<uint16_t*>(ws + L.Xt);
   __nv_bfloat16* D_hi = H(L.D_hi);
   __nv_bfloat16* D_lo = H(L.D_lo);
@@ -409,7 +413,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     timer->algo = P.algo;
     AR_CUDA_TRY(cudaEventRecord(timer->start, st));
   }
-  AR_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), st));
+  AR_CUDA_TRY(cudaMemsetAsync(status, 0, 2 * sizeof(int), st));
   if (init_state) {
     AR_CUDA_TRY(cudaMemsetAsync(Vb[0], 0, elems * 4, st));
     AR_CUDA_TRY(cudaMemsetAsync(V_best, 0, elems * 4, st));
@@ -464,6 +468,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   prep.beta = bb[0];
   prep.D_hi = D_hi;
   prep.D_lo = P.split ? D_lo : nullptr;
+  prep.div_slow = div_slow;
   AR_CUDA_TRY(launch_group_quant(prep, st));
   ++launches;
 
@@ -602,6 +607,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.alpha_best = alpha_best;
   u.beta_best = beta_best;
   u.inv_batch = 1.0f / static_cast<float>(B);
+  u.div_slow = div_slow;
   u.g = static_cast<int>(P.g);
   u.G = static_cast<int>(P.G);
   u.bits = p->bits;
@@ -659,12 +665,9 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
         u.Cc_lo = H(L.Cc_lo) + sched[t] * static_cast<int64_t>(elems);
         u.e_row = F(L.e) + sched[t] * out;
       }
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
       AR_CUDA_TRY(launch_gemm(fpt ? kEpiUpdateFp : kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
-      if (timer) {
-        AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
-        AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
-      }
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
       ++launches;
       if (t > 0) std::swap(best_cur, best_next);
     }
@@ -738,15 +741,15 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       const int64_t b0 = sched[t] * B;
       r.b_row_off = static_cast<int>(b0);
       AR_CUDA_TRY(ensure_block(sched[t]));
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t], st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 1], st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
       u.b_k_off = static_cast<int>(b0);
       u.best_in = best_cur;
       u.best_out = best_next;
       u.rowloss = rowloss + static_cast<int64_t>(t) * out;
       AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, mu, u, sms, st));
-      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[2 * t + 2], st));
+      if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 2], st));
       launches += 2;
       std::swap(best_cur, best_next);
     }
@@ -940,10 +943,11 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
   if (out == 0 || in == 0) return AR_OK;
   float ms = 0.f;
   for (int t = 0; t < p->iters; ++t) {
-    if (cudaEventElapsedTime(&ms, timer.ev[2 * t], timer.ev[2 * t + 1]) != cudaSuccess) return AR_ECUDA;
-    if (timer.algo == AR_ALGO_DIRECT) timing->residual_ms += ms;
-    else timing->update_ms += ms;
-    if (cudaEventElapsedTime(&ms, timer.ev[2 * t + 1], timer.ev[2 * t + 2]) != cudaSuccess) return AR_ECUDA;
+    if (cudaEventElapsedTime(&ms, timer.ev[3 * t], timer.ev[3 * t + 1]) != cudaSuccess) return AR_ECUDA;
+    if (timer.algo == AR_ALGO_DIRECT) {
+      timing->residual_ms += ms;
+      if (cudaEventElapsedTime(&ms, timer.ev[3 * t + 1], timer.ev[3 * t + 2]) != cudaSuccess) return AR_ECUDA;
+    }
     timing->update_ms += ms;
   }
   if (p->iters > 0) {
@@ -1132,6 +1136,13 @@ ar_status ar_tune_status(const void* workspace, void* stream) {
   if (word == kDevOk) return AR_OK;
   if (word == kDevTimeout) return AR_ETIMEOUT;
   return AR_ECUDA;
+}
+
+ar_status ar_selftest_division(const float* a, int64_t na, const float* b, int64_t nb, uint64_t* mismatches,
+                               float* first_bad, void* stream) {
+  if ((na > 0 && !a) || (nb > 0 && !b) || !mismatches || !first_bad || na < 0 || nb < 0) return AR_EINVAL;
+  return from_cuda(launch_division_selftest(a, na, b, nb, reinterpret_cast<unsigned long long*>(mismatches),
+                                            first_bad, static_cast<cudaStream_t>(stream)));
 }
 
 ar_status ar_selftest_timeout(int32_t* status, uint64_t timeout_ns, void* stream) {

@@ -18,8 +18,9 @@ namespace ar {
 // ---------------------------------------------------------------------------
 
 struct GroupScale {
-  float s;   // scale
-  float zp;  // zero-point (integer-valued)
+  float s;    // scale
+  float zp;   // zero-point (integer-valued)
+  float rcp;  // 1/s correctly rounded (for div_rn_by)
 };
 
 __device__ __forceinline__ float qmaxf(int bits) { return (float)((1 << bits) - 1); }
@@ -39,7 +40,32 @@ __device__ __forceinline__ GroupScale group_scale(float wmin, float wmax, float 
     if (g.s == 0.0f) g.s = 1.0f;
     g.zp = fminf(fmaxf(rintf(__fdiv_rn(-__fmul_rn(beta, wmin), g.s)), 0.0f), Q);
   }
+  g.rcp = __frcp_rn(g.s);
   return g;
+}
+
+// Weights whose quotients by their group's scale div_rn_by may form: zero, or
+// 2^-100 <= |w| <= 2^20.  With every weight of a group in that range the scale is a
+// normal number below 2^21, and each quotient and each residual w - s*q of the
+// division is a normal number.
+__device__ __forceinline__ bool div_fast_ok(float w) {
+  const float m = fabsf(w);
+  return w == 0.0f || (m >= 0x1p-100f && m <= 0x1p20f);
+}
+
+// a / b correctly rounded, from y = 1/b correctly rounded, by one residual
+// correction (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also Muller et al.,
+// Handbook of Floating-Point Arithmetic, ch. "Newton-Raphson-based division with
+// an FMA"): q = RN(a y) is within one ulp of a/b, the residual q b - a is exact in
+// one fma, and RN(q - (q b - a) y) is the correctly rounded quotient.  (Writing the
+// residual as q b - a keeps the sign of a zero quotient.)  Valid for b > 0 when
+// a/b and the residual are normal numbers: for div_fast_ok weights divided by
+// their group's (positive) scale.
+__device__ __forceinline__ float div_rn_by(float a, float b, float y) {
+  const float q = __fmul_rn(a, y);
+  const float r = __fmaf_rn(q, b, -a);
+  return __fmaf_rn(-r, y, q);
 }
 
 struct ElemQuant {
@@ -50,9 +76,10 @@ struct ElemQuant {
   float wq;  // s * (q - zp)
 };
 
-__device__ __forceinline__ ElemQuant quant_elem(float w, float v, GroupScale g, float Q) {
+// fast: every weight of the layer is div_fast_ok, so W/s may use div_rn_by.
+__device__ __forceinline__ ElemQuant quant_elem(float w, float v, GroupScale g, float Q, bool fast = false) {
   ElemQuant e;
-  e.u = __fdiv_rn(w, g.s);
+  e.u = fast ? div_rn_by(w, g.s, g.rcp) : __fdiv_rn(w, g.s);
   e.r = rintf(__fadd_rn(e.u, v));
   const float p = __fadd_rn(e.r, g.zp);
   e.q = fminf(fmaxf(p, 0.0f), Q);

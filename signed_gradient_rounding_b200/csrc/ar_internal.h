@@ -29,6 +29,8 @@ struct GroupQuantArgs {
   float* Wq = nullptr;             // [out, in] fp32 s*(q - zp)
   __nv_bfloat16* D_hi = nullptr;   // [out, in] D = s*(q - zp) - W as hi = bf16(D) ...
   __nv_bfloat16* D_lo = nullptr;   // ... and lo = bf16(D - hi) (may be null)
+  int* div_slow = nullptr;         // when set: +1 for every group that has a weight
+                                   // that is not div_fast_ok (W/s must use __fdiv_rn)
 };
 
 cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream);
@@ -50,6 +52,8 @@ cudaError_t launch_loss_trace(const float* rowloss, int64_t out, int iters, int6
 cudaError_t launch_sum_to_double(const float* parts, int64_t count, double denom, double* result,
                                  cudaStream_t stream);
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_division_selftest(const float* a, int64_t na, const float* b, int64_t nb,
+                                     unsigned long long* bad, float* first, cudaStream_t stream);
 
 // Keep-best check of the last step of a Gram-form run (its loss is complete only
 // after the step's launch): per row j, L = sum of part[j, 0 .. nparts) in order,
@@ -183,6 +187,9 @@ struct GemmArgs {
   const __nv_bfloat16* Cc_lo = nullptr;
   const float* Cs = nullptr;
   const float* e_row = nullptr;
+  // kEpiUpdate*: *div_slow == 0 (counted by the prepare pass) lets W/s use the
+  // fast correctly rounded division; null means always __fdiv_rn.
+  const int* div_slow = nullptr;
   float inv_batch = 1.0f;
   int g = 0, G = 0, bits = 4, sym = 0, keep_best = 1;
   float lr = 0.f, mlr = 0.f;

@@ -385,6 +385,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
   }
   const bool snap_now = better && !a.snap_prev;
   const bool snap_old = better && a.snap_prev;
+  const bool fast = a.div_slow && *a.div_slow == 0;
 
   int gl_begin, gl_end;
   epi_group_range<kBN>(a, half, gl_begin, gl_end);
@@ -465,7 +466,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       float vn[kUC];
 #pragma unroll
       for (int i = 0; i < kUC; ++i) {
-        const ElemQuant e = quant_elem(w[i], v[i], gs, Q);
+        const ElemQuant e = quant_elem(w[i], v[i], gs, Q, fast);
         const float d = __fsub_rn(e.wq, w[i]);
         float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
         if (kFp) {
@@ -527,7 +528,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
         load_f32x16(a.V_out + e0 + kUC, v_nx);
       }
 #pragma unroll
-      for (int i = 0; i < kUC; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q).wq, w[i]);
+      for (int i = 0; i < kUC; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q, fast).wq, w[i]);
 #pragma unroll
       for (int q = 0; q < kUC / 8; ++q)
         store_pair8(d + q * 8, a.D_hi + e0 + q * 8, a.D_lo ? a.D_lo + e0 + q * 8 : nullptr);

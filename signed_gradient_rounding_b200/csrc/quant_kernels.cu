@@ -26,24 +26,27 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
   const int64_t col0 = (warp - row * a.G) * a.g;
   const int64_t base = row * a.in + col0;
 
-  float wmin, wmax;
+  // Group statistics, and whether every weight of the group admits the fast
+  // correctly rounded division by the group's scale (div_fast_ok).
+  float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W)
+  bool ok = true;
+  for (int k = lane; k < a.g; k += 32) {
+    const float w = load_w(a.W, a.w_bf16, base + k);
+    mn = fminf(mn, w);
+    mx = fmaxf(mx, w);
+    ok = ok && div_fast_ok(w);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const bool fast = __all_sync(0xffffffffu, ok);
+  if (!fast && lane == 0 && a.div_slow) atomicAdd(a.div_slow, 1);
+  float wmin = mn, wmax = mx;
   if (a.wmin_in) {
     wmin = a.wmin_in[warp];
     wmax = a.wmax_in[warp];
-  } else {
-    float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W)
-    for (int k = lane; k < a.g; k += 32) {
-      const float w = load_w(a.W, a.w_bf16, base + k);
-      mn = fminf(mn, w);
-      mx = fmaxf(mx, w);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    wmin = mn;
-    wmax = mx;
   }
   const float alpha = a.alpha ? a.alpha[warp] : 1.0f;
   const float beta = a.beta ? a.beta[warp] : 1.0f;
@@ -61,7 +64,7 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
   for (int k = lane; k < a.g; k += 32) {
     const float w = load_w(a.W, a.w_bf16, base + k);
     const float v = a.V ? a.V[base + k] : 0.0f;
-    const ElemQuant e = quant_elem(w, v, gs, Q);
+    const ElemQuant e = quant_elem(w, v, gs, Q, fast);
     if (a.codes) a.codes[base + k] = static_cast<uint8_t>(e.q);
     if (a.Wq) a.Wq[base + k] = e.wq;
     if (a.D_hi) {
@@ -166,11 +169,14 @@ __global__ void mse_init_kernel(const void* __restrict__ W, int w_bf16, int64_t 
   auto wat = [&](int k) { return w_bf16 ? bf16_bits_to_f32(wb[k]) : wf[k]; };
 
   float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W) of the group
+  bool ok = true;
   for (int k = lane; k < g; k += 32) {
     const float w = wat(k);
     mn = fminf(mn, w);
     mx = fmaxf(mx, w);
+    ok = ok && div_fast_ok(w);
   }
+  const bool fast = __all_sync(0xffffffffu, ok);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -186,7 +192,7 @@ __global__ void mse_init_kernel(const void* __restrict__ W, int w_bf16, int64_t 
     double acc = 0.0;
     for (int k = 0; k < g; ++k) {
       const float w = wat(k);
-      const double d = static_cast<double>(__fsub_rn(quant_elem(w, 0.0f, gs, Q).wq, w));
+      const double d = static_cast<double>(__fsub_rn(quant_elem(w, 0.0f, gs, Q, fast).wq, w));
       acc = fma(d, d, acc);
     }
     if (live && (acc < best_e || (acc == best_e && i < best_i))) {
@@ -515,6 +521,35 @@ cudaError_t launch_loss_trace(const float* rowloss, int64_t out, int iters, int6
 cudaError_t launch_sum_to_double(const float* parts, int64_t count, double denom, double* result,
                                  cudaStream_t stream) {
   sum_to_double_kernel<<<1, 1024, 0, stream>>>(parts, count, denom, result);
+  return cudaGetLastError();
+}
+
+// Every pair (a[i], b[j]) in the fast division's domain -- div_fast_ok(a[i]), b[j]
+// a positive normal number at most 2^21 (a scale), and a/b zero or a normal number
+// below 2^64 in magnitude -- counts the pairs where the quantiser's fast quotient
+// differs in any bit from __fdiv_rn, and records the first such pair found.
+__global__ void division_selftest_kernel(const float* __restrict__ a, int64_t na, const float* __restrict__ b,
+                                         int64_t nb, unsigned long long* __restrict__ bad, float* __restrict__ first) {
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < na * nb;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float x = a[t % na], y = b[t / na];
+    if (!div_fast_ok(x) || !(y >= 0x1p-126f) || !(y <= 0x1p21f)) continue;
+    const float exact = __fdiv_rn(x, y);
+    if (!(fabsf(exact) < 0x1p64f) || (x != 0.0f && !(fabsf(exact) >= 0x1p-126f))) continue;
+    const float fast = div_rn_by(x, y, __frcp_rn(y));
+    if (__float_as_uint(fast) != __float_as_uint(exact)) {
+      if (atomicAdd(bad, 1ull) == 0ull) {
+        first[0] = x;
+        first[1] = y;
+      }
+    }
+  }
+}
+
+cudaError_t launch_division_selftest(const float* a, int64_t na, const float* b, int64_t nb,
+                                     unsigned long long* bad, float* first, cudaStream_t stream) {
+  if (na <= 0 || nb <= 0) return cudaSuccess;
+  division_selftest_kernel<<<148 * 8, 256, 0, stream>>>(a, na, b, nb, bad, first);
   return cudaGetLastError();
 }
 
