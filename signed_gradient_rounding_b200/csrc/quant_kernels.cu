@@ -110,7 +110,11 @@ __global__ void fill_f32_kernel(float* p, int64_t n, float v) {
 // Xt[c * ld_t + r] = X[r * cols + c].  64 x 64 tiles through shared memory; 256
 // threads.  Full tiles move 16-byte vectors both ways (rows, cols and ld_t
 // multiples of 8 keep them aligned); the tile's ragged edges fall back to single
-// elements.
+// elements.  In shared memory, the 16-byte chunk j of tile row r sits at chunk
+// j ^ ((r >> 3) & 7): the eight rows 8m + k that one read instruction gathers
+// (one per m, for a fixed column) then fall in eight different banks.
+__device__ __forceinline__ int tile_chunk(int r, int chunk) { return chunk ^ ((r >> 3) & 7); }
+
 __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
                                       uint16_t* __restrict__ Xt, int64_t ld_t) {
   __shared__ __align__(16) uint16_t tile[64][72];
@@ -119,15 +123,16 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t ro
   const bool full = (r0 + 64 <= rows) && (c0 + 64 <= cols) && (rows % 8 == 0) && (cols % 8 == 0) && (ld_t % 8 == 0);
   if (full) {
     for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 rows x 8 vectors
-      const int r = v >> 3, c8 = (v & 7) * 8;
-      *reinterpret_cast<uint4*>(&tile[r][c8]) = *reinterpret_cast<const uint4*>(X + (r0 + r) * cols + c0 + c8);
+      const int r = v >> 3, ch = v & 7;
+      *reinterpret_cast<uint4*>(&tile[r][tile_chunk(r, ch) * 8]) =
+          *reinterpret_cast<const uint4*>(X + (r0 + r) * cols + c0 + ch * 8);
     }
     __syncthreads();
     for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 output rows (cols of X) x 8 vectors
       const int c = v >> 3, r8 = (v & 7) * 8;
       uint16_t e[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) e[k] = tile[r8 + k][c];
+      for (int k = 0; k < 8; ++k) e[k] = tile[r8 + k][tile_chunk(r8 + k, c >> 3) * 8 + (c & 7)];
       uint4 o;
       o.x = e[0] | (uint32_t(e[1]) << 16);
       o.y = e[2] | (uint32_t(e[3]) << 16);
