@@ -38,6 +38,8 @@
 // Every mbarrier wait is bounded (GemmArgs::timeout_ns); a role that gives up
 // records the timeout in *status and the CTA drains its in-flight copies and MMAs
 // before it frees tensor memory and exits.
+#include <atomic>
+
 #include "ar_device.cuh"
 #include "ar_internal.h"
 
@@ -813,16 +815,17 @@ cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cu
   cfg.numAttrs = 1;
   // A persistent grid must not exceed the clusters that can be resident at once
   // (a pair needs two SMs of one GPC): queried once per device.
-  static int resident[64];  // 0: not yet known
+  // (One cache per kernel instance; host threads may launch concurrently.)
+  static std::atomic<int> resident[64];  // 0: not yet known
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int max_pairs = (dev >= 0 && dev < 64) ? resident[dev] : 0;
+  int max_pairs = (dev >= 0 && dev < 64) ? resident[dev].load(std::memory_order_relaxed) : 0;
   if (max_pairs <= 0) {
     e = cudaOccupancyMaxActiveClusters(&max_pairs, fn, &cfg);
     if (e != cudaSuccess) return e;
     if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
-    if (dev >= 0 && dev < 64) resident[dev] = max_pairs;
+    if (dev >= 0 && dev < 64) resident[dev].store(max_pairs, std::memory_order_relaxed);
   }
   int pairs = args.num_tiles < num_sms / 2 ? args.num_tiles : num_sms / 2;
   if (pairs > max_pairs) pairs = max_pairs;
