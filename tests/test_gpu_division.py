@@ -89,3 +89,26 @@ def test_random_fp32(ar):
     b = b[np.isfinite(b)]
     bad, first = _run(ar, a, b)
     assert bad == 0, f"{bad} mismatches, first at a={first[0]!r} b={first[1]!r}"
+
+
+@pytest.mark.parametrize("algo", ["direct", "gram"])
+def test_tuning_with_tiny_and_zero_weights(ar, algo):
+    """A layer with nonzero weights below 2^-100 takes the IEEE division in every
+    pass (the fast form's domain check fails); with a zero group as well, the
+    tuned result still meets the parity bars against the oracle."""
+    import oracle
+    from workloads import TINY, make_activations, make_weight
+    c = TINY
+    W = make_weight(c.out, c.inn, c.w_std, "f32", seed=3)
+    W[5, 3] = np.float32(1e-35)              # below 2^-100: no fast division anywhere
+    W[6, 10] = np.float32(-3e-38)
+    W[7, 64:128] = 0.0                       # an all-zero group
+    X = make_activations(c.n_rows, c.inn, c.x_kind, seed=3)
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=30, batch_rows=c.batch_rows, algo=algo)
+    res = ar.tune_layer(torch.from_numpy(W).cuda(), torch.from_numpy(X).to(torch.bfloat16).cuda(), p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, X, c.bits, c.group_size, False, 30, 0.005, -1.0, c.batch_rows, 0)
+    codes = res.codes.cpu().numpy()
+    assert float(np.mean(codes != ref.codes)) <= 0.005
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=0.02)
+    assert np.all(codes[7, 64:128] == ref.codes[7, 64:128])
