@@ -110,3 +110,11 @@ def test_tune_layer_uses_mse_ratios_at_step_zero():
     s, _ = oar.scale_zero_point(wmin, wmax, p, p, 2, False)
     assert np.array_equal(res.scale, s)
     assert np.array_equal(res.alpha, p) and np.array_equal(res.beta, p)
+
+
+def test_all_zero_group_keeps_full_range():
+    """Every ratio gives an all-zero group zero error: the first minimum (p = 1) is kept."""
+    W = np.zeros((2, 64), dtype=np.float32)
+    W[1, :32] = np.random.default_rng(6).normal(0, 0.02, 32).astype(np.float32)   # one live group
+    p, e = oar.mse_init(W, 32, 4, False)
+    assert p[0, 0] == F32(1.0) and p[0, 1] == F32(1.0) and e[0, 0] == 0.0

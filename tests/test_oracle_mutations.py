@@ -70,7 +70,8 @@ def _fq_round_half_up(W, V, s, zp, group_size, bits):
 def _plant(monkeypatch, name, fn):
     """Replace an oracle function everywhere it can be reached from."""
     monkeypatch.setattr(oar, name, fn)
-    monkeypatch.setattr(oracle, name, fn)
+    if hasattr(oracle, name):
+        monkeypatch.setattr(oracle, name, fn)
 
 
 def _caught(*checks) -> bool:
@@ -117,3 +118,57 @@ def test_rounding_mode_is_caught(monkeypatch):
     _plant(monkeypatch, "fake_quant", _fq_round_half_up)
     with pytest.raises(AssertionError):
         pins.test_rounding_is_torch_round()
+
+
+# ---------------------------------------------------------------- MSE init and full-precision target
+
+from tests import test_oracle_mse_init as mse_pins  # noqa: E402
+
+_orig_mse_init = oar.mse_init
+
+
+def _mse_init_variant(W, group_size, bits, sym, score="l2", beta_one=False, last_min=False):
+    """mse_init with one slip: an L1 score, beta left at 1, or the last minimum kept."""
+    W = oar._to_f32(W)
+    out, inn = W.shape
+    g = oar._group(inn, group_size)
+    wmin, wmax = oar.group_minmax(W, g)
+    best_p = np.ones(wmin.shape, dtype=F32)
+    best_e = np.full(wmin.shape, np.inf)
+    for i in range(oar.MSE_GRID):
+        p = F32(100 - i) / F32(100)
+        a = np.full(wmin.shape, p, dtype=F32)
+        b = np.ones_like(a) if beta_one else a
+        sc, zp = oar.scale_zero_point(wmin, wmax, a, b, bits, sym)
+        d = oar.fake_quant(W, np.zeros_like(W), sc, zp, g, bits).Wq - W
+        d = d.astype(np.float64).reshape(out, inn // g, g)
+        e = np.cumsum(np.abs(d) if score == "l1" else d * d, axis=2)[:, :, -1]
+        better = (e <= best_e) if last_min else (e < best_e)
+        best_e = np.where(better, e, best_e)
+        best_p = np.where(better, p, best_p).astype(F32)
+    return best_p, best_e
+
+
+MSE_PINS = (lambda: mse_pins.test_grid_aligned_group_keeps_full_range(),
+            lambda: mse_pins.test_exact_brute_force_agrees(2, False),
+            lambda: mse_pins.test_exact_brute_force_agrees(4, False),
+            lambda: mse_pins.test_never_worse_than_rtn(2, False),
+            lambda: mse_pins.test_all_zero_group_keeps_full_range())
+
+
+@pytest.mark.parametrize("slip", [dict(score="l1"), dict(beta_one=True), dict(last_min=True)],
+                         ids=["l1-score", "beta-left-at-1", "last-minimum"])
+def test_mse_init_mistakes_are_caught(monkeypatch, slip):
+    _plant(monkeypatch, "mse_init", lambda W, gs, bits, sym: _mse_init_variant(W, gs, bits, sym, **slip))
+    assert _caught(*MSE_PINS)
+
+
+def test_dropped_target_input_is_caught(monkeypatch):
+    """The full-precision-target mode silently running the usual loop."""
+    orig = oar.tune_layer
+
+    def dropped(*args, X_target=None, **kw):
+        return orig(*args, **kw)
+    _plant(monkeypatch, "tune_layer", dropped)
+    assert _caught(lambda: pins.test_fp_target_gradients_match_autograd(False),
+                   lambda: pins.test_fp_target_final_mse_and_same_input())
