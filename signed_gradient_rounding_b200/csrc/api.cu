@@ -157,6 +157,9 @@ struct Plan {
   // Gram-form update GEMM on 2-SM pair tiles (256 x 256, tcgen05 cta_group::2):
   // each SM stages 32 KB per K block instead of 48 KB, so six stages fit.
   bool pair_upd = true;
+  // ... with the three pair products fused per K block (Cfg::kFused): the hi tiles
+  // of D and H are staged once per K block rather than twice.
+  bool fused_upd = true;
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
@@ -635,6 +638,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     }
     fill_grid(u, out, in, in, P.bn_upd, nseg_g, P.pair_upd);
     u.raster_m = P.raster_upd;
+    u.fused = (P.fused_upd && P.pair_upd && nseg_g > 1) ? 1 : 0;
     // (D_hi + D_lo)(H_hi + H_lo) ~ D_hi H_hi + D_lo H_hi + D_hi H_lo
     u.seg_a[0] = 0, u.seg_b[0] = 0;
     u.seg_a[1] = 1, u.seg_b[1] = 0;

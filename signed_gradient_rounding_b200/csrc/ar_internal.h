@@ -140,6 +140,9 @@ struct GemmArgs {
   // 2-SM pair tiles (tcgen05 cta_group::2, clusters of two CTAs): 256 x 256 tiles,
   // num_m_blk counts 256-row blocks, B maps use 128-row boxes.
   int pair = 0;
+  // Pair tiles only: one stage per K block holds every operand tile the segments
+  // use (each loaded once) and the MMA warp issues all segments from it.
+  int fused = 0;
   // Tile order: 0 = m fastest over all rows; g > 0 = groups of g m-blocks, m fastest
   // inside a group, the group's n-blocks in turn (keeps a wave's operands compact).
   int raster_m = 0;

@@ -52,11 +52,17 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTileABytes = kBM * kBK * 2;  // 16 KB
 
 // Per-CTA operand staging: 128 A rows and kBN (pair: kBN / 2) B rows per stage.
-template <int kBN, bool kPair>
+// kFused: a stage holds one K block of both operand maps of A and of B (up to
+// four tiles), and the MMA warp issues every segment's product from it, so a
+// pair operand's hi tile crosses from L2 once per K block instead of twice.
+template <int kBN, bool kPair, bool kFused = false>
 struct Cfg {
   static constexpr int kTileBBytes = (kPair ? kBN / 2 : kBN) * kBK * 2;
-  static constexpr int kStageBytes = kTileABytes + kTileBBytes;
-  static constexpr int kStages = (kStageBytes <= 32 * 1024) ? 6 : 4;
+  static constexpr int kStageBytes = (kFused ? 2 : 1) * (kTileABytes + kTileBBytes);
+  static constexpr int kStages = (kStageBytes <= 32 * 1024) ? 6 : (kStageBytes <= 48 * 1024 ? 4 : 3);
+  static constexpr int kOffA1 = kTileABytes;  // kFused: A0, A1, B0, B1
+  static constexpr int kOffB0 = kFused ? 2 * kTileABytes : kTileABytes;
+  static constexpr int kOffB1 = kOffB0 + kTileBBytes;
   static constexpr int kTmemCols = 2 * kBN;
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kSmemBytes = kBarOffset + 1024 + 1024;
@@ -571,12 +577,12 @@ __device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, in
 // full barrier; the leader's MMA thread alone issues M = 256 MMAs and its commits
 // arrive on both CTAs' barriers; each CTA's epilogue reads its own 128 accumulator
 // rows and releases the accumulator with one arrive per warp on the leader.
-template <int kKind, int kBN, bool kPair>
+template <int kKind, int kBN, bool kPair, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                 const __grid_constant__ GemmArgs args) {
-  using C = Cfg<kBN, kPair>;
+  using C = Cfg<kBN, kPair, kFused>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
@@ -625,7 +631,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (kPair) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = sm->tmem_base;
-  const int k_blocks = args.num_seg * args.num_k_blk;
+  // kFused: one stage per K block carries every segment; otherwise one per
+  // (segment, K block), segments outermost.
+  const int k_blocks = kFused ? args.num_k_blk : args.num_seg * args.num_k_blk;
+  // kFused: which of the two maps of A and of B the segments use.
+  bool use_a0 = false, use_a1 = false, use_b0 = false, use_b1 = false;
+  for (int s = 0; s < args.num_seg; ++s) {
+    (args.seg_a[s] ? use_a1 : use_a0) = true;
+    (args.seg_b[s] ? use_b1 : use_b0) = true;
+  }
+  const uint32_t fused_bytes = (use_a0 + use_a1) * kTileABytes + (use_b0 + use_b1) * C::kTileBBytes;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -650,7 +665,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sA = smem + stage * C::kStageBytes;
           uint8_t* sB = sA + kTileABytes;
-          if (kPair) {
+          if (kFused) {
+            const uint32_t tx = kPair ? 2 * fused_bytes : fused_bytes;
+            if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], tx);
+            const int ka = kb * kBK + args.a_k_off, kbb = kb * kBK + args.b_k_off;
+            if (kPair) {
+              const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
+              if (use_a0) tma_load_2d_pair(sA, &tmA0, ka, a_row, leader_full);
+              if (use_a1) tma_load_2d_pair(sA + C::kOffA1, &tmA1, ka, a_row, leader_full);
+              if (use_b0) tma_load_2d_pair(sA + C::kOffB0, &tmB0, kbb, b_row, leader_full);
+              if (use_b1) tma_load_2d_pair(sA + C::kOffB1, &tmB1, kbb, b_row, leader_full);
+            } else {
+              if (use_a0) tma_load_2d(sA, &tmA0, ka, a_row, &sm->full[stage]);
+              if (use_a1) tma_load_2d(sA + C::kOffA1, &tmA1, ka, a_row, &sm->full[stage]);
+              if (use_b0) tma_load_2d(sA + C::kOffB0, &tmB0, kbb, b_row, &sm->full[stage]);
+              if (use_b1) tma_load_2d(sA + C::kOffB1, &tmB1, kbb, b_row, &sm->full[stage]);
+            }
+          } else if (kPair) {
             if (rank == 0) mbar_arrive_expect_tx(&sm->full[stage], 2 * C::kStageBytes);
             const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
             tma_load_2d_pair(sA, mA, kk * kBK + args.a_k_off, a_row, leader_full);
@@ -704,14 +735,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint64_t a_desc = umma_desc_sw128(a_addr);
-          const uint64_t b_desc = umma_desc_sw128(a_addr + kTileABytes);
+          if (kFused) {
+            for (int s = 0; s < args.num_seg; ++s) {
+              const uint64_t a_desc = umma_desc_sw128(a_addr + (args.seg_a[s] ? C::kOffA1 : 0));
+              const uint64_t b_desc = umma_desc_sw128(a_addr + (args.seg_b[s] ? C::kOffB1 : C::kOffB0));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            if (kPair)
-              umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
-            else
-              umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < kBK / 16; ++k) {
+                const uint32_t accum = (kb | s | k) != 0 ? 1u : 0u;
+                if (kPair)
+                  umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, accum);
+                else
+                  umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, accum);
+              }
+            }
+          } else {
+            const uint64_t a_desc = umma_desc_sw128(a_addr);
+            const uint64_t b_desc = umma_desc_sw128(a_addr + kTileABytes);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              if (kPair)
+                umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+              else
+                umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+            }
           }
           if (kPair)
             umma_commit_pair_both(&sm->empty[stage]);
@@ -789,10 +835,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kKind, int kBN, bool kPair>
+template <int kKind, int kBN, bool kPair, bool kFused>
 cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
-  using C = Cfg<kBN, kPair>;
-  auto* fn = gemm_kernel<kKind, kBN, kPair>;
+  using C = Cfg<kBN, kPair, kFused>;
+  auto* fn = gemm_kernel<kKind, kBN, kPair, kFused>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (!kPair) {
@@ -836,19 +882,19 @@ cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cu
   return cudaGetLastError();
 }
 
-template <int kBN, bool kPair>
+template <int kBN, bool kPair, bool kFused = false>
 cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
   switch (kind) {
     case kEpiStore:
-      return launch_kind<kEpiStore, kBN, kPair>(m, args, num_sms, stream);
+      return launch_kind<kEpiStore, kBN, kPair, kFused>(m, args, num_sms, stream);
     case kEpiSumSq:
-      return launch_kind<kEpiSumSq, kBN, kPair>(m, args, num_sms, stream);
+      return launch_kind<kEpiSumSq, kBN, kPair, kFused>(m, args, num_sms, stream);
     case kEpiUpdate:
-      return launch_kind<kEpiUpdate, kBN, kPair>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdate, kBN, kPair, kFused>(m, args, num_sms, stream);
     case kEpiDotD:
-      return launch_kind<kEpiDotD, kBN, kPair>(m, args, num_sms, stream);
+      return launch_kind<kEpiDotD, kBN, kPair, kFused>(m, args, num_sms, stream);
     case kEpiUpdateFp:
-      return launch_kind<kEpiUpdateFp, kBN, kPair>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdateFp, kBN, kPair, kFused>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -861,6 +907,7 @@ cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmAr
   if (args.pair) {
     // Pair tiles: 256 rows x 256 columns; B maps with 128-row boxes; no symmetric mode.
     if (bn != 256 || args.symmetric) return cudaErrorInvalidValue;
+    if (args.fused) return launch_bn<256, true, true>(kind, maps, args, num_sms, stream);
     return launch_bn<256, true>(kind, maps, args, num_sms, stream);
   }
   if (bn == 256) return launch_bn<256, false>(kind, maps, args, num_sms, stream);
