@@ -160,6 +160,9 @@ struct Plan {
   // ... with the three pair products fused per K block (Cfg::kFused): the hi tiles
   // of D and H are staged once per K block rather than twice.
   bool fused_upd = true;
+  // Direct form (residual, update, final MSE): X_b (or X_b^T) staged once per K
+  // block for both halves of the pair operand instead of once per half.
+  bool fused_direct = true;
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
@@ -720,6 +723,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     fill_grid(r, out, B, in, P.bn_res, nseg_d, P.pair_direct);
     r.raster_m = P.raster_upd;
     r.seg_a[1] = 1;
+    r.fused = (P.fused_direct && nseg_d > 1) ? 1 : 0;
     r.timeout_ns = timeout_ns;
     r.status = status;
     r.C_hi = Rh;
@@ -731,6 +735,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     fill_grid(u, out, in, B, P.bn_upd, nseg_d, P.pair_direct);  // update: G = (R_hi + R_lo)^T X_b
     u.raster_m = P.raster_upd;
     u.seg_a[1] = 1;
+    u.fused = r.fused;
     u.V_in = Vb[0];
     u.V_out = Vb[0];
     u.alpha_in = ab[0];
@@ -834,6 +839,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       m.b1 = m.b0;
       fill_grid(f, out, n_rows, in, P.bn_fin, nseg_d);
       f.seg_a[1] = 1;
+      f.fused = (P.fused_direct && nseg_d > 1) ? 1 : 0;
       f.part_ld = f.num_n_blk * kEpiHalves;
       AR_CUDA_TRY(launch_gemm(kEpiSumSq, P.bn_fin, m, f, sms, st));
       ++launches;

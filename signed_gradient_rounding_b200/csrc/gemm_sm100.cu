@@ -52,16 +52,19 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTileABytes = kBM * kBK * 2;  // 16 KB
 
 // Per-CTA operand staging: 128 A rows and kBN (pair: kBN / 2) B rows per stage.
-// kFused: a stage holds one K block of both operand maps of A and of B (up to
-// four tiles), and the MMA warp issues every segment's product from it, so a
-// pair operand's hi tile crosses from L2 once per K block instead of twice.
-template <int kBN, bool kPair, bool kFused = false>
+// Fused stages (kNA > 0): a stage holds one K block of each of the kNA A maps and
+// kNB B maps the segments use, and the MMA warp issues every segment's product
+// from it, so an operand that several segments share (the hi half of a pair, or a
+// plain operand multiplied by both halves of the other) is staged once per K block
+// instead of once per segment.  kNA = kNB = 0: one stage per (segment, K block).
+template <int kBN, bool kPair, int kNA = 0, int kNB = 0>
 struct Cfg {
+  static constexpr bool kFused = kNA > 0;
   static constexpr int kTileBBytes = (kPair ? kBN / 2 : kBN) * kBK * 2;
-  static constexpr int kStageBytes = (kFused ? 2 : 1) * (kTileABytes + kTileBBytes);
+  static constexpr int kStageBytes = kFused ? kNA * kTileABytes + kNB * kTileBBytes : kTileABytes + kTileBBytes;
   static constexpr int kStages = (kStageBytes <= 32 * 1024) ? 6 : (kStageBytes <= 48 * 1024 ? 4 : 3);
-  static constexpr int kOffA1 = kTileABytes;  // kFused: A0, A1, B0, B1
-  static constexpr int kOffB0 = kFused ? 2 * kTileABytes : kTileABytes;
+  static constexpr int kOffA1 = kTileABytes;  // fused: A0, (A1,) B0, (B1)
+  static constexpr int kOffB0 = kFused ? kNA * kTileABytes : kTileABytes;
   static constexpr int kOffB1 = kOffB0 + kTileBBytes;
   static constexpr int kTmemCols = 2 * kBN;
   static constexpr int kBarOffset = kStages * kStageBytes;
@@ -577,12 +580,13 @@ __device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, in
 // full barrier; the leader's MMA thread alone issues M = 256 MMAs and its commits
 // arrive on both CTAs' barriers; each CTA's epilogue reads its own 128 accumulator
 // rows and releases the accumulator with one arrive per warp on the leader.
-template <int kKind, int kBN, bool kPair, bool kFused>
+template <int kKind, int kBN, bool kPair, int kNA, int kNB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                 const __grid_constant__ GemmArgs args) {
-  using C = Cfg<kBN, kPair, kFused>;
+  using C = Cfg<kBN, kPair, kNA, kNB>;
+  constexpr bool kFused = C::kFused;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
@@ -635,12 +639,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (segment, K block), segments outermost.
   const int k_blocks = kFused ? args.num_k_blk : args.num_seg * args.num_k_blk;
   // kFused: which of the two maps of A and of B the segments use.
-  bool use_a0 = false, use_a1 = false, use_b0 = false, use_b1 = false;
+  bool use_a1 = false, use_b1 = false;
   for (int s = 0; s < args.num_seg; ++s) {
-    (args.seg_a[s] ? use_a1 : use_a0) = true;
-    (args.seg_b[s] ? use_b1 : use_b0) = true;
+    use_a1 = use_a1 || args.seg_a[s] != 0;
+    use_b1 = use_b1 || args.seg_b[s] != 0;
   }
-  const uint32_t fused_bytes = (use_a0 + use_a1) * kTileABytes + (use_b0 + use_b1) * C::kTileBBytes;
+  // With one map of an operand staged, it is whichever one the segments use.
+  const CUtensorMap* map_a0 = (kNA == 1 && use_a1) ? &tmA1 : &tmA0;
+  const CUtensorMap* map_b0 = (kNB == 1 && use_b1) ? &tmB1 : &tmB0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -666,20 +672,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sA = smem + stage * C::kStageBytes;
           uint8_t* sB = sA + kTileABytes;
           if (kFused) {
-            const uint32_t tx = kPair ? 2 * fused_bytes : fused_bytes;
-            if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], tx);
+            // every slot of the stage is filled: the host picks kNA, kNB as the
+            // number of distinct maps the segments use
+            if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], (kPair ? 2 : 1) * C::kStageBytes);
             const int ka = kb * kBK + args.a_k_off, kbb = kb * kBK + args.b_k_off;
             if (kPair) {
               const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
-              if (use_a0) tma_load_2d_pair(sA, &tmA0, ka, a_row, leader_full);
-              if (use_a1) tma_load_2d_pair(sA + C::kOffA1, &tmA1, ka, a_row, leader_full);
-              if (use_b0) tma_load_2d_pair(sA + C::kOffB0, &tmB0, kbb, b_row, leader_full);
-              if (use_b1) tma_load_2d_pair(sA + C::kOffB1, &tmB1, kbb, b_row, leader_full);
+              tma_load_2d_pair(sA, map_a0, ka, a_row, leader_full);
+              if (kNA == 2) tma_load_2d_pair(sA + C::kOffA1, &tmA1, ka, a_row, leader_full);
+              tma_load_2d_pair(sA + C::kOffB0, map_b0, kbb, b_row, leader_full);
+              if (kNB == 2) tma_load_2d_pair(sA + C::kOffB1, &tmB1, kbb, b_row, leader_full);
             } else {
-              if (use_a0) tma_load_2d(sA, &tmA0, ka, a_row, &sm->full[stage]);
-              if (use_a1) tma_load_2d(sA + C::kOffA1, &tmA1, ka, a_row, &sm->full[stage]);
-              if (use_b0) tma_load_2d(sA + C::kOffB0, &tmB0, kbb, b_row, &sm->full[stage]);
-              if (use_b1) tma_load_2d(sA + C::kOffB1, &tmB1, kbb, b_row, &sm->full[stage]);
+              tma_load_2d(sA, map_a0, ka, a_row, &sm->full[stage]);
+              if (kNA == 2) tma_load_2d(sA + C::kOffA1, &tmA1, ka, a_row, &sm->full[stage]);
+              tma_load_2d(sA + C::kOffB0, map_b0, kbb, b_row, &sm->full[stage]);
+              if (kNB == 2) tma_load_2d(sA + C::kOffB1, &tmB1, kbb, b_row, &sm->full[stage]);
             }
           } else if (kPair) {
             if (rank == 0) mbar_arrive_expect_tx(&sm->full[stage], 2 * C::kStageBytes);
@@ -737,8 +744,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
           if (kFused) {
             for (int s = 0; s < args.num_seg; ++s) {
-              const uint64_t a_desc = umma_desc_sw128(a_addr + (args.seg_a[s] ? C::kOffA1 : 0));
-              const uint64_t b_desc = umma_desc_sw128(a_addr + (args.seg_b[s] ? C::kOffB1 : C::kOffB0));
+              const uint64_t a_desc = umma_desc_sw128(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0));
+              const uint64_t b_desc =
+                  umma_desc_sw128(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0));
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k) {
                 const uint32_t accum = (kb | s | k) != 0 ? 1u : 0u;
@@ -835,66 +843,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kKind, int kBN, bool kPair, bool kFused>
-cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
-  using C = Cfg<kBN, kPair, kFused>;
-  auto* fn = gemm_kernel<kKind, kBN, kPair, kFused>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  if (!kPair) {
-    const int grid = args.num_tiles < num_sms ? args.num_tiles : num_sms;
-    if (grid <= 0) return cudaSuccess;
-    fn<<<grid, kThreads, C::kSmemBytes, stream>>>(m.a0, m.a1, m.b0, m.b1, args);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // A persistent grid must not exceed the clusters that can be resident at once
-  // (a pair needs two SMs of one GPC): queried once per device.
-  // (One cache per kernel instance; host threads may launch concurrently.)
-  static std::atomic<int> resident[64];  // 0: not yet known
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  int max_pairs = (dev >= 0 && dev < 64) ? resident[dev].load(std::memory_order_relaxed) : 0;
-  if (max_pairs <= 0) {
-    e = cudaOccupancyMaxActiveClusters(&max_pairs, fn, &cfg);
-    if (e != cudaSuccess) return e;
-    if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
-    if (dev >= 0 && dev < 64) resident[dev].store(max_pairs, std::memory_order_relaxed);
-  }
-  int pairs = args.num_tiles < num_sms / 2 ? args.num_tiles : num_sms / 2;
-  if (pairs > max_pairs) pairs = max_pairs;
-  if (pairs <= 0) return cudaSuccess;
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  e = cudaLaunchKernelEx(&cfg, fn, m.a0, m.a1, m.b0, m.b1, args);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+// The fused instances that the library's GEMMs use (the others are not compiled):
+// pair 2+2 (the Gram step), pair 2+1 (direct form on pair tiles), 1-SM 2+1 (the
+// direct form's residual, update and final MSE).
+template <int kKind, int kBN, bool kPair, int kNA, int kNB>
+constexpr bool fused_instance() {
+  if (kNA == 0) return kNB == 0;
+  if (kPair && kNA == 2 && kNB == 2) return kKind == kEpiUpdate || kKind == kEpiUpdateFp;
+  if (kPair && kNA == 2 && kNB == 1) return kKind == kEpiStore || kKind == kEpiUpdate;
+  if (!kPair && kBN == 256 && kNA == 2 && kNB == 1)
+    return kKind == kEpiStore || kKind == kEpiUpdate || kKind == kEpiSumSq;
+  return false;
 }
 
-template <int kBN, bool kPair, bool kFused = false>
+template <int kKind, int kBN, bool kPair, int kNA, int kNB>
+cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
+  if constexpr (!fused_instance<kKind, kBN, kPair, kNA, kNB>()) {
+    return cudaErrorInvalidValue;
+  } else {
+    using C = Cfg<kBN, kPair, kNA, kNB>;
+    auto* fn = gemm_kernel<kKind, kBN, kPair, kNA, kNB>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (!kPair) {
+      const int grid = args.num_tiles < num_sms ? args.num_tiles : num_sms;
+      if (grid <= 0) return cudaSuccess;
+      fn<<<grid, kThreads, C::kSmemBytes, stream>>>(m.a0, m.a1, m.b0, m.b1, args);
+      return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // A persistent grid must not exceed the clusters that can be resident at once
+    // (a pair needs two SMs of one GPC): queried once per device.
+    // (One cache per kernel instance; host threads may launch concurrently.)
+    static std::atomic<int> resident[64];  // 0: not yet known
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int max_pairs = (dev >= 0 && dev < 64) ? resident[dev].load(std::memory_order_relaxed) : 0;
+    if (max_pairs <= 0) {
+      e = cudaOccupancyMaxActiveClusters(&max_pairs, fn, &cfg);
+      if (e != cudaSuccess) return e;
+      if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
+      if (dev >= 0 && dev < 64) resident[dev].store(max_pairs, std::memory_order_relaxed);
+    }
+    int pairs = args.num_tiles < num_sms / 2 ? args.num_tiles : num_sms / 2;
+    if (pairs > max_pairs) pairs = max_pairs;
+    if (pairs <= 0) return cudaSuccess;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, fn, m.a0, m.a1, m.b0, m.b1, args);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+}
+
+template <int kBN, bool kPair, int kNA = 0, int kNB = 0>
 cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
   switch (kind) {
     case kEpiStore:
-      return launch_kind<kEpiStore, kBN, kPair, kFused>(m, args, num_sms, stream);
+      return launch_kind<kEpiStore, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
     case kEpiSumSq:
-      return launch_kind<kEpiSumSq, kBN, kPair, kFused>(m, args, num_sms, stream);
+      return launch_kind<kEpiSumSq, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
     case kEpiUpdate:
-      return launch_kind<kEpiUpdate, kBN, kPair, kFused>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdate, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
     case kEpiDotD:
-      return launch_kind<kEpiDotD, kBN, kPair, kFused>(m, args, num_sms, stream);
+      return launch_kind<kEpiDotD, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
     case kEpiUpdateFp:
-      return launch_kind<kEpiUpdateFp, kBN, kPair, kFused>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdateFp, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -904,11 +929,29 @@ cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int
 cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmArgs& args, int num_sms,
                         cudaStream_t stream) {
   if (args.num_seg < 1 || args.num_seg > 3) return cudaErrorInvalidValue;
+  // Fused stages: as many A (B) tiles per stage as the segments use distinct maps.
+  int na = 0, nb = 0;
+  if (args.fused) {
+    bool a[2] = {false, false}, b[2] = {false, false};
+    for (int s = 0; s < args.num_seg; ++s) {
+      a[args.seg_a[s] ? 1 : 0] = true;
+      b[args.seg_b[s] ? 1 : 0] = true;
+    }
+    na = a[0] + a[1];
+    nb = b[0] + b[1];
+  }
   if (args.pair) {
     // Pair tiles: 256 rows x 256 columns; B maps with 128-row boxes; no symmetric mode.
     if (bn != 256 || args.symmetric) return cudaErrorInvalidValue;
-    if (args.fused) return launch_bn<256, true, true>(kind, maps, args, num_sms, stream);
-    return launch_bn<256, true>(kind, maps, args, num_sms, stream);
+    if (!args.fused) return launch_bn<256, true>(kind, maps, args, num_sms, stream);
+    if (na == 2 && nb == 2) return launch_bn<256, true, 2, 2>(kind, maps, args, num_sms, stream);
+    if (na == 2 && nb == 1) return launch_bn<256, true, 2, 1>(kind, maps, args, num_sms, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (args.fused) {
+    if (bn == 256 && na == 2 && nb == 1 && !args.symmetric)
+      return launch_bn<256, false, 2, 1>(kind, maps, args, num_sms, stream);
+    return cudaErrorInvalidValue;
   }
   if (bn == 256) return launch_bn<256, false>(kind, maps, args, num_sms, stream);
   if (bn == 128) return launch_bn<128, false>(kind, maps, args, num_sms, stream);
