@@ -161,8 +161,10 @@ ar_status ar_pack(const uint8_t* codes, int64_t rows, int64_t cols, int32_t bits
                   int32_t* packed, void* stream);
 
 /* Bytes of workspace ar_tune_layer needs for these sizes and params (0 if they are
- * invalid).  Dominated by a transposed copy of X (n_rows*in*2 bytes) and, for
- * AR_ALGO_GRAM, the Gram matrices (n_rows/batch_rows * in^2 * 4 bytes). */
+ * invalid).  X is read in place (never copied).  Dominated by the per-weight state
+ * (about 12 bytes per element of W, 20 in the Gram form), the direct form's residual
+ * (out*batch_rows*4 bytes) and, for AR_ALGO_GRAM, the Gram matrices
+ * (n_rows/batch_rows * in^2 * 4 bytes). */
 size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
                                const ar_tune_params* params);
 
@@ -211,7 +213,7 @@ typedef struct {
   int32_t kernel_launches;   /* every kernel this call launched */
   int32_t algo;              /* the ar_algo the call ran (DIRECT or GRAM) */
   float setup_ms;            /* device time before the first step (group statistics, and the
-                                first block's transpose and Gram matrix; later blocks are
+                                first block's Gram matrix; later blocks are
                                 prepared just before their first step) */
 } ar_tune_timing;
 

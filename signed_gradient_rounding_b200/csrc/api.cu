@@ -217,13 +217,12 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
 
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
-  size_t status, Xt, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
+  size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
       part0, part1, rowloss, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
-      // full-precision-target mode: this block's dX = X - X_target (pair, row-major
-      // and transposed), M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b
+      // full-precision-target mode: this block's dX = X - X_target (pair), M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b
       // (pair), their sum Cs (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the
       // partials of e_b, and W as a pair when it is fp32
-      dX_hi, dX_lo, dXt_hi, dXt_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo, total;
+      dX_hi, dX_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo, total;
 };
 
 Layout make_layout(const Plan& P) {
@@ -239,7 +238,6 @@ Layout make_layout(const Plan& P) {
   const bool gram = P.algo == AR_ALGO_GRAM;
   const int64_t nparts = std::max(std::max(P.nparts_res, P.nparts_upd), P.nparts_fin);
   L.status = take(256);
-  L.Xt = take(static_cast<size_t>(P.in) * P.n * 2);
   L.D_hi = take(elems * 2);
   L.D_lo = take(elems * 2);
   // The Gram form reads D_t and writes D_{t+1} in the same launch: two buffers.
@@ -273,8 +271,6 @@ Layout make_layout(const Plan& P) {
       const size_t blk = static_cast<size_t>(P.B) * P.in * 2;
       L.dX_hi = take(blk);
       L.dX_lo = take(blk);
-      L.dXt_hi = take(blk);
-      L.dXt_lo = take(blk);
       L.Mt_hi = take(h);
       L.Mt_lo = take(h);
       L.Cc_hi = take(elems * 2 * P.nb);
@@ -373,7 +369,6 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   int* status = reinterpret_cast<int*>(ws + L.status);
   // Second word of the status block: groups whose weights need the IEEE division.
   int* div_slow = status + 1;
-  uint16_t* Xt = reinterpret_cast<uint16_t*>(ws + L.Xt);
   __nv_bfloat16* D_hi = H(L.D_hi);
   __nv_bfloat16* D_lo = H(L.D_lo);
   __nv_bfloat16* Dh[2] = {D_hi, H(L.D_hi1)};
@@ -487,11 +482,12 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   GemmMaps gram_maps{};
   GemmArgs h;
   if (gram) {
-    AR_CUDA_TRY(make_tmap_bf16(&gram_maps.a0, Xt, in, n_rows, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&gram_maps.b0, Xt, in, n_rows, P.bn_gram));
-    gram_maps.a1 = gram_maps.a0;
-    gram_maps.b1 = gram_maps.b0;
+    // Both operands are X_b^T, read MN-major from the row-major activations through
+    // a map of block b alone (made per block), so a K tile that runs past the
+    // block's last row reads zeros rather than the next block.
     fill_grid(h, in, in, B, P.bn_gram, 1);
+    h.a_mn = 1;
+    h.b_mn = 1;
     h.symmetric = 1;  // H_b = X_b^T X_b: compute the tiles reaching the upper triangle
     h.num_tiles = 0;
     for (int nn = 0; nn < h.num_n_blk; ++nn)
@@ -512,11 +508,11 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   GemmArgs mg, cg, eg;
   if (fpt) {
     const int nseg_w = P.w_f32 ? 3 : 2;  // W pair x operand pair, or W x operand pair
-    mt_maps.a0 = gram_maps.a0;
-    mt_maps.a1 = gram_maps.a0;
-    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b0, H(L.dXt_hi), in, B, 256));
-    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b1, H(L.dXt_lo), in, B, 256));
+    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b0, H(L.dX_hi), B, in, 64));
+    AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b1, H(L.dX_lo), B, in, 64));
     fill_grid(mg, in, in, B, 256, 2);
+    mg.a_mn = 1;  // X_b^T and dX_b^T, read MN-major from the row-major blocks
+    mg.b_mn = 1;
     mg.seg_b[1] = 1;
     mg.timeout_ns = timeout_ns;
     mg.status = status;
@@ -554,13 +550,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   auto fp_target_block = [&](int64_t b) -> cudaError_t {
     const int64_t blk = B * in;
     cudaError_t e = launch_diff_pair(X + b * blk, X_target + b * blk, blk, H(L.dX_hi), H(L.dX_lo), st);
-    if (e == cudaSuccess)
-      e = launch_transpose_bf16(reinterpret_cast<const uint16_t*>(H(L.dX_hi)), B, in,
-                                reinterpret_cast<uint16_t*>(H(L.dXt_hi)), B, st);
-    if (e == cudaSuccess)
-      e = launch_transpose_bf16(reinterpret_cast<const uint16_t*>(H(L.dX_lo)), B, in,
-                                reinterpret_cast<uint16_t*>(H(L.dXt_lo)), B, st);
-    mg.a_k_off = static_cast<int>(b * B);
+    mt_maps.a0 = gram_maps.a0;  // block b of X (made by ensure_block)
+    mt_maps.a1 = gram_maps.a0;
     if (e == cudaSuccess) e = launch_gemm(kEpiStore, 256, mt_maps, mg, sms, st);
     cg.c_row_off = b * out;
     if (e == cudaSuccess) e = launch_gemm(kEpiStore, 256, c_maps, cg, sms, st);
@@ -569,13 +560,13 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
                             static_cast<int64_t>(elems), F(L.Cs), st);
     if (e == cudaSuccess) e = launch_gemm(kEpiSumSq, 256, e_maps, eg, sms, st);
     if (e == cudaSuccess) e = launch_row_sum(F(L.epart), eg.part_ld, out, F(L.e) + b * out, F(L.es), st);
-    launches += 8;
+    launches += 6;
     return e;
   };
 
-  // Each calibration block is transposed into its columns of Xt (and, in the Gram
-  // form, its Gram matrix is made) just before the first step that uses it.  With
-  // block_ready events, the block's copy to the device is awaited first.
+  // In the Gram form each calibration block's Gram matrix is made just before the
+  // first step that uses it.  With block_ready events, the block's copy to the
+  // device is awaited first (in both forms).
   std::vector<char> have_block(static_cast<size_t>(P.nb), 0), waited_block(static_cast<size_t>(P.nb), 0);
   auto wait_block = [&](int64_t b) -> cudaError_t {
     if (!block_ready || waited_block[b]) return cudaSuccess;
@@ -586,12 +577,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     if (have_block[b]) return cudaSuccess;
     have_block[b] = 1;
     cudaError_t e = wait_block(b);
-    if (e != cudaSuccess) return e;
-    e = launch_transpose_bf16(X + b * B * in, B, in, Xt + b * B, n_rows, st);
-    ++launches;
     if (e != cudaSuccess || !gram) return e;
-    h.a_k_off = static_cast<int>(b * B);
-    h.b_k_off = static_cast<int>(b * B);
+    e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);
+    if (e != cudaSuccess) return e;
+    gram_maps.a1 = gram_maps.b0 = gram_maps.b1 = gram_maps.a0;
     h.c_row_off = b * in;
     ++launches;
     e = launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
@@ -709,15 +698,13 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     GemmMaps mr{}, mu{};
     // Pair tiles (as for the Gram step): each CTA stages half of a tile's B rows.
     const uint32_t res_box = P.pair_direct ? P.bn_res / 2 : P.bn_res;
-    const uint32_t upd_box = P.pair_direct ? P.bn_upd / 2 : P.bn_upd;
     AR_CUDA_TRY(make_tmap_bf16(&mr.a0, D_hi, out, in, kBM));
     AR_CUDA_TRY(make_tmap_bf16(&mr.a1, D_lo, out, in, kBM));
     AR_CUDA_TRY(make_tmap_bf16(&mr.b0, X, n_rows, in, res_box));
     mr.b1 = mr.b0;
     AR_CUDA_TRY(make_tmap_bf16(&mu.a0, Rh, out, B, kBM));
     AR_CUDA_TRY(make_tmap_bf16(&mu.a1, Rl, out, B, kBM));
-    AR_CUDA_TRY(make_tmap_bf16(&mu.b0, Xt, in, n_rows, upd_box));
-    mu.b1 = mu.b0;
+    // mu.b0 (X_b^T, read MN-major from block b of X) is made per step.
 
     GemmArgs r;  // residual: R^T = D X_b^T, (D_hi + D_lo) X_b^T
     fill_grid(r, out, B, in, P.bn_res, nseg_d, P.pair_direct);
@@ -735,6 +722,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     fill_grid(u, out, in, B, P.bn_upd, nseg_d, P.pair_direct);  // update: G = (R_hi + R_lo)^T X_b
     u.raster_m = P.raster_upd;
     u.seg_a[1] = 1;
+    u.b_mn = 1;
     u.fused = r.fused;
     u.V_in = Vb[0];
     u.V_out = Vb[0];
@@ -753,7 +741,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
-      u.b_k_off = static_cast<int>(b0);
+      AR_CUDA_TRY(make_tmap_bf16(&mu.b0, X + b0 * in, B, in, 64));
+      mu.b1 = mu.b0;
       u.best_in = best_cur;
       u.best_out = best_next;
       u.rowloss = rowloss + static_cast<int64_t>(t) * out;

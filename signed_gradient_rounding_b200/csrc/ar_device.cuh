@@ -342,6 +342,10 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D, both
 // operands K-major, tile M x N.
+// Instruction-descriptor bits that mark A (bit 15) or B (bit 16) as MN-major.
+constexpr uint32_t kIdescAMn = 1u << 15;
+constexpr uint32_t kIdescBMn = 1u << 16;
+
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
   return (1u << 4)                          // D format: f32
          | (1u << 7)                        // A format: bf16
@@ -360,6 +364,23 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);   // start address
   d |= (uint64_t)1 << 16;                        // leading byte offset (unused for swizzled K-major)
   d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                        // layout: 128-byte swizzle
+  return d;
+}
+
+// Shared-memory matrix descriptor for an MN-major operand tile (the operand read
+// from a row-major [K, M or N] tensor without a transpose).  TMA writes it as
+// 64 x 64 boxes in the 128-byte swizzle pattern: each box holds 64 K rows of 64
+// consecutive M (or N) elements, 128 bytes a row, 8 KB a box.  In the canonical
+// MN-major layout the 64-element blocks along M or N are then 8 KB apart (leading
+// byte offset) and the eight-row K groups 1 KB apart (stride byte offset).
+// Advancing K by 16 rows adds 2 KB (128 units) to the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);   // start address
+  d |= (uint64_t)(8192 >> 4) << 16;              // leading byte offset: next 64 along M/N
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: next 8 K rows
   d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;                        // layout: 128-byte swizzle
   return d;

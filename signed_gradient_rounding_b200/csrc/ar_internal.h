@@ -41,10 +41,6 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t strea
 // round-to-nearest squared error, written to alpha and beta [out, in/g].
 cudaError_t launch_mse_init(const void* W, int w_bf16, int64_t out, int64_t in, int g, int bits, bool sym,
                             float* alpha, float* beta, cudaStream_t stream);
-// Xt[c * ld_t + r] = X[r * cols + c] for r < rows, c < cols (a row block of X
-// into the matching columns of a wider Xt when ld_t > rows).
-cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt, int64_t ld_t,
-                                  cudaStream_t stream);
 // loss_trace[t] = sum_j rowloss[t*out + j] / (batch_rows * out), t < iters (fixed order).
 cudaError_t launch_loss_trace(const float* rowloss, int64_t out, int iters, int64_t batch_rows,
                               float* loss_trace, cudaStream_t stream);
@@ -122,6 +118,10 @@ struct GemmArgs {
   int num_seg = 1;
   int seg_a[3] = {0, 0, 0};
   int seg_b[3] = {0, 0, 0};
+  // MN-major operands: the map covers a row-major [K, M] (A) or [K, N] (B) tensor
+  // (activations read without a transpose), built with 64-row boxes; loaded in
+  // 64 x 64 boxes.  Otherwise the map covers [M or N, K] (K-major).
+  int a_mn = 0, b_mn = 0;
   int a_k_off = 0;    // added to A's K coordinate
   int b_row_off = 0;  // added to B's row coordinate
   int b_k_off = 0;    // added to B's K coordinate

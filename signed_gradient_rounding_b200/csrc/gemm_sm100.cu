@@ -72,6 +72,33 @@ struct Cfg {
   static constexpr uint32_t kIdesc = umma_idesc_bf16(kPair ? 2 * kBM : kBM, kBN);
 };
 
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr, int mn) {
+  return mn ? umma_desc_sw128_mn(addr) : umma_desc_sw128(addr);
+}
+
+// One operand tile of `rows` M (or N) indices x kBK K values into shared memory.
+// K-major maps: one box.  MN-major maps: rows / 64 boxes of 64 x 64, 8 KB apart
+// (the canonical MN-major layout of umma_desc_sw128_mn).
+constexpr int kMnBoxBytes = 64 * kBK * 2;
+
+template <bool kPair>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, bool mn, int k, int row, int rows,
+                                          uint64_t* full, uint32_t leader_full) {
+  if (!mn) {
+    if (kPair)
+      tma_load_2d_pair(dst, map, k, row, leader_full);
+    else
+      tma_load_2d(dst, map, k, row, full);
+    return;
+  }
+  for (int j = 0; j < rows / 64; ++j) {
+    if (kPair)
+      tma_load_2d_pair(dst + j * kMnBoxBytes, map, row + 64 * j, k, leader_full);
+    else
+      tma_load_2d(dst + j * kMnBoxBytes, map, row + 64 * j, k, full);
+  }
+}
+
 struct Smem {
   uint64_t full[8];
   uint64_t empty[8];
@@ -647,6 +674,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // With one map of an operand staged, it is whichever one the segments use.
   const CUtensorMap* map_a0 = (kNA == 1 && use_a1) ? &tmA1 : &tmA0;
   const CUtensorMap* map_b0 = (kNB == 1 && use_b1) ? &tmB1 : &tmB0;
+  constexpr int kBRows = kPair ? kBN / 2 : kBN;  // B rows this CTA stages
+  // Operand majors: the instruction descriptor's bits, the shared-memory
+  // descriptor, and its start-address step per K16 (32 B K-major, 2 KB MN-major).
+  const uint32_t idesc = C::kIdesc | (args.a_mn ? kIdescAMn : 0u) | (args.b_mn ? kIdescBMn : 0u);
+  const uint32_t a_kstep = args.a_mn ? 128u : 2u, b_kstep = args.b_mn ? 128u : 2u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -676,27 +708,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // number of distinct maps the segments use
             if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], (kPair ? 2 : 1) * C::kStageBytes);
             const int ka = kb * kBK + args.a_k_off, kbb = kb * kBK + args.b_k_off;
-            if (kPair) {
-              const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
-              tma_load_2d_pair(sA, map_a0, ka, a_row, leader_full);
-              if (kNA == 2) tma_load_2d_pair(sA + C::kOffA1, &tmA1, ka, a_row, leader_full);
-              tma_load_2d_pair(sA + C::kOffB0, map_b0, kbb, b_row, leader_full);
-              if (kNB == 2) tma_load_2d_pair(sA + C::kOffB1, &tmB1, kbb, b_row, leader_full);
-            } else {
-              tma_load_2d(sA, map_a0, ka, a_row, &sm->full[stage]);
-              if (kNA == 2) tma_load_2d(sA + C::kOffA1, &tmA1, ka, a_row, &sm->full[stage]);
-              tma_load_2d(sA + C::kOffB0, map_b0, kbb, b_row, &sm->full[stage]);
-              if (kNB == 2) tma_load_2d(sA + C::kOffB1, &tmB1, kbb, b_row, &sm->full[stage]);
-            }
-          } else if (kPair) {
-            if (rank == 0) mbar_arrive_expect_tx(&sm->full[stage], 2 * C::kStageBytes);
-            const uint32_t leader_full = mapa_shared(smem_u32(&sm->full[stage]), 0);
-            tma_load_2d_pair(sA, mA, kk * kBK + args.a_k_off, a_row, leader_full);
-            tma_load_2d_pair(sB, mB, kk * kBK + args.b_k_off, b_row, leader_full);
+            const uint32_t leader_full = kPair ? mapa_shared(smem_u32(&sm->full[stage]), 0) : 0u;
+            uint64_t* full = &sm->full[stage];
+            load_tile<kPair>(sA, map_a0, args.a_mn, ka, a_row, kBM, full, leader_full);
+            if (kNA == 2) load_tile<kPair>(sA + C::kOffA1, &tmA1, args.a_mn, ka, a_row, kBM, full, leader_full);
+            load_tile<kPair>(sA + C::kOffB0, map_b0, args.b_mn, kbb, b_row, kBRows, full, leader_full);
+            if (kNB == 2) load_tile<kPair>(sA + C::kOffB1, &tmB1, args.b_mn, kbb, b_row, kBRows, full, leader_full);
           } else {
-            mbar_arrive_expect_tx(&sm->full[stage], C::kStageBytes);
-            tma_load_2d(sA, mA, kk * kBK + args.a_k_off, a_row, &sm->full[stage]);
-            tma_load_2d(sB, mB, kk * kBK + args.b_k_off, b_row, &sm->full[stage]);
+            if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], (kPair ? 2 : 1) * C::kStageBytes);
+            const uint32_t leader_full = kPair ? mapa_shared(smem_u32(&sm->full[stage]), 0) : 0u;
+            load_tile<kPair>(sA, mA, args.a_mn, kk * kBK + args.a_k_off, a_row, kBM, &sm->full[stage], leader_full);
+            load_tile<kPair>(sB, mB, args.b_mn, kk * kBK + args.b_k_off, b_row, kBRows, &sm->full[stage], leader_full);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -744,27 +766,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
           if (kFused) {
             for (int s = 0; s < args.num_seg; ++s) {
-              const uint64_t a_desc = umma_desc_sw128(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0));
+              const uint64_t a_desc =
+                  operand_desc(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0), args.a_mn);
               const uint64_t b_desc =
-                  umma_desc_sw128(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0));
+                  operand_desc(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0), args.b_mn);
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k) {
                 const uint32_t accum = (kb | s | k) != 0 ? 1u : 0u;
                 if (kPair)
-                  umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, accum);
+                  umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
                 else
-                  umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, accum);
+                  umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
               }
             }
           } else {
-            const uint64_t a_desc = umma_desc_sw128(a_addr);
-            const uint64_t b_desc = umma_desc_sw128(a_addr + kTileABytes);
+            const uint64_t a_desc = operand_desc(a_addr, args.a_mn);
+            const uint64_t b_desc = operand_desc(a_addr + kTileABytes, args.b_mn);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
+              const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
               if (kPair)
-                umma_bf16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+                umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
               else
-                umma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+                umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
             }
           }
           if (kPair)

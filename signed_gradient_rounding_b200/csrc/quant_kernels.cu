@@ -1,7 +1,6 @@
 // Elementwise and reduction kernels of libar: group min-max statistics, scale and
 // zero-point, offset fake-quantisation (RTN when V = 0, alpha = beta = 1), int32
-// bit packing, the bf16 transpose of the calibration activations, and the
-// fixed-order loss reductions.
+// bit packing, and the fixed-order loss reductions.
 #include <math.h>
 
 #include "ar_device.cuh"
@@ -105,54 +104,6 @@ __global__ void fill_f32_kernel(float* p, int64_t n, float v) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p[i] = v;
-}
-
-// Xt[c * ld_t + r] = X[r * cols + c].  64 x 64 tiles through shared memory; 256
-// threads.  Full tiles move 16-byte vectors both ways (rows, cols and ld_t
-// multiples of 8 keep them aligned); the tile's ragged edges fall back to single
-// elements.  In shared memory, the 16-byte chunk j of tile row r sits at chunk
-// j ^ ((r >> 3) & 7): the eight rows 8m + k that one read instruction gathers
-// (one per m, for a fixed column) then fall in eight different banks.
-__device__ __forceinline__ int tile_chunk(int r, int chunk) { return chunk ^ ((r >> 3) & 7); }
-
-__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, int64_t rows, int64_t cols,
-                                      uint16_t* __restrict__ Xt, int64_t ld_t) {
-  __shared__ __align__(16) uint16_t tile[64][72];
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 64;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 64;
-  const bool full = (r0 + 64 <= rows) && (c0 + 64 <= cols) && (rows % 8 == 0) && (cols % 8 == 0) && (ld_t % 8 == 0);
-  if (full) {
-    for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 rows x 8 vectors
-      const int r = v >> 3, ch = v & 7;
-      *reinterpret_cast<uint4*>(&tile[r][tile_chunk(r, ch) * 8]) =
-          *reinterpret_cast<const uint4*>(X + (r0 + r) * cols + c0 + ch * 8);
-    }
-    __syncthreads();
-    for (int v = threadIdx.x; v < 64 * 8; v += blockDim.x) {  // 64 output rows (cols of X) x 8 vectors
-      const int c = v >> 3, r8 = (v & 7) * 8;
-      uint16_t e[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) e[k] = tile[r8 + k][tile_chunk(r8 + k, c >> 3) * 8 + (c & 7)];
-      uint4 o;
-      o.x = e[0] | (uint32_t(e[1]) << 16);
-      o.y = e[2] | (uint32_t(e[3]) << 16);
-      o.z = e[4] | (uint32_t(e[5]) << 16);
-      o.w = e[6] | (uint32_t(e[7]) << 16);
-      *reinterpret_cast<uint4*>(Xt + (c0 + c) * ld_t + r0 + r8) = o;
-    }
-    return;
-  }
-  const int tx = threadIdx.x & 63;
-  const int ty = threadIdx.x >> 6;  // 0..3
-  for (int i = ty; i < 64; i += 4) {
-    const int64_t r = r0 + i, c = c0 + tx;
-    if (r < rows && c < cols) tile[i][tx] = X[r * cols + c];
-  }
-  __syncthreads();
-  for (int i = ty; i < 64; i += 4) {
-    const int64_t c = c0 + i, r = r0 + tx;
-    if (r < rows && c < cols) Xt[c * ld_t + r] = tile[tx][i];
-  }
 }
 
 // AR_INIT_MSE: one warp per group, one lane per grid ratio (two rounds for the 51
@@ -461,14 +412,6 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t strea
   int64_t blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, n, value);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_bf16(const uint16_t* X, int64_t rows, int64_t cols, uint16_t* Xt, int64_t ld_t,
-                                  cudaStream_t stream) {
-  if (rows <= 0 || cols <= 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>((cols + 63) / 64), static_cast<unsigned>((rows + 63) / 64));
-  transpose_bf16_kernel<<<grid, 256, 0, stream>>>(X, rows, cols, Xt, ld_t);
   return cudaGetLastError();
 }
 

@@ -116,8 +116,9 @@ def _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed):
 
 @pytest.mark.parametrize("case", [(256, 256, 512, 512, 40, 4, 64, "f32"),
                                   (256, 512, 4096, 1024, 30, 3, 128, "bf16"),
-                                  (200, 384, 2048, 512, 24, 2, 128, "bf16")],
-                         ids=["tiny-f32-full-batch", "multiblock-bf16", "ragged-W2"])
+                                  (200, 384, 2048, 512, 24, 2, 128, "bf16"),
+                                  (200, 256, 1560, 520, 20, 3, 128, "bf16")],
+                         ids=["tiny-f32-full-batch", "multiblock-bf16", "ragged-W2", "batch-520"])
 def test_fp_target_parity(ar, case):
     out, inn, n, B, iters, bits, g, wdt = case
     res, ref, *_ = _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed=21)

@@ -200,6 +200,18 @@ def test_ragged_multiblock(ar, bits, g, sym, wdt, algo):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
+def test_batch_rows_not_a_multiple_of_the_k_tile(ar, algo):
+    """batch_rows = 520 (a multiple of 8, not of the 64-row K tile): a block's last
+    K tile must read zeros past the block's rows, not the next block's."""
+    out, inn, n, B = 200, 256, 1560, 520
+    W = make_weight(out, inn, 0.02, "bf16", seed=8)
+    X = make_activations(n, inn, "llm", seed=8)
+    res, ref = _tune_both(ar, W, X, "bf16", 4, 128, False, 24, 0.005, 0.005, B, 4, algo=algo)
+    _assert_tuned_close(res, ref, "batch 520")
+    np.testing.assert_allclose(_np(res.loss_trace).astype(np.float64), ref.loss_trace, rtol=0.05)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
 @pytest.mark.parametrize("size", [(256, 512, 512), (256, 4096, 16384)])
 def test_one_step_signs(ar, algo, size):
     """One step from V = 0, clip factors frozen: V1 = -lr*sign(G)*m wherever the
