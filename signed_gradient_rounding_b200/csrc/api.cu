@@ -163,6 +163,8 @@ struct Plan {
   // Direct form (residual, update, final MSE): X_b (or X_b^T) staged once per K
   // block for both halves of the pair operand instead of once per half.
   bool fused_direct = true;
+  // Full-precision-target products (M_b^T, C_b, e_b) on pair tiles with fused stages.
+  bool pair_fpt = true;
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
@@ -510,7 +512,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     const int nseg_w = P.w_f32 ? 3 : 2;  // W pair x operand pair, or W x operand pair
     AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b0, H(L.dX_hi), B, in, 64));
     AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b1, H(L.dX_lo), B, in, 64));
-    fill_grid(mg, in, in, B, 256, 2);
+    fill_grid(mg, in, in, B, 256, 2, P.pair_fpt);
+    mg.fused = P.pair_fpt ? 1 : 0;
     mg.a_mn = 1;  // X_b^T and dX_b^T, read MN-major from the row-major blocks
     mg.b_mn = 1;
     mg.seg_b[1] = 1;
@@ -526,12 +529,14 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       else
         m->a1 = m->a0;
     }
-    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b0, H(L.Mt_hi), in, in, 256));
-    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b1, H(L.Mt_lo), in, in, 256));
-    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b0, H(L.dX_hi), B, in, 256));
-    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b1, H(L.dX_lo), B, in, 256));
+    const uint32_t fpt_box = P.pair_fpt ? 128 : 256;  // pair tiles: half the B rows per CTA
+    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b0, H(L.Mt_hi), in, in, fpt_box));
+    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b1, H(L.Mt_lo), in, in, fpt_box));
+    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b0, H(L.dX_hi), B, in, fpt_box));
+    AR_CUDA_TRY(make_tmap_bf16(&e_maps.b1, H(L.dX_lo), B, in, fpt_box));
     for (GemmArgs* g : {&cg, &eg}) {
-      fill_grid(*g, out, g == &cg ? in : B, in, 256, nseg_w);
+      fill_grid(*g, out, g == &cg ? in : B, in, 256, nseg_w, P.pair_fpt);
+      g->fused = P.pair_fpt ? 1 : 0;
       if (P.w_f32) {  // W_hi X_hi + W_lo X_hi + W_hi X_lo
         g->seg_a[1] = 1;
         g->seg_b[2] = 1;

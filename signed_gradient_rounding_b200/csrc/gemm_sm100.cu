@@ -868,12 +868,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // The fused instances that the library's GEMMs use (the others are not compiled):
-// pair 2+2 (the Gram step), pair 2+1 (direct form on pair tiles), 1-SM 2+1 (the
-// direct form's residual, update and final MSE).
+// pair 2+2 (the Gram step; the full-precision-target products with an fp32 W),
+// pair 1+2 (those products with a bf16 W), pair 2+1 (direct form on pair tiles),
+// 1-SM 2+1 (the direct form's residual, update and final MSE).
 template <int kKind, int kBN, bool kPair, int kNA, int kNB>
 constexpr bool fused_instance() {
   if (kNA == 0) return kNB == 0;
-  if (kPair && kNA == 2 && kNB == 2) return kKind == kEpiUpdate || kKind == kEpiUpdateFp;
+  if (kPair && kNA == 2 && kNB == 2)
+    return kKind == kEpiUpdate || kKind == kEpiUpdateFp || kKind == kEpiStore || kKind == kEpiSumSq;
+  if (kPair && kNA == 1 && kNB == 2) return kKind == kEpiStore || kKind == kEpiSumSq;
   if (kPair && kNA == 2 && kNB == 1) return kKind == kEpiStore || kKind == kEpiUpdate;
   if (!kPair && kBN == 256 && kNA == 2 && kNB == 1)
     return kKind == kEpiStore || kKind == kEpiUpdate || kKind == kEpiSumSq;
@@ -970,6 +973,7 @@ cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmAr
     if (!args.fused) return launch_bn<256, true>(kind, maps, args, num_sms, stream);
     if (na == 2 && nb == 2) return launch_bn<256, true, 2, 2>(kind, maps, args, num_sms, stream);
     if (na == 2 && nb == 1) return launch_bn<256, true, 2, 1>(kind, maps, args, num_sms, stream);
+    if (na == 1 && nb == 2) return launch_bn<256, true, 1, 2>(kind, maps, args, num_sms, stream);
     return cudaErrorInvalidValue;
   }
   if (args.fused) {
