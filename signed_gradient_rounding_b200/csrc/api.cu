@@ -165,6 +165,8 @@ struct Plan {
   bool fused_direct = true;
   // Full-precision-target products (M_b^T, C_b, e_b) on pair tiles with fused stages.
   bool pair_fpt = true;
+  // Gram matrices (symmetric, upper tiles only) on pair tiles.
+  bool pair_gram = true;
   // Pair tiles in groups of 8 m-blocks (2048 rows): measured ~1.5% faster than
   // one sweep over all rows on the 4096 x 4096 layer.
   int raster_upd = 8;
@@ -487,13 +489,14 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     // Both operands are X_b^T, read MN-major from the row-major activations through
     // a map of block b alone (made per block), so a K tile that runs past the
     // block's last row reads zeros rather than the next block.
-    fill_grid(h, in, in, B, P.bn_gram, 1);
+    fill_grid(h, in, in, B, P.bn_gram, 1, P.pair_gram);
     h.a_mn = 1;
     h.b_mn = 1;
     h.symmetric = 1;  // H_b = X_b^T X_b: compute the tiles reaching the upper triangle
     h.num_tiles = 0;
+    const int64_t m_height = P.pair_gram ? 2 * kBM : kBM;
     for (int nn = 0; nn < h.num_n_blk; ++nn)
-      h.num_tiles += static_cast<int>(std::min<int64_t>(h.num_m_blk, cdiv((nn + 1) * int64_t(P.bn_gram), kBM)));
+      h.num_tiles += static_cast<int>(std::min<int64_t>(h.num_m_blk, cdiv((nn + 1) * int64_t(P.bn_gram), m_height)));
     h.timeout_ns = timeout_ns;
     h.status = status;
     h.C_hi = H(L.H_hi);

@@ -225,8 +225,9 @@ __device__ __forceinline__ void store_pair8(const float* x, __nv_bfloat16* hi_ds
 }
 
 // Tile t of the launch -> (m_blk, n_blk).  Plain: m fastest.  Symmetric: only the
-// tiles with some column >= row, n-major, ceil((n + 1) * BN / BM) of them per n.
-template <int kBN>
+// tiles with some column >= row, n-major, ceil((n + 1) * BN / BM) of them per n
+// (BM: the m-block height, 256 rows for pair tiles).
+template <int kBN, bool kPair>
 __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, int& n_blk) {
   if (!a.symmetric) {
     if (a.raster_m <= 0 || a.raster_m >= a.num_m_blk) {
@@ -243,7 +244,8 @@ __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, i
     return;
   }
   for (n_blk = 0; n_blk < a.num_n_blk; ++n_blk) {
-    const int cnt = min(a.num_m_blk, ((n_blk + 1) * kBN + kBM - 1) / kBM);
+    constexpr int kMH = kPair ? 2 * kBM : kBM;
+    const int cnt = min(a.num_m_blk, ((n_blk + 1) * kBN + kMH - 1) / kMH);
     if (t < cnt) break;
     t -= cnt;
   }
@@ -689,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
         int m_blk, n_blk;
-        tile_pos<kBN>(args, tile, m_blk, n_blk);
+        tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
         const int a_row = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM;
         const int b_row = n_blk * kBN + args.b_row_off + (kPair ? static_cast<int>(rank) * (kBN / 2) : 0);
         for (int kb = 0; kb < k_blocks; ++kb) {
@@ -827,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = unit0; tile < args.num_tiles; tile += unit_stride) {
       int m_blk, n_blk;
-      tile_pos<kBN>(args, tile, m_blk, n_blk);
+      tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
       const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
       if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN>(args, j, n0, half);
@@ -968,8 +970,8 @@ cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmAr
     nb = b[0] + b[1];
   }
   if (args.pair) {
-    // Pair tiles: 256 rows x 256 columns; B maps with 128-row boxes; no symmetric mode.
-    if (bn != 256 || args.symmetric) return cudaErrorInvalidValue;
+    // Pair tiles: 256 rows x 256 columns; K-major B maps with 128-row boxes.
+    if (bn != 256) return cudaErrorInvalidValue;
     if (!args.fused) return launch_bn<256, true>(kind, maps, args, num_sms, stream);
     if (na == 2 && nb == 2) return launch_bn<256, true, 2, 2>(kind, maps, args, num_sms, stream);
     if (na == 2 && nb == 1) return launch_bn<256, true, 2, 1>(kind, maps, args, num_sms, stream);
