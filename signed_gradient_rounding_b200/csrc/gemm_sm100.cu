@@ -72,7 +72,7 @@ struct Cfg {
   static constexpr uint32_t kIdesc = umma_idesc_bf16(kPair ? 2 * kBM : kBM, kBN);
 };
 
-__device__ __forceinline__ uint64_t operand_desc(uint32_t addr, int mn) {
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr, bool mn) {
   return mn ? umma_desc_sw128_mn(addr) : umma_desc_sw128(addr);
 }
 
@@ -609,7 +609,8 @@ __device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, in
 // full barrier; the leader's MMA thread alone issues M = 256 MMAs and its commits
 // arrive on both CTAs' barriers; each CTA's epilogue reads its own 128 accumulator
 // rows and releases the accumulator with one arrive per warp on the leader.
-template <int kKind, int kBN, bool kPair, int kNA, int kNB>
+// kMaj: bit 0 set when A is MN-major, bit 1 when B is (GemmArgs::a_mn, b_mn).
+template <int kKind, int kBN, bool kPair, int kNA, int kNB, int kMaj>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
@@ -679,8 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBRows = kPair ? kBN / 2 : kBN;  // B rows this CTA stages
   // Operand majors: the instruction descriptor's bits, the shared-memory
   // descriptor, and its start-address step per K16 (32 B K-major, 2 KB MN-major).
-  const uint32_t idesc = C::kIdesc | (args.a_mn ? kIdescAMn : 0u) | (args.b_mn ? kIdescBMn : 0u);
-  const uint32_t a_kstep = args.a_mn ? 128u : 2u, b_kstep = args.b_mn ? 128u : 2u;
+  constexpr bool kAMn = (kMaj & 1) != 0, kBMn = (kMaj & 2) != 0;
+  constexpr uint32_t idesc = C::kIdesc | (kAMn ? kIdescAMn : 0u) | (kBMn ? kIdescBMn : 0u);
+  constexpr uint32_t a_kstep = kAMn ? 128u : 2u, b_kstep = kBMn ? 128u : 2u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -712,15 +714,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ka = kb * kBK + args.a_k_off, kbb = kb * kBK + args.b_k_off;
             const uint32_t leader_full = kPair ? mapa_shared(smem_u32(&sm->full[stage]), 0) : 0u;
             uint64_t* full = &sm->full[stage];
-            load_tile<kPair>(sA, map_a0, args.a_mn, ka, a_row, kBM, full, leader_full);
-            if (kNA == 2) load_tile<kPair>(sA + C::kOffA1, &tmA1, args.a_mn, ka, a_row, kBM, full, leader_full);
-            load_tile<kPair>(sA + C::kOffB0, map_b0, args.b_mn, kbb, b_row, kBRows, full, leader_full);
-            if (kNB == 2) load_tile<kPair>(sA + C::kOffB1, &tmB1, args.b_mn, kbb, b_row, kBRows, full, leader_full);
+            load_tile<kPair>(sA, map_a0, kAMn, ka, a_row, kBM, full, leader_full);
+            if (kNA == 2) load_tile<kPair>(sA + C::kOffA1, &tmA1, kAMn, ka, a_row, kBM, full, leader_full);
+            load_tile<kPair>(sA + C::kOffB0, map_b0, kBMn, kbb, b_row, kBRows, full, leader_full);
+            if (kNB == 2) load_tile<kPair>(sA + C::kOffB1, &tmB1, kBMn, kbb, b_row, kBRows, full, leader_full);
           } else {
             if (!kPair || rank == 0) mbar_arrive_expect_tx(&sm->full[stage], (kPair ? 2 : 1) * C::kStageBytes);
             const uint32_t leader_full = kPair ? mapa_shared(smem_u32(&sm->full[stage]), 0) : 0u;
-            load_tile<kPair>(sA, mA, args.a_mn, kk * kBK + args.a_k_off, a_row, kBM, &sm->full[stage], leader_full);
-            load_tile<kPair>(sB, mB, args.b_mn, kk * kBK + args.b_k_off, b_row, kBRows, &sm->full[stage], leader_full);
+            load_tile<kPair>(sA, mA, kAMn, kk * kBK + args.a_k_off, a_row, kBM, &sm->full[stage], leader_full);
+            load_tile<kPair>(sB, mB, kBMn, kk * kBK + args.b_k_off, b_row, kBRows, &sm->full[stage], leader_full);
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -769,9 +771,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kFused) {
             for (int s = 0; s < args.num_seg; ++s) {
               const uint64_t a_desc =
-                  operand_desc(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0), args.a_mn);
+                  operand_desc(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0), kAMn);
               const uint64_t b_desc =
-                  operand_desc(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0), args.b_mn);
+                  operand_desc(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0), kBMn);
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k) {
                 const uint32_t accum = (kb | s | k) != 0 ? 1u : 0u;
@@ -782,8 +784,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           } else {
-            const uint64_t a_desc = operand_desc(a_addr, args.a_mn);
-            const uint64_t b_desc = operand_desc(a_addr + kTileABytes, args.b_mn);
+            const uint64_t a_desc = operand_desc(a_addr, kAMn);
+            const uint64_t b_desc = operand_desc(a_addr + kTileABytes, kBMn);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
               const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
@@ -874,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // pair 1+2 (those products with a bf16 W), pair 2+1 (direct form on pair tiles),
 // 1-SM 2+1 (the direct form's residual, update and final MSE).
 template <int kKind, int kBN, bool kPair, int kNA, int kNB>
-constexpr bool fused_instance() {
+constexpr bool stage_instance() {
   if (kNA == 0) return kNB == 0;
   if (kPair && kNA == 2 && kNB == 2)
     return kKind == kEpiUpdate || kKind == kEpiUpdateFp || kKind == kEpiStore || kKind == kEpiSumSq;
@@ -885,13 +887,25 @@ constexpr bool fused_instance() {
   return false;
 }
 
-template <int kKind, int kBN, bool kPair, int kNA, int kNB>
+// MN-major operands (the activations read in place): both for the Gram matrices
+// and the full-precision-target M_b (kEpiStore), B for the direct update.
+template <int kKind, int kBN, bool kPair, int kNA, int kNB, int kMaj>
+constexpr bool kernel_instance() {
+  if (!stage_instance<kKind, kBN, kPair, kNA, kNB>()) return false;
+  if (kMaj == 0) return true;
+  if (kBN != 256) return false;
+  if (kMaj == 3) return kKind == kEpiStore && ((kNA == 0 && kNB == 0) || (kNA == 1 && kNB == 2));
+  if (kMaj == 2) return kKind == kEpiUpdate && ((kNA == 0 && kNB == 0) || (kNA == 2 && kNB == 1));
+  return false;
+}
+
+template <int kKind, int kBN, bool kPair, int kNA, int kNB, int kMaj>
 cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
-  if constexpr (!fused_instance<kKind, kBN, kPair, kNA, kNB>()) {
+  if constexpr (!kernel_instance<kKind, kBN, kPair, kNA, kNB, kMaj>()) {
     return cudaErrorInvalidValue;
   } else {
     using C = Cfg<kBN, kPair, kNA, kNB>;
-    auto* fn = gemm_kernel<kKind, kBN, kPair, kNA, kNB>;
+    auto* fn = gemm_kernel<kKind, kBN, kPair, kNA, kNB, kMaj>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     if (!kPair) {
@@ -936,19 +950,34 @@ cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cu
   }
 }
 
-template <int kBN, bool kPair, int kNA = 0, int kNB = 0>
+template <int kBN, bool kPair, int kNA, int kNB, int kMaj>
 cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
   switch (kind) {
     case kEpiStore:
-      return launch_kind<kEpiStore, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
+      return launch_kind<kEpiStore, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiSumSq:
-      return launch_kind<kEpiSumSq, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
+      return launch_kind<kEpiSumSq, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiUpdate:
-      return launch_kind<kEpiUpdate, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdate, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiDotD:
-      return launch_kind<kEpiDotD, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
+      return launch_kind<kEpiDotD, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiUpdateFp:
-      return launch_kind<kEpiUpdateFp, kBN, kPair, kNA, kNB>(m, args, num_sms, stream);
+      return launch_kind<kEpiUpdateFp, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// The operand majors of a launch as the kernel's kMaj.
+template <int kBN, bool kPair, int kNA = 0, int kNB = 0>
+cudaError_t launch_major(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int num_sms, cudaStream_t stream) {
+  const int maj = (args.a_mn ? 1 : 0) | (args.b_mn ? 2 : 0);
+  switch (maj) {
+    case 0:
+      return launch_bn<kBN, kPair, kNA, kNB, 0>(kind, m, args, num_sms, stream);
+    case 2:
+      return launch_bn<kBN, kPair, kNA, kNB, 2>(kind, m, args, num_sms, stream);
+    case 3:
+      return launch_bn<kBN, kPair, kNA, kNB, 3>(kind, m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -972,19 +1001,19 @@ cudaError_t launch_gemm(EpiKind kind, int bn, const GemmMaps& maps, const GemmAr
   if (args.pair) {
     // Pair tiles: 256 rows x 256 columns; K-major B maps with 128-row boxes.
     if (bn != 256) return cudaErrorInvalidValue;
-    if (!args.fused) return launch_bn<256, true>(kind, maps, args, num_sms, stream);
-    if (na == 2 && nb == 2) return launch_bn<256, true, 2, 2>(kind, maps, args, num_sms, stream);
-    if (na == 2 && nb == 1) return launch_bn<256, true, 2, 1>(kind, maps, args, num_sms, stream);
-    if (na == 1 && nb == 2) return launch_bn<256, true, 1, 2>(kind, maps, args, num_sms, stream);
+    if (!args.fused) return launch_major<256, true>(kind, maps, args, num_sms, stream);
+    if (na == 2 && nb == 2) return launch_major<256, true, 2, 2>(kind, maps, args, num_sms, stream);
+    if (na == 2 && nb == 1) return launch_major<256, true, 2, 1>(kind, maps, args, num_sms, stream);
+    if (na == 1 && nb == 2) return launch_major<256, true, 1, 2>(kind, maps, args, num_sms, stream);
     return cudaErrorInvalidValue;
   }
   if (args.fused) {
     if (bn == 256 && na == 2 && nb == 1 && !args.symmetric)
-      return launch_bn<256, false, 2, 1>(kind, maps, args, num_sms, stream);
+      return launch_major<256, false, 2, 1>(kind, maps, args, num_sms, stream);
     return cudaErrorInvalidValue;
   }
-  if (bn == 256) return launch_bn<256, false>(kind, maps, args, num_sms, stream);
-  if (bn == 128) return launch_bn<128, false>(kind, maps, args, num_sms, stream);
+  if (bn == 256) return launch_major<256, false>(kind, maps, args, num_sms, stream);
+  if (bn == 128) return launch_major<128, false>(kind, maps, args, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 
