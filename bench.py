@@ -103,17 +103,54 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def _recorded_traffic(key: str):
-    """DRAM bytes per launch from profiles/traffic.txt, if the GEMM source is unchanged."""
+GEMM_SOURCES = ("gemm_sm100.cu", "ar_device.cuh", "ar_internal.h")
+
+
+def _strip_comments(text: str) -> str:
+    """C++ source without // and /* */ comments, trailing blanks or empty lines."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                                   # string or character literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
+def gemm_code_fingerprint() -> str:
+    """First 16 hex digits of the sha256 of the GEMM kernel's code (its source and the
+    device headers it includes, comments and blank lines removed): the ncu figures in
+    profiles/traffic.txt hold while this is unchanged."""
     import hashlib
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "signed_gradient_rounding_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _strip_comments(f.read()).encode() + b"\0")
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic(key: str):
+    """DRAM bytes per launch from profiles/traffic.txt, if the GEMM code is unchanged."""
     try:
         rec = {}
         for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
             parts = line.split()
             if len(parts) == 2 and not line.startswith("#"):
                 rec[parts[0]] = parts[1]
-        src = open(os.path.join(ROOT, "signed_gradient_rounding_b200", "csrc", "gemm_sm100.cu"), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != rec.get("gemm_source_sha256_16"):
+        if gemm_code_fingerprint() != rec.get("gemm_code_sha256_16"):
             return None
         return int(rec[key]) if key in rec else None
     except (OSError, ValueError):

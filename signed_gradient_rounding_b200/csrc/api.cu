@@ -151,11 +151,11 @@ struct Plan {
   int64_t out = 0, in = 0, n = 0, B = 0, g = 0, G = 0, nb = 0, iters = 0;
   int bn_res = 256;   // direct: residual GEMM (N = B)
   int bn_upd = 256;   // update GEMM (N = in)
-  int bn_gram = 128;  // Gram matrices (N = in)
+  int bn_gram = 256;  // Gram matrices (N = in)
   int bn_fin = 256;   // final-MSE GEMM
   int64_t nparts_res = 0, nparts_upd = 0, nparts_fin = 0;
   // Gram-form update GEMM on 2-SM pair tiles (256 x 256, tcgen05 cta_group::2):
-  // each SM stages 32 KB per K block instead of 48 KB, so six stages fit.
+  // each SM stages half of the tile's B rows.
   bool pair_upd = true;
   // ... with the three pair products fused per K block (Cfg::kFused): the hi tiles
   // of D and H are staged once per K block rather than twice.

@@ -2,19 +2,23 @@
 //
 //   C[M, N] = sum over segments s of  A_s[M, K] * B_s[N, K]^T
 //
-// A and B are bf16, K-major, loaded by TMA; C is fp32 in tensor memory.  A
-// "segment" is one pass over K with its own pair of operand maps, so an operand
-// kept as an exact bf16 pair x = hi + lo (hi = bf16(x), lo = bf16(x - hi), about
-// 16 significant bits) is multiplied as extra segments of the same accumulation:
+// A and B are bf16, loaded by TMA in the 128-byte swizzle, K-major ([rows, K]) or
+// MN-major ([K, rows]: activations read in place); C is fp32 in tensor memory.  A
+// "segment" is one product with its own pair of operand maps, so an operand kept
+// as an exact bf16 pair x = hi + lo (hi = bf16(x), lo = bf16(x - hi), about 16
+// significant bits) is multiplied as extra segments of the same accumulation:
 // (hi_a + lo_a)(hi_b + lo_b) ~ hi_a hi_b + lo_a hi_b + hi_a lo_b.
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage, 128-byte
-//               swizzle, completion counted on the stage's mbarrier.
-//   warp 1      MMA issuer: four tcgen05.mma (M=128, N=BN, K=16) per stage into one
-//               of two BN-column fp32 accumulators in tensor memory;
-//               tcgen05.commit frees the stage and, after the last K block, hands
-//               the accumulator to the epilogue.
+// Roles (320 threads, one CTA per SM; or clusters of two CTAs on 256-row pair
+// tiles with tcgen05 cta_group::2):
+//   warp 0      TMA producer.  Per stage either one 64-wide K block of one
+//               segment's A and B tiles, or (fused stages) one K block of every
+//               map the segments use, each staged once; completion counted on the
+//               stage's mbarrier.
+//   warp 1      MMA issuer: tcgen05.mma (M=128 or 256, N=BN, K=16), four per
+//               segment in the stage, into one of two BN-column fp32 accumulators
+//               in tensor memory; tcgen05.commit frees the stage and, after the
+//               last K block, hands the accumulator to the epilogue.
 //   warps 2..9  epilogue: two warps per 32-lane slice of tensor memory (a warp may
 //               only read the slice warp % 4), one per column half of the tile.
 //               Each thread owns one accumulator row and walks its half's columns

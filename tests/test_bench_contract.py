@@ -40,3 +40,15 @@ def test_rejects_short_warmup():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], cwd=ROOT,
                          capture_output=True, text=True, timeout=120)
     assert out.returncode != 0
+
+
+def test_gemm_fingerprint_ignores_comments_only():
+    """The ncu traffic figures stay valid across comment edits, not code edits."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) {  // first\n  /* block */ return x + 1;\n}\n\nconst char* s = \"a//b\";\n"
+    b = "// header\nint f(int x) {\n  return x + 1;   // other words\n}\nconst char* s = \"a//b\";\n"
+    assert bench._strip_comments(a) == bench._strip_comments(b)
+    assert bench._strip_comments(a) != bench._strip_comments(a.replace("x + 1", "x + 2"))
+    assert "a//b" in bench._strip_comments(a)
+    assert len(bench.gemm_code_fingerprint()) == 16
