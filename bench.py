@@ -107,7 +107,7 @@ GEMM_SOURCES = ("gemm_sm100.cu", "ar_device.cuh", "ar_internal.h")
 
 
 def _strip_comments(text: str) -> str:
-    """C++ source without // and /* */ comments, trailing blanks or empty lines."""
+    """C++ source without // and /* */ comments, indentation, trailing blanks or empty lines."""
     out, i, n = [], 0, len(text)
     while i < n:
         c = text[i]
@@ -126,7 +126,7 @@ def _strip_comments(text: str) -> str:
         else:
             out.append(c)
             i += 1
-    lines = (line.rstrip() for line in "".join(out).splitlines())
+    lines = (line.strip() for line in "".join(out).splitlines())
     return "\n".join(line for line in lines if line)
 
 
