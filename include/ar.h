@@ -191,9 +191,12 @@ size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
  *   loss_trace  [iters] fp32 out (batch loss of each step), may be NULL.
  *   final_mse   1 double out: mean((X W'^T - X W^T)^2) over all n_rows rows with
  *               the applied W', may be NULL (skips one pass over X).
- * Supported shapes: in a multiple of 32; batch_rows a multiple of 8; group_size a
- * multiple of 32 that divides 256 or equals in with in <= 256 (else
- * AR_EUNSUPPORTED).  out == 0 or in == 0 is a no-op.
+ * Supported shapes: in a multiple of 32; batch_rows a multiple of 8; group size
+ * (group_size, or in for -1) a multiple of 32 (else AR_EUNSUPPORTED).  Groups that
+ * divide 256 (or a whole row of at most 256) are updated inside the step kernel;
+ * any other (a whole row of a wider layer, or sizes such as 96 or 384) through
+ * per-segment partials and one small kernel per step.  out == 0 or in == 0 is a
+ * no-op.
  * AR_EINVAL: bad bits/group_size, iters < 0, lr < 0, batch_rows <= 0 or not a
  * divisor of n_rows, NULL or misaligned pointers.  AR_ENOMEM: ws_bytes too small.
  * Calls sharing a workspace or state must not overlap on the device. */

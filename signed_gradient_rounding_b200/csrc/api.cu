@@ -118,12 +118,17 @@ ar_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AR_OK : AR_ECUDA;
     if (e_ != cudaSuccess) return AR_ECUDA; \
   } while (0)
 
-// The update epilogue needs whole groups inside one thread's tile columns.
+// Groups are whole multiples of 32 columns (the update epilogue walks 16-column
+// chunks that never straddle a group).
 bool tune_shape_supported(int64_t in, int64_t g, int64_t B) {
   if (in % 32 != 0 || B % 8 != 0) return false;
-  if (g % 32 != 0) return false;
-  return (256 % g == 0) || (g == in && in <= 256);
+  return g % 32 == 0;
 }
+
+// Groups that fit inside one epilogue thread's columns are updated in the step's
+// epilogue; wider or unaligned ones (whole-row groups of a wide layer, or sizes
+// that do not divide 256) through per-segment partials and launch_group_finish.
+bool wide_groups(int64_t in, int64_t g) { return !((256 % g == 0) || (g == in && in <= 256)); }
 
 ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune_params* p) {
   if (!p || out < 0 || in < 0 || n_rows < 0) return AR_EINVAL;
@@ -174,6 +179,9 @@ struct Plan {
   // whether W is fp32 (then held as a bf16 pair for its contractions).
   bool fp_target = false;
   bool w_f32 = false;
+  // Wide groups (see wide_groups) and the segment slots of their partials.
+  bool wide = false;
+  int gslots = 0;
   // Direct-form residual and update GEMMs on pair tiles: measured 3% faster on the
   // 4096-wide layer, 3-10% slower (more energy per step at the power cap) on the
   // 29568-wide one, which is where the automatic choice picks the direct form.
@@ -212,6 +220,8 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   P.bn_upd = 256;
   P.bn_gram = 256;
   P.bn_fin = 256;
+  P.wide = wide_groups(in, P.g);
+  P.gslots = P.wide ? static_cast<int>(cdiv(P.g, kSegCols) + 1) : 0;
   // Row partial sums: kEpiHalves per n-tile (one per epilogue column half).
   P.nparts_res = cdiv(P.B, P.bn_res) * kEpiHalves;
   P.nparts_upd = cdiv(in, P.bn_upd) * kEpiHalves;
@@ -222,7 +232,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
   size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
-      part0, part1, rowloss, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
+      part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
       // full-precision-target mode: this block's dX = X - X_target (pair), M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b
       // (pair), their sum Cs (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the
       // partials of e_b, and W as a pair when it is fp32
@@ -263,6 +273,7 @@ Layout make_layout(const Plan& P) {
   L.part0 = take(static_cast<size_t>(P.out) * nparts * 4);
   L.part1 = gram ? take(static_cast<size_t>(P.out) * nparts * 4) : L.part0;
   L.rowloss = take(static_cast<size_t>(P.out) * std::max<int64_t>(P.iters, 1) * 4);
+  L.gpart = P.wide ? take(groups * P.gslots * 2 * 4) : 0;
   if (gram) {
     const size_t h = static_cast<size_t>(P.in) * P.in * 2;
     L.H_hi = take(h * P.nb);
@@ -618,6 +629,44 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.keep_best = p->keep_best != 0;
   u.lr = p->lr;
   u.mlr = mlr;
+  u.gpart = P.wide ? F(L.gpart) : nullptr;
+  u.gslots = P.gslots;
+  // Wide groups: the group updates and the next D after each step launch.
+  auto finish_groups = [&]() -> cudaError_t {
+    if (!P.wide) return cudaSuccess;
+    GroupFinishArgs f;
+    f.W = u.W;
+    f.w_bf16 = u.w_bf16;
+    f.out = out;
+    f.in = in;
+    f.g = u.g;
+    f.G = u.G;
+    f.gslots = u.gslots;
+    f.gpart = u.gpart;
+    f.V = u.V_out;
+    f.wmin = u.wmin;
+    f.wmax = u.wmax;
+    f.alpha_in = u.alpha_in;
+    f.beta_in = u.beta_in;
+    f.alpha_out = u.alpha_out;
+    f.beta_out = u.beta_out;
+    f.alpha_best = u.alpha_best;
+    f.beta_best = u.beta_best;
+    f.judged = u.part_in != nullptr;
+    f.keep_best = u.keep_best;
+    f.snap_prev = u.snap_prev;
+    f.best_in = u.best_in;
+    f.best_out = u.best_out;
+    f.D_hi = u.D_hi;
+    f.D_lo = u.D_lo;
+    f.div_slow = u.div_slow;
+    f.bits = u.bits;
+    f.sym = u.sym;
+    f.mlr = u.mlr;
+    ++launches;
+    return launch_group_finish(f, st);
+  };
+  const EpiKind upd_kind = fpt ? (P.wide ? kEpiUpdateFpWide : kEpiUpdateFp) : (P.wide ? kEpiUpdateWide : kEpiUpdate);
 
   float* best_cur = best_loss;
   float* best_next = best_alt;
@@ -670,7 +719,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
         u.e_row = F(L.e) + sched[t] * out;
       }
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
-      AR_CUDA_TRY(launch_gemm(fpt ? kEpiUpdateFp : kEpiUpdate, P.bn_upd, m[cur], u, sms, st));
+      AR_CUDA_TRY(launch_gemm(upd_kind, P.bn_upd, m[cur], u, sms, st));
+      AR_CUDA_TRY(finish_groups());
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
       ++launches;
       if (t > 0) std::swap(best_cur, best_next);
@@ -754,7 +804,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       u.best_in = best_cur;
       u.best_out = best_next;
       u.rowloss = rowloss + static_cast<int64_t>(t) * out;
-      AR_CUDA_TRY(launch_gemm(kEpiUpdate, P.bn_upd, mu, u, sms, st));
+      AR_CUDA_TRY(launch_gemm(upd_kind, P.bn_upd, mu, u, sms, st));
+      AR_CUDA_TRY(finish_groups());
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 2], st));
       launches += 2;
       std::swap(best_cur, best_next);

@@ -90,6 +90,41 @@ __device__ __forceinline__ ElemQuant quant_elem(float w, float v, GroupScale g, 
 
 __device__ __forceinline__ float sgnf(float x) { return (x > 0.0f) ? 1.0f : ((x < 0.0f) ? -1.0f : 0.0f); }
 
+// Straight-through derivatives of a group's scale and zero-point with respect to
+// its clip factors ("[llm-compressor] AutoRound ...": rint treated as identity,
+// a clamp passing the gradient inside its range).
+struct GroupDeriv {
+  float ds_a, ds_b;    // ds/d alpha, ds/d beta
+  float dzp_a, dzp_b;  // dzp/d alpha, dzp/d beta (0 when zp is clamped, and when symmetric)
+};
+
+__device__ __forceinline__ GroupDeriv group_deriv(float wmn, float wmx, float be, const GroupScale& gs, float Q,
+                                                  bool sym) {
+  GroupDeriv d;
+  d.dzp_a = 0.f;
+  d.dzp_b = 0.f;
+  if (sym) {
+    d.ds_a = __fdiv_rn(__fmul_rn(2.0f, fmaxf(-wmn, wmx)), Q);
+    d.ds_b = 0.f;
+  } else {
+    d.ds_a = __fdiv_rn(wmx, Q);
+    d.ds_b = __fdiv_rn(-wmn, Q);
+    const float z0 = __fdiv_rn(-__fmul_rn(be, wmn), gs.s);
+    const float rz = rintf(z0);
+    if (rz >= 0.f && rz <= Q) {
+      d.dzp_a = -z0 * d.ds_a / gs.s;
+      d.dzp_b = -wmn / gs.s - z0 * d.ds_b / gs.s;
+    }
+  }
+  return d;
+}
+
+// A clip factor after one sign step of size mlr against its gradient, clamped to
+// [0.5, 1].
+__device__ __forceinline__ float clip_step(float c, float mlr, float grad) {
+  return fminf(fmaxf(__fsub_rn(c, __fmul_rn(mlr, sgnf(grad))), 0.5f), 1.0f);
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }

@@ -104,8 +104,18 @@ enum EpiKind : int {
   kEpiSumSq = 1,   // per-(row, n-tile) sums of C^2
   kEpiUpdate = 2,  // C = G: the SignSGD step (sign updates, keep-best, next D, Gram-form loss)
   kEpiDotD = 3,    // per-(row, n-tile) sums of D * C
-  kEpiUpdateFp = 4 // kEpiUpdate with the full-precision-target terms (Cc_hi, e_row)
+  kEpiUpdateFp = 4, // kEpiUpdate with the full-precision-target terms (Cc_hi, e_row)
+  // Groups wider than a thread's columns (group_size not dividing 256): the
+  // per-element part of the step (G, loss, V, V snapshot) and per-(row, group,
+  // 128-column segment) partials of d alpha, d beta into GemmArgs::gpart; the
+  // group's update and the next D follow in launch_group_finish.
+  kEpiUpdateWide = 5,
+  kEpiUpdateFpWide = 6
 };
+
+// Columns per thread in the update epilogue (one column half of a 256-wide tile):
+// the segment width of the wide-group partials.
+constexpr int kSegCols = 128;
 
 // Operand maps: segment s reads A from a{seg_a[s]} and B from b{seg_b[s]}.
 struct GemmMaps {
@@ -196,7 +206,44 @@ struct GemmArgs {
   float inv_batch = 1.0f;
   int g = 0, G = 0, bits = 4, sym = 0, keep_best = 1;
   float lr = 0.f, mlr = 0.f;
+  // kEpiUpdate*Wide: [M * G, gslots, 2] partial (d alpha, d beta); slot k of group
+  // gg holds the sum over the group's columns in 128-column segment
+  // floor(gg * g / 128) + k.
+  float* gpart = nullptr;
+  int gslots = 0;
 };
+
+// After a wide-group step launch: per (row, group), d alpha and d beta as the sum
+// of the group's segment partials in slot order, the clip-factor sign updates
+// (with the keep-best snapshot of alpha and beta), and the next step's
+// D = W' - W from the updated state as a bf16 pair.  One warp per group.
+struct GroupFinishArgs {
+  const void* W = nullptr;
+  int w_bf16 = 0;
+  int64_t out = 0, in = 0;
+  int g = 0, G = 0, gslots = 0;
+  const float* gpart = nullptr;
+  const float* V = nullptr;  // the state after the step (the launch's V_out)
+  const float* wmin = nullptr;
+  const float* wmax = nullptr;
+  const float* alpha_in = nullptr;
+  const float* beta_in = nullptr;
+  float* alpha_out = nullptr;
+  float* beta_out = nullptr;
+  float* alpha_best = nullptr;
+  float* beta_best = nullptr;
+  // keep-best: the launch judged a loss (part_in set) and row j improved iff
+  // best_out[j] < best_in[j]; snap_prev as in GemmArgs
+  int judged = 0, keep_best = 1, snap_prev = 0;
+  const float* best_in = nullptr;
+  const float* best_out = nullptr;
+  __nv_bfloat16* D_hi = nullptr;
+  __nv_bfloat16* D_lo = nullptr;
+  const int* div_slow = nullptr;
+  int bits = 4, sym = 0;
+  float mlr = 0.f;
+};
+cudaError_t launch_group_finish(const GroupFinishArgs& a, cudaStream_t stream);
 
 // Tile sizes: M and K tiles fixed, N tile 128 or 256 per launch.
 constexpr int kBM = 128;

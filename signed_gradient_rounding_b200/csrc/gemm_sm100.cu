@@ -392,20 +392,14 @@ __device__ __forceinline__ void load_upd_chunk(const GemmArgs& a, int64_t e0, in
   if (a.diag_in) load_f32x16(a.diag_in + col, dg);
 }
 
-// kFp: the full-precision-target terms (GemmArgs::Cc_hi set) are compiled in.
-template <int kBN, bool kFp>
-__device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
-  const bool row_ok = j < a.M;
-  const float Q = qmaxf(a.bits);
-  const bool sym = a.sym != 0;
-  const int64_t row_base = static_cast<int64_t>(j) * a.N;
-
-  // Keep-best: the row's batch loss (sum of the per-n-tile partials in a fixed
-  // order, so every n-tile of the row reaches the same decision) against the best
-  // so far.  Direct form: the loss of this step (computed by the residual GEMM),
-  // snapshot of the state read now.  Gram form: the loss of the previous step
-  // (computed by the previous launch), snapshot of the previous state, which still
-  // sits in the output buffers until this epilogue overwrites it.
+// Keep-best: the row's batch loss (sum of the per-n-tile partials in a fixed
+// order, so every n-tile of the row reaches the same decision) against the best
+// so far; the row's lead thread records the new best and the loss.  Direct form:
+// the loss of this step (computed by the residual GEMM), snapshot of the state read
+// now.  Gram form: the loss of the previous step (computed by the previous
+// launch), snapshot of the previous state, which still sits in the output buffers
+// until this epilogue overwrites it.
+__device__ __forceinline__ bool row_better(const GemmArgs& a, int j, bool row_ok, int n_blk, int half) {
   bool better = false;
   if (row_ok && a.part_in) {
     // Sum in index order; eight loads are in flight at a time.
@@ -427,6 +421,51 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
     }
     if (n_blk == 0 && half == 0) a.rowloss[j] = L;
   }
+  return better;
+}
+
+// One element of the step: G (the accumulator, plus the exact Gram-diagonal term
+// and, with a full-precision target, this block's C), the element's share of the
+// row loss, its new V, and its terms of the group's d alpha and d beta.
+template <bool kFp>
+__device__ __forceinline__ float sign_step_elem(const GemmArgs& a, float w, float v, float acc, float dg, float cv,
+                                                const GroupScale& gs, const GroupDeriv& gd, float Q, bool fast,
+                                                float& loss_acc, float& dal, float& dbe) {
+  const ElemQuant e = quant_elem(w, v, gs, Q, fast);
+  const float d = __fsub_rn(e.wq, w);
+  float G = a.diag_in ? fmaf(d, dg, acc) : acc;
+  if (kFp) {
+    // row loss: d H d^T + 2 d C^T (+ e_row once per row); gradient D H + C
+    G = __fadd_rn(G, cv);
+    loss_acc = fmaf(d, __fadd_rn(G, cv), loss_acc);
+  } else {
+    loss_acc = fmaf(d, G, loss_acc);
+  }
+  const float sg = e.m ? sgnf(G) : 0.0f;
+  const float vn = fminf(fmaxf(__fsub_rn(v, __fmul_rn(a.lr, sg)), -0.5f), 0.5f);
+  float dwa, dwb;
+  if (e.m) {
+    const float ru = e.r - e.u;
+    dwa = gd.ds_a * ru;
+    dwb = gd.ds_b * ru;
+  } else {
+    const float qz = e.q - gs.zp;
+    dwa = gd.ds_a * qz - gs.s * gd.dzp_a;
+    dwb = gd.ds_b * qz - gs.s * gd.dzp_b;
+  }
+  dal = fmaf(G, dwa, dal);
+  dbe = fmaf(G, dwb, dbe);
+  return vn;
+}
+
+// kFp: the full-precision-target terms (GemmArgs::Cc_hi set) are compiled in.
+template <int kBN, bool kFp>
+__device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
+  const bool row_ok = j < a.M;
+  const float Q = qmaxf(a.bits);
+  const bool sym = a.sym != 0;
+  const int64_t row_base = static_cast<int64_t>(j) * a.N;
+  const bool better = row_better(a, j, row_ok, n_blk, half);
   const bool snap_now = better && !a.snap_prev;
   const bool snap_old = better && a.snap_prev;
   const bool fast = a.div_slow && *a.div_slow == 0;
@@ -449,21 +488,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       be = a.beta_in[gidx];
     }
     const GroupScale gs = group_scale(wmn, wmx, al, be, a.bits, sym);
-    // Straight-through derivatives of s and zp with respect to alpha and beta.
-    float ds_a, ds_b, dzp_a = 0.f, dzp_b = 0.f;
-    if (sym) {
-      ds_a = __fdiv_rn(__fmul_rn(2.0f, fmaxf(-wmn, wmx)), Q);
-      ds_b = 0.f;
-    } else {
-      ds_a = __fdiv_rn(wmx, Q);
-      ds_b = __fdiv_rn(-wmn, Q);
-      const float z0 = __fdiv_rn(-__fmul_rn(be, wmn), gs.s);
-      const float rz = rintf(z0);
-      if (rz >= 0.f && rz <= Q) {
-        dzp_a = -z0 * ds_a / gs.s;
-        dzp_b = -wmn / gs.s - z0 * ds_b / gs.s;
-      }
-    }
+    const GroupDeriv gd = group_deriv(wmn, wmx, be, gs, Q, sym);
 
     // Pass 1: sign updates of V, and the group's d alpha, d beta.
     float dal = 0.f, dbe = 0.f;
@@ -509,39 +534,16 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       }
       float vn[kUC];
 #pragma unroll
-      for (int i = 0; i < kUC; ++i) {
-        const ElemQuant e = quant_elem(w[i], v[i], gs, Q, fast);
-        const float d = __fsub_rn(e.wq, w[i]);
-        float G = a.diag_in ? fmaf(d, dg[i], __uint_as_float(r[i])) : __uint_as_float(r[i]);
-        if (kFp) {
-          // row loss: d H d^T + 2 d C^T (+ e_row once per row, below); gradient D H + C
-          G = __fadd_rn(G, cv[i]);
-          loss_acc = fmaf(d, __fadd_rn(G, cv[i]), loss_acc);
-        } else {
-          loss_acc = fmaf(d, G, loss_acc);
-        }
-        const float sg = e.m ? sgnf(G) : 0.0f;
-        vn[i] = fminf(fmaxf(__fsub_rn(v[i], __fmul_rn(a.lr, sg)), -0.5f), 0.5f);
-        float dwa, dwb;
-        if (e.m) {
-          const float ru = e.r - e.u;
-          dwa = ds_a * ru;
-          dwb = ds_b * ru;
-        } else {
-          const float qz = e.q - gs.zp;
-          dwa = ds_a * qz - gs.s * dzp_a;
-          dwb = ds_b * qz - gs.s * dzp_b;
-        }
-        dal = fmaf(G, dwa, dal);
-        dbe = fmaf(G, dwb, dbe);
-      }
+      for (int i = 0; i < kUC; ++i)
+        vn[i] = sign_step_elem<kFp>(a, w[i], v[i], __uint_as_float(r[i]), dg[i], kFp ? cv[i] : 0.0f, gs, gd, Q, fast,
+                                    loss_acc, dal, dbe);
       store_f32x16(a.V_out + e0, vn);
       if (snap_now) store_f32x16(a.V_best + e0, v);
     }
     if (!row_ok) continue;
 
-    const float al_n = fminf(fmaxf(__fsub_rn(al, __fmul_rn(a.mlr, sgnf(dal))), 0.5f), 1.0f);
-    const float be_n = sym ? be : fminf(fmaxf(__fsub_rn(be, __fmul_rn(a.mlr, sgnf(dbe))), 0.5f), 1.0f);
+    const float al_n = clip_step(al, a.mlr, dal);
+    const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
     if (snap_now) {
       a.alpha_best[gidx] = al;
       a.beta_best[gidx] = be;
@@ -582,15 +584,109 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
   if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = loss_acc;
 }
 
+// kEpiUpdate*Wide: groups wider than a thread's columns, or not aligned to them.
+// This thread walks its column half (kSegCols columns, one 128-column segment of
+// the row) in chunks of kUC; a chunk lies in one group (g is a multiple of 32).
+// Per element it does what epi_update's first pass does (G, the row loss, the new
+// V, the V snapshot); the group's d alpha and d beta over this segment go to
+// GemmArgs::gpart, and launch_group_finish completes the group.
+template <int kBN, bool kFp>
+__device__ __forceinline__ void epi_update_wide(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk,
+                                                int half) {
+  static_assert(kBN / kEpiHalves == kSegCols, "one segment per thread");
+  const bool row_ok = j < a.M;
+  const float Q = qmaxf(a.bits);
+  const bool sym = a.sym != 0;
+  const int64_t row_base = static_cast<int64_t>(j) * a.N;
+  const bool better = row_better(a, j, row_ok, n_blk, half);
+  const bool snap_now = better && !a.snap_prev;
+  const bool snap_old = better && a.snap_prev;
+  const bool fast = a.div_slow && *a.div_slow == 0;
+  const int c_begin = n0 + half * kSegCols;
+  const int c_end = min(a.N, c_begin + kSegCols);
+  const int seg = c_begin / kSegCols;
+
+  float loss_acc = 0.0f;
+  int cur = -1;  // group of the running sums
+  float dal = 0.f, dbe = 0.f;
+  GroupScale gs{1.f, 0.f, 1.f};
+  GroupDeriv gd{0.f, 0.f, 0.f, 0.f};
+  auto flush = [&]() {
+    const int k = seg - static_cast<int>((static_cast<int64_t>(cur) * a.g) / kSegCols);
+    float* p = a.gpart + ((static_cast<int64_t>(j) * a.G + cur) * a.gslots + k) * 2;
+    p[0] = dal;
+    p[1] = dbe;
+  };
+#pragma unroll 1
+  for (int col = c_begin; col < c_end; col += kUC) {  // warp-uniform bounds
+    const int gg = col / a.g;
+    if (gg != cur) {
+      if (cur >= 0 && row_ok) flush();
+      cur = gg;
+      dal = 0.f;
+      dbe = 0.f;
+      float wmn = 0.f, wmx = 0.f, al = 1.f, be = 1.f;
+      if (row_ok) {
+        const int64_t gidx = static_cast<int64_t>(j) * a.G + gg;
+        wmn = a.wmin[gidx];
+        wmx = a.wmax[gidx];
+        al = a.alpha_in[gidx];
+        be = a.beta_in[gidx];
+      }
+      gs = group_scale(wmn, wmx, al, be, a.bits, sym);
+      gd = group_deriv(wmn, wmx, be, gs, Q, sym);
+    }
+    const int64_t e0 = row_base + col;
+    float w[kUC], v[kUC], dg[kUC], cv[kUC];
+    if (row_ok) {
+      load_upd_chunk(a, e0, col, w, v, dg);
+      if (kFp) {
+        float clo[kUC];
+        load_w16(a.Cc_hi, 1, e0, cv);
+        load_w16(a.Cc_lo, 1, e0, clo);
+#pragma unroll
+        for (int i = 0; i < kUC; ++i) cv[i] = __fadd_rn(cv[i], clo[i]);
+      }
+    }
+    uint32_t r[kUC];
+    __syncwarp();
+    tmem_ld_16cols(t_row + (col - n0), r);
+    tmem_ld_wait();
+    if (!row_ok) continue;  // nothing warp-collective follows in this iteration
+    if (snap_old) {
+      float vo[kUC];
+      load_f32x16(a.V_out + e0, vo);
+      store_f32x16(a.V_best + e0, vo);
+    }
+    float vn[kUC];
+#pragma unroll
+    for (int i = 0; i < kUC; ++i)
+      vn[i] = sign_step_elem<kFp>(a, w[i], v[i], __uint_as_float(r[i]), dg[i], kFp ? cv[i] : 0.0f, gs, gd, Q, fast,
+                                  loss_acc, dal, dbe);
+    store_f32x16(a.V_out + e0, vn);
+    if (snap_now) store_f32x16(a.V_best + e0, v);
+  }
+  if (cur >= 0 && row_ok) flush();
+  if (kFp && row_ok && a.e_row && n_blk == 0 && half == 0) loss_acc += a.e_row[j];
+  if (row_ok && a.part_out) a.part_out[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = loss_acc;
+}
+
 // Before waiting for a tile's accumulator, ask L2 for the W and V row segments the
 // update epilogue of that tile will read, so the wait covers their memory latency.
-template <int kBN>
+// (kWide: the thread's column half, which epi_update_wide walks.)
+template <int kBN, bool kWide>
 __device__ __forceinline__ void epi_update_prefetch(const GemmArgs& a, int j, int n0, int half) {
   if (j >= a.M) return;
-  int gl_begin, gl_end;
-  epi_group_range<kBN>(a, half, gl_begin, gl_end);
-  const int c0 = n0 + gl_begin * a.g;
-  const int c1 = min(a.N, n0 + gl_end * a.g);
+  int c0, c1;
+  if (kWide) {
+    c0 = n0 + half * (kBN / kEpiHalves);
+    c1 = min(a.N, c0 + kBN / kEpiHalves);
+  } else {
+    int gl_begin, gl_end;
+    epi_group_range<kBN>(a, half, gl_begin, gl_end);
+    c0 = n0 + gl_begin * a.g;
+    c1 = min(a.N, n0 + gl_end * a.g);
+  }
   if (c0 >= c1) return;
   const int64_t e0 = static_cast<int64_t>(j) * a.N + c0;
   const uint32_t cols = static_cast<uint32_t>(c1 - c0);  // a multiple of 8
@@ -838,16 +934,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
       const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
-      if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN>(args, j, n0, half);
+      if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN, false>(args, j, n0, half);
+      if (kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide) epi_update_prefetch<kBN, true>(args, j, n0, half);
       // No early exit on another role's abort: every epilogue warp of the CTA takes
       // the same decision here (the phase completes for all of them, or for none).
       if (!mbar_wait<kPair>(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns, false)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
-      if (kKind == kEpiUpdate)
+      if constexpr (kKind == kEpiUpdate)
         epi_update<kBN, false>(args, t_row, j, n0, n_blk, half);
-      else if (kKind == kEpiUpdateFp)
+      else if constexpr (kKind == kEpiUpdateFp)
         epi_update<kBN, true>(args, t_row, j, n0, n_blk, half);
+      else if constexpr (kKind == kEpiUpdateWide)
+        epi_update_wide<kBN, false>(args, t_row, j, n0, n_blk, half);
+      else if constexpr (kKind == kEpiUpdateFpWide)
+        epi_update_wide<kBN, true>(args, t_row, j, n0, n_blk, half);
       else
         epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk, half);
       tc_fence_before();
@@ -895,6 +996,13 @@ constexpr bool stage_instance() {
 // and the full-precision-target M_b (kEpiStore), B for the direct update.
 template <int kKind, int kBN, bool kPair, int kNA, int kNB, int kMaj>
 constexpr bool kernel_instance() {
+  // Wide-group steps: the Gram step on pair tiles (pair or single operands, with or
+  // without a full-precision target) and the direct update on 1-SM tiles.
+  if (kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide) {
+    if (kBN != 256 || !((kNA == 2 && kNB == 2) || (kNA == 0 && kNB == 0) || (kNA == 2 && kNB == 1))) return false;
+    if (kPair) return kMaj == 0 && kNB != 1;
+    return kKind == kEpiUpdateWide && kMaj == 2 && kNB != 2;
+  }
   if (!stage_instance<kKind, kBN, kPair, kNA, kNB>()) return false;
   if (kMaj == 0) return true;
   if (kBN != 256) return false;
@@ -967,6 +1075,10 @@ cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int
       return launch_kind<kEpiDotD, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiUpdateFp:
       return launch_kind<kEpiUpdateFp, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
+    case kEpiUpdateWide:
+      return launch_kind<kEpiUpdateWide, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
+    case kEpiUpdateFpWide:
+      return launch_kind<kEpiUpdateFpWide, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -289,6 +289,55 @@ __global__ void finalize_best_kernel(FinalizeBestArgs a) {
   }
 }
 
+// One warp per (row, group) of a wide-group step: the group's d alpha and d beta
+// from its segment partials (summed in slot order), the clip-factor sign updates
+// with their keep-best snapshot (as the update epilogue takes it for narrow
+// groups), then the next step's D = W' - W over the group's columns.
+__global__ void group_finish_kernel(GroupFinishArgs a) {
+  const int64_t grp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (grp >= a.out * a.G) return;  // warp-uniform
+  const int64_t j = grp / a.G;
+  const int64_t gg = grp - j * a.G;
+  const int first = static_cast<int>((gg * a.g) / kSegCols);
+  const int last = static_cast<int>(((gg + 1) * a.g - 1) / kSegCols);
+  float dal = 0.f, dbe = 0.f;
+  const float* p = a.gpart + grp * a.gslots * 2;
+  for (int k = 0; k <= last - first; ++k) {
+    dal += p[2 * k];
+    dbe += p[2 * k + 1];
+  }
+  const bool sym = a.sym != 0;
+  const float al = a.alpha_in[grp], be = a.beta_in[grp];
+  const float al_n = clip_step(al, a.mlr, dal);
+  const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
+  const bool better = a.judged && a.keep_best && a.best_out[j] < a.best_in[j];
+  __syncwarp();  // every lane has read alpha_in, beta_in (they may alias the outputs)
+  if (lane == 0) {
+    if (better && !a.snap_prev) {
+      a.alpha_best[grp] = al;
+      a.beta_best[grp] = be;
+    }
+    if (better && a.snap_prev) {
+      a.alpha_best[grp] = a.alpha_out[grp];
+      a.beta_best[grp] = a.beta_out[grp];
+    }
+    a.alpha_out[grp] = al_n;
+    a.beta_out[grp] = be_n;
+  }
+  const GroupScale gn = group_scale(a.wmin[grp], a.wmax[grp], al_n, be_n, a.bits, sym);
+  const float Q = qmaxf(a.bits);
+  const bool fast = a.div_slow && *a.div_slow == 0;
+  const int64_t base = j * a.in + gg * a.g;
+  for (int k = lane; k < a.g; k += 32) {
+    const float w = load_w(a.W, a.w_bf16, base + k);
+    const float d = __fsub_rn(quant_elem(w, a.V[base + k], gn, Q, fast).wq, w);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(d);
+    a.D_hi[base + k] = hi;
+    if (a.D_lo) a.D_lo[base + k] = __float2bfloat16_rn(__fsub_rn(d, __bfloat162float(hi)));
+  }
+}
+
 __global__ void gram_sum_kernel(const __nv_bfloat16* __restrict__ H_hi, const __nv_bfloat16* __restrict__ H_lo,
                                 int nb, int64_t count, __nv_bfloat16* __restrict__ Hs_hi,
                                 __nv_bfloat16* __restrict__ Hs_lo) {
@@ -412,6 +461,14 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float value, cudaStream_t strea
   int64_t blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, n, value);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_finish(const GroupFinishArgs& a, cudaStream_t stream) {
+  const int64_t warps = a.out * a.G;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  group_finish_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
