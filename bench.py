@@ -20,6 +20,7 @@ bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import ctypes
 import json
 import os
@@ -39,6 +40,16 @@ from workloads import (BLOCK_7B, BLOCK_7B_LAYERS, DOWN_7B, DOWN_72B, Q_PROJ_7B, 
 WORKLOADS = {"q_proj": Q_PROJ_7B, "q_proj_2blk": Q_PROJ_7B_2BLK, "tiny": TINY, "down_7b": DOWN_7B,
              "down_72b": DOWN_72B, "block_7b": BLOCK_7B}
 METRIC = "signsgd_steps_per_sec"
+
+
+def _workload(args):
+    """The named layer workload, with --group-size applied (-1: one group per row)."""
+    c = WORKLOADS[args.workload]
+    gs = getattr(args, "group_size", None)
+    if gs is None or gs == c.group_size:
+        return c
+    label = "per-channel (group_size -1)" if gs == -1 else f"group_size {gs}"
+    return dataclasses.replace(c, group_size=gs, name=f"{c.name}, {label}")
 UNIT = "steps/s"
 
 
@@ -237,7 +248,7 @@ def run_fp_target(args):
         return None if rank else {"metric": METRIC, "unavailable": "--mode fp_target runs on one GPU"}
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    c = WORKLOADS[args.workload]
+    c = _workload(args)
     W = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0))
     Wd = (W.to(torch.bfloat16) if c.w_dtype == "bf16" else W).to(dev)
     Xt = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
@@ -295,7 +306,7 @@ def run_ours(args):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    c = WORKLOADS[args.workload]
+    c = _workload(args)
     # Each rank tunes its own shard of output rows (weak scaling): rank r's rows
     # are drawn with seed r; the calibration activations are the same on every rank.
     W = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=rank))
@@ -305,7 +316,7 @@ def run_ours(args):
                        minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
                        split=bool(args.split))
     ws = torch.empty(ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
-    G = c.inn // c.group_size
+    G = c.inn // (c.inn if c.group_size == -1 else c.group_size)
     outs = (torch.empty((c.out, c.inn), dtype=torch.uint8, device=dev),
             torch.empty((c.out, G), dtype=torch.float32, device=dev),
             torch.empty((c.out, G), dtype=torch.int32, device=dev),
@@ -495,7 +506,7 @@ def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
         return None
-    c = WORKLOADS[args.workload]
+    c = _workload(args)
     import oracle
     X = _host_x(c)
     W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
@@ -538,6 +549,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--algo", choices=["auto", "direct", "gram"], default="auto")
     ap.add_argument("--split", type=int, default=1, help="1: bf16-pair operands (default); 0: single bf16")
+    ap.add_argument("--group-size", type=int, default=None,
+                    help="override the workload's group size (-1: one group per row)")
     ap.add_argument("--mode", choices=["layer", "fp_target"], default="layer",
                     help="fp_target: quant-aware input with a full-precision target")
     args = ap.parse_args()
