@@ -409,6 +409,12 @@ def run_ours(args):
     else:
         dom_name, dom_ms, dom_flops = "update (kEpiUpdate)", upd_ms, flops_upd
         traffic = _recorded_traffic(f"{algo}_update_bytes")
+        g_eff = c.inn if c.group_size == -1 else c.group_size
+        if not (256 % g_eff == 0 or (g_eff == c.inn and c.inn <= 256)):
+            # groups wider than an epilogue thread's columns: the step is the
+            # kEpiUpdateWide launch plus group_finish_kernel (timed together); the
+            # recorded traffic is the narrow-group kernel's
+            dom_name, traffic = "update (kEpiUpdateWide) + group_finish_kernel", None
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     layer_s = ms_max / args.steps / 1e3
     step_ms = res_ms + upd_ms
