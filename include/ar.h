@@ -192,7 +192,7 @@ size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
  *   final_mse   1 double out: mean((X W'^T - X W^T)^2) over all n_rows rows with
  *               the applied W', may be NULL (skips one pass over X).
  * Supported shapes: in a multiple of 32; batch_rows a multiple of 8; group size
- * (group_size, or in for -1) a multiple of 32 (else AR_EUNSUPPORTED).  Groups that
+ * (group_size, or in for -1) a multiple of 16 (else AR_EUNSUPPORTED).  Groups that
  * divide 256 (or a whole row of at most 256) are updated inside the step kernel;
  * any other (a whole row of a wider layer, or sizes such as 96 or 384) through
  * per-segment partials and one small kernel per step.  out == 0 or in == 0 is a

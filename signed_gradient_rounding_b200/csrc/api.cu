@@ -118,11 +118,11 @@ ar_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AR_OK : AR_ECUDA;
     if (e_ != cudaSuccess) return AR_ECUDA; \
   } while (0)
 
-// Groups are whole multiples of 32 columns (the update epilogue walks 16-column
+// Groups are whole multiples of 16 columns (the update epilogue walks 16-column
 // chunks that never straddle a group).
 bool tune_shape_supported(int64_t in, int64_t g, int64_t B) {
   if (in % 32 != 0 || B % 8 != 0) return false;
-  return g % 32 == 0;
+  return g % 16 == 0;
 }
 
 // Groups that fit inside one epilogue thread's columns are updated in the step's

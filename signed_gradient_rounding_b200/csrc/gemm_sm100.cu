@@ -586,7 +586,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
 
 // kEpiUpdate*Wide: groups wider than a thread's columns, or not aligned to them.
 // This thread walks its column half (kSegCols columns, one 128-column segment of
-// the row) in chunks of kUC; a chunk lies in one group (g is a multiple of 32).
+// the row) in chunks of kUC; a chunk lies in one group (g is a multiple of 16).
 // Per element it does what epi_update's first pass does (G, the row loss, the new
 // V, the V snapshot); the group's d alpha and d beta over this segment go to
 // GemmArgs::gpart, and launch_group_finish completes the group.

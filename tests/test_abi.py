@@ -63,11 +63,11 @@ def test_tune_validation(ar):
     assert call(64, 256, 1000, batch_rows=512, group_size=64) == ar.AR_EINVAL         # n % B
     assert call(64, 256, 1024, batch_rows=512, group_size=64, iters=-1) == ar.AR_EINVAL
     assert call(64, 256, 1024, batch_rows=512, group_size=64, lr=-0.1) == ar.AR_EINVAL
-    assert call(64, 256, 1024, batch_rows=512, group_size=16) == ar.AR_EUNSUPPORTED   # g < 32
-    assert call(64, 288, 1024, batch_rows=512, group_size=48) == ar.AR_EUNSUPPORTED   # g % 32
+    assert call(64, 256, 1024, batch_rows=512, group_size=8) == ar.AR_EUNSUPPORTED    # g < 16
+    assert call(64, 288, 1024, batch_rows=512, group_size=24) == ar.AR_EUNSUPPORTED   # g % 16
     assert call(64, 1024, 1024, batch_rows=512, group_size=384) == ar.AR_EINVAL        # in % g
     # groups wider than an epilogue thread's columns (or not dividing 256) are supported
-    for inn, g in ((1024, 512), (1024, -1), (288, 96), (768, 384), (4096, -1)):
+    for inn, g in ((1024, 512), (1024, -1), (288, 96), (768, 384), (4096, -1), (256, 16), (288, 48)):
         p = ar.make_params(batch_rows=512, group_size=g)
         assert ar.tune_workspace_bytes(64, inn, 1024, p) > 0, (inn, g)
     assert call(64, 250, 1024, batch_rows=512, group_size=-1) == ar.AR_EUNSUPPORTED   # in % 32
@@ -126,7 +126,7 @@ def test_host_entry_validation(ar):
     assert call(64, 256, 1000, batch_rows=512, group_size=64) == ar.AR_EINVAL
     assert call(64, 256, 1024, W=None, batch_rows=512, group_size=64) == ar.AR_EINVAL
     assert call(64, 256, 1024, codes=None, batch_rows=512, group_size=64) == ar.AR_EINVAL
-    assert call(64, 256, 1024, batch_rows=512, group_size=16) == ar.AR_EUNSUPPORTED
+    assert call(64, 256, 1024, batch_rows=512, group_size=8) == ar.AR_EUNSUPPORTED
     assert call(64, 256, 1024, ws_bytes=need - 1, batch_rows=512, group_size=64) == ar.AR_ENOMEM
     assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK
 

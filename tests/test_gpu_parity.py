@@ -300,7 +300,7 @@ def test_rejects_unsupported(ar):
     W = torch.zeros((64, 256), dtype=torch.bfloat16, device="cuda")
     X = torch.zeros((512, 256), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ar.ArError) as e:
-        ar.tune_layer(W, X, ar.make_params(group_size=16, batch_rows=512))
+        ar.tune_layer(W, X, ar.make_params(group_size=8, batch_rows=512))
     assert e.value.status in (ar.AR_EUNSUPPORTED, ar.AR_EINVAL)
 
 

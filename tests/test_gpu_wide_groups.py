@@ -1,9 +1,9 @@
-"""Tuning with groups wider than an epilogue thread's columns, against the oracle.
+"""Tuning with group sizes other than the usual 32 .. 256, against the oracle.
 
 The pages' group size is -1 (a whole row) or any divisor of the row width.  Groups
-that divide 256 are updated inside the step kernel's epilogue.  Any other group
-(a whole row of a wide layer, 384 or 512 columns, or sizes such as 96 and 160 whose
-groups straddle the epilogue's 128-column segments) takes the wide path: the
+that divide 256 (16 included) are updated inside the step kernel's epilogue.  Any
+other group (a whole row of a wide layer, 384 or 512 columns, or sizes such as 48,
+96 and 160 whose groups straddle the epilogue's 128-column segments) takes the wide path: the
 epilogue writes per-segment partials of d alpha and d beta, and a per-group kernel
 finishes the clip-factor update and the next D.  Both evaluation orders, both
 quantiser modes, keep-best and the last iterate, the MSE init and the
@@ -48,7 +48,7 @@ def _close(res, ref, what):
 
 # (in, group_size): whole rows wider than 256, groups spanning several segments,
 # and groups that straddle segment boundaries (96, 160).
-SHAPES = [(384, -1), (512, -1), (768, 384), (1024, 512), (288, 96), (320, 160)]
+SHAPES = [(384, -1), (512, -1), (768, 384), (1024, 512), (288, 96), (320, 160), (256, 16), (288, 48)]
 
 
 @pytest.mark.parametrize("algo", ["gram", "direct"])
