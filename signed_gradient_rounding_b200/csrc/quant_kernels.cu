@@ -328,13 +328,46 @@ __global__ void group_finish_kernel(GroupFinishArgs a) {
   const GroupScale gn = group_scale(a.wmin[grp], a.wmax[grp], al_n, be_n, a.bits, sym);
   const float Q = qmaxf(a.bits);
   const bool fast = a.div_slow && *a.div_slow == 0;
+  // Eight consecutive elements per lane and iteration (g is a multiple of 16 and
+  // in of 32, so the vectors are aligned and never straddle a group).
   const int64_t base = j * a.in + gg * a.g;
-  for (int k = lane; k < a.g; k += 32) {
-    const float w = load_w(a.W, a.w_bf16, base + k);
-    const float d = __fsub_rn(quant_elem(w, a.V[base + k], gn, Q, fast).wq, w);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(d);
-    a.D_hi[base + k] = hi;
-    if (a.D_lo) a.D_lo[base + k] = __float2bfloat16_rn(__fsub_rn(d, __bfloat162float(hi)));
+  for (int k = lane * 8; k < a.g; k += 32 * 8) {
+    const int64_t e = base + k;
+    float w[8], v[8];
+    if (a.w_bf16) {
+      const uint4 x = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.W) + e);
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        w[2 * h] = __uint_as_float(xs[h] << 16);
+        w[2 * h + 1] = __uint_as_float(xs[h] & 0xFFFF0000u);
+      }
+    } else {
+      const float4 x0 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.W) + e);
+      const float4 x1 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.W) + e + 4);
+      w[0] = x0.x, w[1] = x0.y, w[2] = x0.z, w[3] = x0.w, w[4] = x1.x, w[5] = x1.y, w[6] = x1.z, w[7] = x1.w;
+    }
+    const float4 v0 = *reinterpret_cast<const float4*>(a.V + e);
+    const float4 v1 = *reinterpret_cast<const float4*>(a.V + e + 4);
+    v[0] = v0.x, v[1] = v0.y, v[2] = v0.z, v[3] = v0.w, v[4] = v1.x, v[5] = v1.y, v[6] = v1.z, v[7] = v1.w;
+    uint32_t hi2[4], lo2[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float hv[2], lv[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int i = 2 * h + q;
+        const float d = __fsub_rn(quant_elem(w[i], v[i], gn, Q, fast).wq, w[i]);
+        hv[q] = __bfloat162float(__float2bfloat16_rn(d));
+        lv[q] = __fsub_rn(d, hv[q]);
+      }
+      const __nv_bfloat162 hp = __floats2bfloat162_rn(hv[0], hv[1]);
+      const __nv_bfloat162 lp = __floats2bfloat162_rn(lv[0], lv[1]);
+      hi2[h] = *reinterpret_cast<const uint32_t*>(&hp);
+      lo2[h] = *reinterpret_cast<const uint32_t*>(&lp);
+    }
+    *reinterpret_cast<uint4*>(a.D_hi + e) = make_uint4(hi2[0], hi2[1], hi2[2], hi2[3]);
+    if (a.D_lo) *reinterpret_cast<uint4*>(a.D_lo + e) = make_uint4(lo2[0], lo2[1], lo2[2], lo2[3]);
   }
 }
 
