@@ -476,6 +476,18 @@ def _threads():
     return os.cpu_count()
 
 
+def _cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "" when unknown."""
+    try:
+        with open("/proc/cpuinfo", encoding="utf-8") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 def _host_x(c, Xd=None):
     """The workload's activations on the host as bf16 bit patterns (same bytes as the GPU run)."""
     try:
@@ -505,7 +517,7 @@ def cpu_baseline(c, Xd, rows: int, steps: int):
     return {"value": steps * (len(sel) / c.out) / dt, "unit": UNIT, "cores": _threads(), "kind": "oracle",
             "sample": f"{len(sel)} of {c.out} output rows x {steps} steps on the full activations, "
                       f"{dt:.1f} s; rate scaled by rows/out (rows tune independently)",
-            "host_cpu": os.cpu_count()}
+            "host_cpu": os.cpu_count(), "cpu_model": _cpu_model()}
 
 
 def run_reference(args):
@@ -538,7 +550,8 @@ def run_reference(args):
                        "group_size": c.group_size, "sym": c.sym},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
                              "sample": f"each step: {len(sel)} of {c.out} output rows x {args.cpu_steps} "
-                                       f"SignSGD steps; rate scaled by rows/out"},
+                                       f"SignSGD steps; rate scaled by rows/out",
+                             "host_cpu": os.cpu_count(), "cpu_model": _cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
