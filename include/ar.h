@@ -210,7 +210,9 @@ ar_status ar_tune_layer(const void* W, ar_dtype w_dtype, int64_t out, int64_t in
 typedef struct {
   float residual_ms;         /* DIRECT: summed device time of the R = X_b (W' - W)^T
                                 contractions; GRAM: 0 */
-  float update_ms;           /* summed device time of the G contractions + updates */
+  float update_ms;           /* summed device time of the G contractions + updates (with
+                                groups wider than 256 or not dividing it, each step's
+                                group-finish kernel too) */
   float total_ms;            /* device time of the whole call */
   int32_t gemm_launches;     /* launches of each timed contraction (= iters) */
   int32_t kernel_launches;   /* every kernel this call launched */
