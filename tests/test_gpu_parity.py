@@ -325,9 +325,10 @@ def _check_full_size(ar, case, algo, mse_rows=65536):
     codes = _np(res.codes)[rows]
     frac = float(np.mean(codes != ref.codes))
     # MSE of the GPU's sampled rows, evaluated by the oracle's own fp64 loss
+    g = c.inn if c.group_size == -1 else c.group_size
     s = _np(res.scale)[rows]
     z = _np(res.zero_point)[rows].astype(np.float32)
-    Wq_gpu = np.repeat(s, c.group_size, 1) * (codes.astype(np.float32) - np.repeat(z, c.group_size, 1))
+    Wq_gpu = np.repeat(s, g, 1) * (codes.astype(np.float32) - np.repeat(z, g, 1))
     mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:mse_rows])
     mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:mse_rows])
     print(f"{c.name} {algo}: {frac:.3%} of sampled codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
@@ -348,6 +349,16 @@ def test_down_72b_full_size_sampled_rows(ar, algo):
     """Qwen2.5-72B down_proj, 8192 x 29568 W2 g128, 262144 x 29568 activations (15.5 GB),
     200 steps; the oracle replays 32 sampled rows."""
     _check_full_size(ar, _full_size_case(DOWN_72B, 32), algo, mse_rows=16384)
+
+
+@pytest.mark.parametrize("algo", ["gram"])
+def test_q_proj_per_channel_full_size_sampled_rows(ar, algo):
+    """The q_proj workload at full size with per-channel groups (group_size -1: one
+    4096-wide group per row, the wide-group path), 200 steps; the oracle replays 32
+    sampled rows."""
+    import dataclasses
+    c = dataclasses.replace(Q_PROJ_7B, group_size=-1, name="q_proj per-channel")
+    _check_full_size(ar, _full_size_case(c, 32), algo)
 
 
 @pytest.fixture(scope="module")
