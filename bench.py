@@ -48,8 +48,9 @@ def _workload(args):
     gs = getattr(args, "group_size", None)
     if gs is None or gs == c.group_size:
         return c
-    label = "per-channel (group_size -1)" if gs == -1 else f"group_size {gs}"
-    return dataclasses.replace(c, group_size=gs, name=f"{c.name}, {label}")
+    label = "per-channel" if gs == -1 else f"g{gs}"
+    name = c.name.replace(f" g{c.group_size}", f" {label}") if f" g{c.group_size}" in c.name else f"{c.name}, {label}"
+    return dataclasses.replace(c, group_size=gs, name=name)
 UNIT = "steps/s"
 
 
