@@ -191,24 +191,36 @@ def _autograd_grads(W, V, alpha, beta, wmin, wmax, X, g, bits, sym, X_target=Non
 @pytest.mark.parametrize("sym", [False, True])
 @pytest.mark.parametrize("bits", [2, 4])
 def test_gradients_match_autograd(sym, bits):
-    out, inn, g, n = 8, 64, 16, 48
+    _check_gradients(sym, bits, 16)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("bits", [2, 4])
+def test_whole_row_gradients_match_autograd(sym, bits):
+    """group_size = -1: d alpha and d beta summed over the whole row."""
+    _check_gradients(sym, bits, -1)
+
+
+def _check_gradients(sym, bits, group_size):
+    out, inn, n = 8, 64, 48
+    g = inn if group_size == -1 else group_size
     W = make_weight(out, inn, 0.02, "f32", seed=11)
     X = _tiny_x(n, inn, seed=12)
     rng = np.random.default_rng(13)
     V = rng.uniform(-0.5, 0.5, W.shape).astype(np.float32)
-    wmin, wmax = oracle.group_minmax(W, g)
+    wmin, wmax = oracle.group_minmax(W, group_size)
     alpha = rng.uniform(0.5, 1.0, wmin.shape).astype(np.float32)
     beta = rng.uniform(0.5, 1.0, wmin.shape).astype(np.float32)
     dV, da, db, R = _autograd_grads(W, V, alpha, beta, wmin, wmax, X, g, bits, sym)
     G = R.T @ X.astype(np.float64)
-    sgn, dalpha, dbeta = oracle.step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym)
+    sgn, dalpha, dbeta = oracle.step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size, bits, sym)
     c = 2.0 / (n * out)                    # the factor the oracle leaves out of G
     assert np.array_equal(sgn[np.abs(dV) > 1e-12], np.sign(dV)[np.abs(dV) > 1e-12])
     assert np.all(sgn[dV == 0] == 0)
     np.testing.assert_allclose(c * dalpha, da, rtol=1e-9, atol=1e-15)
     np.testing.assert_allclose(c * dbeta, db, rtol=1e-9, atol=1e-15)
     # the clamp must have been active somewhere, so the clamped branch is exercised
-    fq = oracle.fake_quant(W, V, *oracle.scale_zero_point(wmin, wmax, alpha, beta, bits, sym), g, bits)
+    fq = oracle.fake_quant(W, V, *oracle.scale_zero_point(wmin, wmax, alpha, beta, bits, sym), group_size, bits)
     assert (~fq.m).any() and fq.m.any()
 
 
