@@ -909,7 +909,7 @@ using namespace ar;
 
 extern "C" {
 
-const char* ar_version(void) { return "ar 0.3.0 sm_100a"; }
+const char* ar_version(void) { return "ar 0.4.0 sm_100a"; }
 
 const char* ar_status_string(ar_status s) {
   switch (s) {
