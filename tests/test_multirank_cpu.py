@@ -36,7 +36,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, W, X, result_q):
+def _worker(rank, world, port, W, X, result_q, group_size=32):
     import oracle
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -44,7 +44,7 @@ def _worker(rank, world, port, W, X, result_q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
 
     def compute(Wr, Xr):
-        res = oracle.tune_layer(Wr.numpy(), Xr.numpy(), 4, 32, False, 12, 0.005, 0.005, 32, 4,
+        res = oracle.tune_layer(Wr.numpy(), Xr.numpy(), 4, group_size, False, 12, 0.005, 0.005, 32, 4,
                                 want_final_mse=False)
         return (torch.from_numpy(res.codes), torch.from_numpy(res.scale), torch.from_numpy(res.zero_point))
 
@@ -58,7 +58,8 @@ def _worker(rank, world, port, W, X, result_q):
     dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_gather_equals_single_run():
+@pytest.mark.parametrize("group_size", [32, -1], ids=["g32", "per-channel"])
+def test_two_gloo_ranks_gather_equals_single_run(group_size):
     import oracle
     from workloads import bf16_round, make_weight
     W = make_weight(300, 64, 0.02, "f32", seed=3)
@@ -66,14 +67,14 @@ def test_two_gloo_ranks_gather_equals_single_run():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, W, X, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, W, X, q, group_size)) for r in range(2)]
     for p in procs:
         p.start()
     codes, scale, zp, rng, tmax = q.get(timeout=240)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    ref = oracle.tune_layer(W, X, 4, 32, False, 12, 0.005, 0.005, 32, 4, want_final_mse=False)
+    ref = oracle.tune_layer(W, X, 4, group_size, False, 12, 0.005, 0.005, 32, 4, want_final_mse=False)
     assert rng == (0, 300)
     assert np.array_equal(codes, ref.codes)
     assert np.array_equal(scale, ref.scale)
