@@ -207,7 +207,8 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   const double pieces_direct = P.split ? 2.0 : 1.0;
   const double pieces_gram = P.split ? 3.0 : 1.0;
   const double direct = P.iters * pieces_direct * 4.0 * P.B * out * in + pieces_direct * 2.0 * n * out * in;
-  const double gram = P.iters * pieces_gram * 2.0 * out * in * in + 2.0 * n * in * in + pieces_gram * 2.0 * out * in * in;
+  const double gram =
+      P.iters * pieces_gram * 2.0 * out * in * in + 2.0 * n * in * in + pieces_gram * 2.0 * out * in * in;
   const double gram_bytes = (P.nb + 1.0) * in * in * 2.0 * (P.split ? 2.0 : 1.0);
   if (p->algo == AR_ALGO_GRAM || (fp_target && p->algo == AR_ALGO_AUTO))
     P.algo = AR_ALGO_GRAM;
@@ -231,11 +232,12 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
 
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
-  size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1, wmin, wmax,
-      part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
-      // full-precision-target mode: this block's dX = X - X_target (pair), M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b
-      // (pair), their sum Cs (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the
-      // partials of e_b, and W as a pair when it is fp32
+  size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1,
+      wmin, wmax, part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
+      // full-precision-target mode: this block's dX = X - X_target (pair),
+      // M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b (pair), their sum Cs
+      // (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the partials of e_b, and W as
+      // a pair when it is fp32
       dX_hi, dX_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo, total;
 };
 
