@@ -52,3 +52,15 @@ def test_gemm_fingerprint_ignores_comments_only():
     assert bench._strip_comments(a) != bench._strip_comments(a.replace("x + 1", "x + 2"))
     assert "a//b" in bench._strip_comments(a)
     assert len(bench.gemm_code_fingerprint()) == 16
+
+
+def test_group_size_override_names_the_workload():
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    c = bench._workload(argparse.Namespace(workload="q_proj", group_size=-1))
+    assert c.group_size == -1 and "per-channel" in c.name and "g128" not in c.name
+    c = bench._workload(argparse.Namespace(workload="q_proj", group_size=64))
+    assert c.group_size == 64 and " g64" in c.name
+    c = bench._workload(argparse.Namespace(workload="q_proj", group_size=None))
+    assert c is bench.WORKLOADS["q_proj"]
