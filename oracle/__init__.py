@@ -48,6 +48,7 @@ from .autoround import (  # noqa: F401
     qmax,
     rtn,
     scale_zero_point,
+    sign_step,
     step_gradients,
     tune_layer,
 )

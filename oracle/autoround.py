@@ -192,7 +192,8 @@ def mse_init(W, group_size: int, bits: int, sym: bool):
 # backward: straight-through derivatives of W' with respect to V, alpha, beta
 # --------------------------------------------------------------------------
 
-def step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size: int, bits: int, sym: bool):
+def step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size: int, bits: int, sym: bool,
+                   with_scale: bool = False):
     """Gradients of the loss at (V, alpha, beta), given G = dL/dW' up to a positive factor.
 
     The page's loop back-propagates through ``torch.round``; reading: a
@@ -200,7 +201,10 @@ def step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size: int, bits: int,
     passes the gradient as the identity, and every clamp passes it only where its
     input lies inside the closed interval (torch.clamp's rule).
 
-    Returns (sgn_dV fp32 [out, in] in {-1, 0, 1}, dalpha fp64 [out, G], dbeta fp64 [out, G]).
+    Returns (sgn_dV fp32 [out, in] in {-1, 0, 1}, dalpha fp64 [out, G], dbeta fp64 [out, G]);
+    with ``with_scale`` also the sums of the terms' magnitudes, sum_k |G*dW'/dalpha| and
+    sum_k |G*dW'/dbeta| per group: the scale against which a rounding error in a
+    group sum is measured (a sum far below it is a near-tie of its sign).
     With ds_a = ds/dalpha, ds_b = ds/dbeta:
       in range (m = 1):  W' = s*r, so dW'/dtheta = ds_theta * (r - W/s)  (zp cancels);
       clamped  (m = 0):  W' = s*(q - zp), so dW'/dtheta = ds_theta*(q - zp) - s*dzp/dtheta,
@@ -247,12 +251,69 @@ def step_gradients(W, V, alpha, beta, wmin, wmax, G, group_size: int, bits: int,
     if sym:
         dbeta = np.zeros_like(dbeta)
     sgn_dV = (np.sign(G) * m).astype(F32)
-    return sgn_dV, dalpha, dbeta
+    if not with_scale:
+        return sgn_dV, dalpha, dbeta
+    abs_a = np.abs(G * dWa).reshape(out, inn // g, g).sum(axis=2)
+    abs_b = np.zeros_like(abs_a) if sym else np.abs(G * dWb).reshape(out, inn // g, g).sum(axis=2)
+    return sgn_dV, dalpha, dbeta, abs_a, abs_b
 
 
 # --------------------------------------------------------------------------
 # the tuning loop
 # --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Step:
+    """One SignSGD step of the tuning loop from a given state (see ``sign_step``)."""
+
+    row_loss: np.ndarray     # fp64 [out]: batch MSE of each output row, mean_b (Y' - Y)_bj^2
+    G: np.ndarray            # fp64 [out, in]: R^T X_b, dL/dW' up to the factor 2/(B*out)
+    sgn_dV: np.ndarray       # fp32 [out, in]: sign(dL/dV) in {-1, 0, 1}
+    dalpha: np.ndarray       # fp64 [out, G]
+    dbeta: np.ndarray        # fp64 [out, G] (zeros when sym)
+    dalpha_abs: np.ndarray | None  # fp64 [out, G]: sum_k |G*dW'/dalpha|, the scale of dalpha's rounding
+    dbeta_abs: np.ndarray | None   # fp64 [out, G]
+    V: np.ndarray            # fp32 [out, in]: the state after the update
+    alpha: np.ndarray        # fp32 [out, G]
+    beta: np.ndarray         # fp32 [out, G]
+
+
+def sign_step(W, Xb, V, alpha, beta, wmin, wmax, group_size: int, bits: int, sym: bool, lr: float,
+              minmax_lr: float, Xt_b=None, with_scale: bool = False) -> Step:
+    """One step of the per-layer loop ("[llm-compressor] AutoRound ...", "on_event with
+    SEQUENTIAL_EPOCH_END": fake-quantise, forward, MSE, backward, sign update).
+
+    Xb: this step's calibration block as fp64 [B, in] (Xt_b: the target's inputs of
+    the same rows, or None for Y = X_b W^T).  R = Y' - Y = X_b W'^T - X_b W^T (or
+    X_b W'^T - Xt_b W^T), the row losses mean_b R_bj^2, G = R^T X_b, the
+    straight-through gradients, then V <- clamp(V - lr*sign(dL/dV), -0.5, 0.5) and
+    alpha, beta <- clamp(. - minmax_lr*sign(.), 0.5, 1), all from the same point.
+    ``with_scale`` also fills dalpha_abs and dbeta_abs (otherwise None).
+    """
+    W = _to_f32(W)
+    g = _group(W.shape[1], group_size)
+    lr32 = F32(lr)
+    mlr32 = F32(lr if minmax_lr < 0 else minmax_lr)
+    s, zp = scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
+    Wq = fake_quant(W, V, s, zp, g, bits).Wq
+    if Xt_b is None:
+        R = Xb @ (Wq.astype(F64) - W.astype(F64)).T      # Y' - Y  [B, out]
+    else:
+        R = Xb @ Wq.astype(F64).T - Xt_b @ W.astype(F64).T
+    row_loss = np.sum(R * R, axis=0) / Xb.shape[0]
+    G = R.T @ Xb                                          # dL/dW' * (B*out/2)  [out, in]
+    if with_scale:
+        sgn_dV, dalpha, dbeta, abs_a, abs_b = step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym,
+                                                             with_scale=True)
+    else:
+        sgn_dV, dalpha, dbeta = step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym)
+        abs_a = abs_b = None
+    V_new = np.clip(V - lr32 * sgn_dV, F32(-0.5), F32(0.5)).astype(F32)
+    a_new = np.clip(alpha - mlr32 * np.sign(dalpha).astype(F32), F32(0.5), F32(1.0)).astype(F32)
+    b_new = beta.copy() if sym else np.clip(beta - mlr32 * np.sign(dbeta).astype(F32), F32(0.5),
+                                            F32(1.0)).astype(F32)
+    return Step(row_loss, G, sgn_dV, dalpha, dbeta, abs_a, abs_b, V_new, a_new, b_new)
+
 
 @dataclasses.dataclass
 class TuneResult:
@@ -269,6 +330,9 @@ class TuneResult:
     V_best: np.ndarray       # per row, the state at that row's best step (initial if none)
     alpha_best: np.ndarray
     beta_best: np.ndarray
+    row_loss_trace: np.ndarray | None = None  # fp64 [iters, out]: each row's batch loss per step
+    best_step: np.ndarray | None = None       # int64 [out]: step index (start_step-based) of the
+                                              # applied best state; -1 if no step improved on best0
 
 
 def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
@@ -346,31 +410,25 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     W64 = W.astype(F64)
     cache: dict[int, np.ndarray] = {}
     trace = np.zeros(iters, dtype=F64)
+    row_trace = np.zeros((iters, out), dtype=F64)
+    best_step = np.full(out, -1, dtype=np.int64)
     for t in range(iters):
         blk = sched[t]
         if blk not in cache:
             cache[blk] = _rows_f64(X, blk * batch_rows, (blk + 1) * batch_rows)
         Xb = cache[blk]
-        s, zp = scale_zero_point(wmin, wmax, alpha, beta, bits, sym)
-        Wq = fake_quant(W, V, s, zp, g, bits).Wq
-        if X_target is None:
-            R = Xb @ (Wq.astype(F64) - W64).T      # Y' - Y  [B, out]
-        else:
-            Xt_b = _rows_f64(X_target, blk * batch_rows, (blk + 1) * batch_rows)
-            R = Xb @ Wq.astype(F64).T - Xt_b @ W64.T
-        row_loss = np.sum(R * R, axis=0) / batch_rows
+        Xt_b = None if X_target is None else _rows_f64(X_target, blk * batch_rows, (blk + 1) * batch_rows)
+        st = sign_step(W, Xb, V, alpha, beta, wmin, wmax, g, bits, sym, lr32, mlr32, Xt_b)
+        row_loss = st.row_loss
+        row_trace[t] = row_loss
         trace[t] = float(np.sum(row_loss)) / out
         better = row_loss < best_loss
         best_loss = np.where(better, row_loss, best_loss)
+        best_step[better] = start_step + t
         V_best[better] = V[better]
         a_best[better] = alpha[better]
         b_best[better] = beta[better]
-        G = R.T @ Xb                                # dL/dW' * (B*out/2)  [out, in]
-        sgn_dV, dalpha, dbeta = step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym)
-        V = np.clip(V - lr32 * sgn_dV, F32(-0.5), F32(0.5)).astype(F32)
-        alpha = np.clip(alpha - mlr32 * np.sign(dalpha).astype(F32), F32(0.5), F32(1.0)).astype(F32)
-        if not sym:
-            beta = np.clip(beta - mlr32 * np.sign(dbeta).astype(F32), F32(0.5), F32(1.0)).astype(F32)
+        V, alpha, beta = st.V, st.alpha, st.beta
 
     Va, aa, ba = (V_best, a_best, b_best) if keep_best else (V, alpha, beta)
     s, zp = scale_zero_point(wmin, wmax, aa, ba, bits, sym)
@@ -390,7 +448,7 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
             acc += float(np.sum(R * R))
         mse = acc / (n * out)
     return TuneResult(fq.q.astype(np.uint8), s, zp.astype(np.int32), fq.Wq, V, alpha, beta,
-                      trace, mse, best_loss, V_best, a_best, b_best)
+                      trace, mse, best_loss, V_best, a_best, b_best, row_trace, best_step)
 
 
 def layer_mse(W, Wq, X) -> float:
