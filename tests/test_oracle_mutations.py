@@ -172,3 +172,25 @@ def test_dropped_target_input_is_caught(monkeypatch):
     _plant(monkeypatch, "tune_layer", dropped)
     assert _caught(lambda: pins.test_fp_target_gradients_match_autograd(False),
                    lambda: pins.test_fp_target_final_mse_and_same_input())
+
+
+_orig_tune = oar.tune_layer
+
+
+def _tune_shrink_ignored(*args, **kw):
+    kw["minmax_shrink"] = 1.0                                            # the start ignores minmax_shrink
+    return _orig_tune(*args, **kw)
+
+
+def _tune_shrink_alpha_only(W, X, bits, group_size, sym, iters, lr, minmax_lr, batch_rows, seed,
+                            minmax_shrink=1.0, **kw):
+    wmin, _ = oar.group_minmax(W, group_size)
+    kw["beta0"] = np.ones(wmin.shape, F32)                               # beta left at 1
+    return _orig_tune(W, X, bits, group_size, sym, iters, lr, minmax_lr, batch_rows, seed,
+                      minmax_shrink=minmax_shrink, **kw)
+
+
+@pytest.mark.parametrize("slip", [_tune_shrink_ignored, _tune_shrink_alpha_only])
+def test_minmax_shrink_mistakes_are_caught(monkeypatch, slip):
+    _plant(monkeypatch, "tune_layer", slip)
+    assert _caught(lambda: pins.test_minmax_shrink_worked_example(0), lambda: pins.test_minmax_shrink_worked_example(1))

@@ -39,6 +39,31 @@ def test_rtn_worked_grid_example():
     assert np.array_equal(Wq, W)
 
 
+@pytest.mark.parametrize("case", [0, 1])
+def test_minmax_shrink_worked_example(case):
+    """minmax_shrink ("AutoRoundModifier 생성자 파라미터": the initial min/max range is
+    scaled by this factor) on hand-worked grid groups: at iters = 0 the applied
+    state is alpha = beta = shrink with V = 0, so the tuned layer's scale, zero-point
+    and codes are the hand-worked ones; with shrink 1 they are the RTN ones."""
+    d = json.load(open(os.path.join(GOLDEN, "shrink_grid_example.json")))["cases"][case]
+    W = np.array([d["w"]], dtype=np.float32)
+    X = _tiny_x(8, W.shape[1], seed=case)
+    res = oracle.tune_layer(W, X, d["bits"], d["group_size"], d["sym"], 0, 0.005, -1.0, 8, 0,
+                            minmax_shrink=d["minmax_shrink"])
+    assert res.scale[0, 0] == F32(d["scale"])
+    assert res.zero_point[0, 0] == d["zero_point"]
+    assert res.codes[0].tolist() == d["codes"]
+    one = oracle.tune_layer(W, X, d["bits"], d["group_size"], d["sym"], 0, 0.005, -1.0, 8, 0, minmax_shrink=1.0)
+    assert one.scale[0, 0] == F32(d["rtn_scale"])
+    assert one.codes[0].tolist() == d["rtn_codes"]
+    # the shrunk start is where tuning begins: one step moves alpha (and beta) off it
+    # by at most minmax_lr, inside [0.5, 1]
+    r1 = oracle.tune_layer(W, X, d["bits"], d["group_size"], d["sym"], 1, 0.005, 0.005, 8, 0,
+                           minmax_shrink=d["minmax_shrink"], keep_best=False)
+    assert abs(float(r1.alpha[0, 0]) - d["minmax_shrink"]) <= 0.005 + 1e-9
+    assert 0.5 <= float(r1.alpha[0, 0]) <= 1.0
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
 @pytest.mark.parametrize("sym", [False, True])
 def test_rtn_is_nearest_level(bits, sym):
