@@ -27,6 +27,23 @@
  *     enqueued and no output has been written.  Errors detected on the device
  *     (a bounded wait that ran out) are recorded in the workspace and read with
  *     ar_tune_status().  Nothing aborts the process.
+ *   - Test hooks, read from the environment on every call (no GPU fault is ever
+ *     made; a test can set and clear them between calls):
+ *       AR_FAULT=param   every argument check fails: AR_EINVAL, nothing enqueued.
+ *       AR_FAULT=alloc   the tuning entry points fail as if their workspace (or,
+ *                        for ar_tune_layer_host, its stream and events) could not
+ *                        be had: AR_ENOMEM, nothing enqueued.
+ *       AR_FAULT=launch  the first contraction launch of a tuning call fails:
+ *                        AR_ECUDA; set-up work already enqueued on the workspace
+ *                        stays, no output is written, the next call works.
+ *       AR_FAULT=bounds  with AR_CHECKS, the step kernels are told that V and D hold
+ *                        one element fewer than they do: their last store is
+ *                        refused and reported (AR_ECHECK from ar_tune_status).
+ *       AR_CHECKS=1      the tuning kernels check every store to V, V_best, D, the
+ *                        clip factors, the Gram matrices, the residual and the
+ *                        outputs against the buffer sizes; a store outside is
+ *                        skipped and recorded in the workspace's status word
+ *                        (ar_tune_status returns AR_ECHECK).  Never traps.
  *   - Shapes: W is [out, in]; a quantisation group is `group_size` consecutive
  *     elements of one row (-1: the whole row); G = in / group_size groups per row.
  *     Q = 2^bits - 1.  Codes are unsigned in [0, Q].
@@ -56,7 +73,8 @@ typedef enum {
   AR_EUNSUPPORTED = 2,  /* valid for the method, not implemented by this library */
   AR_ENOMEM = 3,        /* the workspace is smaller than ar_tune_workspace_bytes() */
   AR_ECUDA = 4,         /* a CUDA call failed (no device, launch failure, ...) */
-  AR_ETIMEOUT = 5       /* a device-side bounded wait ran out (see ar_tune_status) */
+  AR_ETIMEOUT = 5,      /* a device-side bounded wait ran out (see ar_tune_status) */
+  AR_ECHECK = 6         /* a device-side bounds check refused a store (AR_CHECKS) */
 } ar_status;
 
 typedef enum { AR_F32 = 0, AR_BF16 = 1 } ar_dtype;
@@ -179,8 +197,11 @@ size_t ar_tune_workspace_bytes(int64_t out, int64_t in, int64_t n_rows,
  *      0.5, 1) with mlr = minmax_lr (lr if < 0); all from gradients at the same point.
  * Step t uses block perm_e[t mod (n_rows/batch_rows)], perm_e a Fisher-Yates shuffle
  * per epoch driven by one SplitMix64 stream seeded with `seed`.  The contractions
- * run on bf16 tensor cores with fp32 accumulation: W' - W and R are rounded to
- * bf16 before their products.
+ * run on bf16 tensor cores with fp32 accumulation.  With params->split = 1 (the
+ * default) every operand that is not exactly bf16 (D = W' - W, R, the Gram
+ * matrices) is held as an exact bf16 pair hi + lo (about 16 significant bits) and
+ * multiplied as the products hi*hi + lo*hi + hi*lo; with split = 0 it is rounded to
+ * one bf16.
  *   W           [out, in], fp32 or bf16, 16-byte aligned.
  *   X           [n_rows, in] bf16 (uint16 bit patterns), 16-byte aligned.
  *   params      host pointer, see ar_tune_params.
@@ -231,8 +252,9 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
                               uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
                               double* final_mse, void* stream, ar_tune_timing* timing);
 
-/* Workspace of ar_tune_layer_fp_target, in bytes (0 if the arguments are invalid or
- * ask for the direct form).  On top of ar_tune_workspace_bytes' Gram-form layout:
+/* Workspace of ar_tune_layer_fp_target, in bytes (0 if the arguments are invalid,
+ * ask for the direct form, or need more than 64 GiB -- the limit of this mode, which
+ * runs in the Gram form only; ar_tune_layer_fp_target then returns AR_EUNSUPPORTED).  On top of ar_tune_workspace_bytes' Gram-form layout:
  * two copies of one calibration block as a bf16 pair (4 * batch_rows * in * 2
  * bytes), the in x in pair M_b^T, every block's out x in pair C_b
  * (n_rows/batch_rows * out * in * 4 bytes), their fp32 sum, and W as a pair when it
@@ -256,7 +278,9 @@ size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows
  * the step kernel adds C_b to G and the two loss terms to the row loss.
  * final_mse = mean((X W'^T - X_target W^T)^2) over all rows.  Gram form only
  * (params->algo AR_ALGO_AUTO or AR_ALGO_GRAM; AR_ALGO_DIRECT gives
- * AR_EUNSUPPORTED).  X_target NULL: AR_EINVAL.  Otherwise arguments, results and
+ * AR_EUNSUPPORTED), and only for layers whose workspace stays within 64 GiB
+ * (AR_EUNSUPPORTED otherwise: e.g. an 8192 x 29568 layer with 262144 calibration
+ * rows in blocks of 16384 would need about 80 GB).  X_target NULL: AR_EINVAL.  Otherwise arguments, results and
  * errors as ar_tune_layer, with workspace of ar_tune_fp_target_workspace_bytes(). */
 ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
                                   const uint16_t* X, const uint16_t* X_target, int64_t n_rows,
@@ -338,6 +362,10 @@ ar_status ar_silu_mul(const uint16_t* a, const uint16_t* b, int64_t count, uint1
 /* Size of the fixed device scratch array used by ar_tune_layer_static (64 MiB). */
 #define AR_STATIC_SCRATCH_BYTES (64ull << 20)
 
+/* AR_STATIC_SCRATCH_BYTES as the library was built with it (for bindings that do
+ * not read this header).  No GPU needed. */
+size_t ar_static_scratch_bytes(void);
+
 /* ar_tune_layer for callers that cannot allocate device memory at call time --
  * code that runs where cudaMalloc is not allowed or not wanted (inside a region
  * whose memory is owned by another allocator, or a path that must not trigger the
@@ -352,7 +380,12 @@ ar_status ar_silu_mul(const uint16_t* a, const uint16_t* b, int64_t count, uint1
  *   AR_ENOMEM: the layer needs more scratch than AR_STATIC_SCRATCH_BYTES
  *              (ar_tune_workspace_bytes() tells how much it needs); nothing is enqueued.
  * The first call on each device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream capture.
+ * device current) and caches it with the id of the current CUDA context; a later
+ * call that finds another context current (after cudaDeviceReset, say) looks it
+ * up again.  With CUDA's lazy module loading (the default) that first call may
+ * also be what loads the library's device code onto the device, and so what
+ * creates the array: make the first call on each device before any stream
+ * capture and outside any stretch of code that must not allocate.
  * All calls share the one array, and it keeps the last call's contents; every call
  * initialises what it reads.  Calls that overlap on the device (other streams,
  * other threads) race on the array: serialise them.  ar_tune_status() is not
@@ -364,8 +397,28 @@ ar_status ar_tune_layer_static(const void* W, ar_dtype w_dtype, int64_t out, int
 
 /* Device status of the last ar_tune_layer call that used `workspace`: synchronises
  * `stream`, then returns AR_OK, or AR_ETIMEOUT if a kernel's bounded wait ran out
- * (its results are then invalid), or AR_ECUDA if the stream reports an error. */
+ * (its results are then invalid), AR_ECHECK if a bounds check of the AR_CHECKS
+ * mode refused a store (results invalid), or AR_ECUDA if the stream reports an
+ * error.  (The tuning library's replacement for a global last-error query: the
+ * status lives in the call's own workspace, so concurrent calls on different
+ * workspaces never see each other's errors.) */
 ar_status ar_tune_status(const void* workspace, void* stream);
+
+/* Per-row batch losses of the last ar_tune_layer (or ar_tune_layer_timed) call that
+ * used `workspace`, called with the same out, in, n_rows and params: the loss the
+ * keep-best choice compares ("[llm-compressor] AutoRound ...", "on_event with
+ * SEQUENTIAL_EPOCH_END": the step loss total_loss, split by output row).
+ *   row_loss  [iters, out] fp32 out, device or host memory (copied with unified
+ *             addressing): row_loss[t*out + j] = sum over the rows b of step t's
+ *             calibration block of R_bj^2, R = X_b (W' - W)^T at the state before
+ *             step t's update.  Divide by batch_rows for the row's batch MSE.
+ * Asynchronous on `stream`, after the tuning call it reads.  iters == 0, out == 0 or
+ * in == 0: nothing to copy.  AR_EINVAL as ar_tune_layer, or a NULL pointer;
+ * AR_ENOMEM: ws_bytes smaller than ar_tune_workspace_bytes() for these arguments.
+ * (Workspaces of ar_tune_layer_fp_target, ar_tune_layer_host and
+ * ar_tune_layer_static have other layouts and are not read by this call.) */
+ar_status ar_tune_row_losses(const void* workspace, size_t ws_bytes, int64_t out, int64_t in, int64_t n_rows,
+                             const ar_tune_params* params, float* row_loss, void* stream);
 
 /* Test hook for the bounded-wait path: one CTA waits on a barrier that nothing
  * arrives on, gives up after timeout_ns nanoseconds, writes AR_ETIMEOUT into

@@ -20,7 +20,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libar.so")
 
-AR_OK, AR_EINVAL, AR_EUNSUPPORTED, AR_ENOMEM, AR_ECUDA, AR_ETIMEOUT = range(6)
+AR_OK, AR_EINVAL, AR_EUNSUPPORTED, AR_ENOMEM, AR_ECUDA, AR_ETIMEOUT, AR_ECHECK = range(7)
 AR_F32, AR_BF16 = 0, 1
 AR_ALGO_AUTO, AR_ALGO_DIRECT, AR_ALGO_GRAM = 0, 1, 2
 ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
@@ -32,7 +32,7 @@ EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack
            "ar_tune_workspace_bytes", "ar_tune_layer", "ar_tune_layer_timed", "ar_block_schedule",
            "ar_tune_host_workspace_bytes", "ar_tune_layer_host", "ar_tune_fp_target_workspace_bytes",
            "ar_tune_layer_fp_target", "ar_selftest_division",
-           "ar_tune_status", "ar_selftest_timeout", "ar_tune_layer_static", "ar_dequant", "ar_linear",
+           "ar_tune_status", "ar_tune_row_losses", "ar_selftest_timeout", "ar_tune_layer_static", "ar_static_scratch_bytes", "ar_dequant", "ar_linear",
            "ar_silu_mul")
 
 
@@ -101,6 +101,8 @@ def _load() -> ctypes.CDLL:
     lib.ar_tune_layer_static.restype = ctypes.c_int
     lib.ar_tune_layer_static.argtypes = [P, ctypes.c_int, I64, I64, P, I64, ctypes.POINTER(TuneParams),
                                          P, P, P, P, P, P]
+    lib.ar_static_scratch_bytes.restype = SZ
+    lib.ar_static_scratch_bytes.argtypes = []
     lib.ar_dequant.restype = ctypes.c_int
     lib.ar_dequant.argtypes = [P, P, P, I64, I64, I32, P, P, P, P]
     lib.ar_linear.restype = ctypes.c_int
@@ -109,6 +111,8 @@ def _load() -> ctypes.CDLL:
     lib.ar_silu_mul.argtypes = [P, P, I64, P, P]
     lib.ar_tune_status.restype = ctypes.c_int
     lib.ar_tune_status.argtypes = [P, P]
+    lib.ar_tune_row_losses.restype = ctypes.c_int
+    lib.ar_tune_row_losses.argtypes = [P, SZ, I64, I64, I64, ctypes.POINTER(TuneParams), P, P]
     lib.ar_selftest_division.restype = ctypes.c_int
     lib.ar_selftest_division.argtypes = [P, I64, P, I64, P, P, P]
     lib.ar_selftest_timeout.restype = ctypes.c_int
@@ -125,8 +129,8 @@ def version() -> str:
 
 
 def lib_static_scratch_bytes() -> int:
-    """Size of the fixed device scratch of ar_tune_layer_static (AR_STATIC_SCRATCH_BYTES)."""
-    return 64 << 20
+    """Size of the fixed device scratch of ar_tune_layer_static, as the library was built."""
+    return int(_lib.ar_static_scratch_bytes())
 
 
 def _check(status: int, what: str) -> None:
@@ -372,6 +376,16 @@ def tune_layer_fp_target(W: torch.Tensor, X: torch.Tensor, X_target: torch.Tenso
                                         _ptr(codes), _ptr(scale), _ptr(zp), _ptr(trace), _ptr(mse),
                                         _stream(stream)), "ar_tune_layer_fp_target")
     return TuneResult(codes, scale, zp, trace[:params.iters], mse, workspace)
+
+
+def tune_row_losses(workspace: torch.Tensor, out: int, inn: int, n_rows: int, params: TuneParams,
+                    stream=None) -> torch.Tensor:
+    """Per-row batch losses of the last tune_layer call on ``workspace`` (same sizes and
+    params): fp32 [iters, out], the sum over the step's block rows of R_bj^2."""
+    dst = torch.empty((max(params.iters, 1), out), dtype=torch.float32, device=workspace.device)
+    _check(_lib.ar_tune_row_losses(_ptr(workspace), workspace.numel(), out, inn, n_rows, ctypes.byref(params),
+                                   _ptr(dst), _stream(stream)), "ar_tune_row_losses")
+    return dst[:params.iters]
 
 
 def tune_status(workspace: torch.Tensor, stream=None) -> int:

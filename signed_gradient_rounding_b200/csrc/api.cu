@@ -2,6 +2,7 @@
 // schedule and the launch sequence of the tuning loop.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -112,6 +113,26 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 ar_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AR_OK : AR_ECUDA; }
 
+// Test hooks read from the environment on every call (see ar.h):
+//   AR_FAULT=param|alloc|launch|bounds  makes one kind of failure happen on the host;
+//   AR_CHECKS=1                          turns on the device-side bounds checks.
+enum Fault { kFaultNone = 0, kFaultParam, kFaultAlloc, kFaultLaunch, kFaultBounds };
+
+Fault injected_fault() {
+  const char* f = getenv("AR_FAULT");
+  if (!f || !*f) return kFaultNone;
+  if (!strcmp(f, "param")) return kFaultParam;
+  if (!strcmp(f, "alloc")) return kFaultAlloc;
+  if (!strcmp(f, "launch")) return kFaultLaunch;
+  if (!strcmp(f, "bounds")) return kFaultBounds;
+  return kFaultNone;
+}
+
+bool checks_on() {
+  const char* c = getenv("AR_CHECKS");
+  return c && *c && strcmp(c, "0") != 0;
+}
+
 #define AR_CUDA_TRY(expr)                   \
   do {                                      \
     cudaError_t e_ = (expr);                \
@@ -131,6 +152,7 @@ bool tune_shape_supported(int64_t in, int64_t g, int64_t B) {
 bool wide_groups(int64_t in, int64_t g) { return !((256 % g == 0) || (g == in && in <= 256)); }
 
 ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune_params* p) {
+  if (injected_fault() == kFaultParam) return AR_EINVAL;
   if (!p || out < 0 || in < 0 || n_rows < 0) return AR_EINVAL;
   if (!bits_ok(p->bits)) return AR_EINVAL;
   if (p->iters < 0 || !(p->lr >= 0.0f) || !isfinite(p->lr) || !isfinite(p->minmax_lr)) return AR_EINVAL;
@@ -186,9 +208,24 @@ struct Plan {
   // 4096-wide layer, 3-10% slower (more energy per step at the power cap) on the
   // 29568-wide one, which is where the automatic choice picks the direct form.
   bool pair_direct = false;
+  // Gram matrices summed over chunks of at most gram_chunk calibration rows, one
+  // launch per chunk, in an fp32 running sum (round to nearest): no tensor-core
+  // accumulation runs over more than gram_chunk rows.  The tensor cores' fp32
+  // accumulation loses low bits on each of its additions; over a whole 16384-row
+  // block that shrank every entry of H_b by about 6e-5 (relative), enough to turn
+  // gradient signs that sit within about 1e-5 of their rms.
+  int64_t gram_chunk = 2048;
+  int64_t gram_nchunk = 1;
 };
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
+// The full-precision-target mode runs in the Gram form only: on top of the Gram
+// matrices it keeps every block's C_b = W M_b as a bf16 pair (n_rows/batch_rows *
+// out * in * 4 bytes).  A layer whose workspace would exceed this is refused
+// (AR_EUNSUPPORTED), as the automatic choice refuses Gram matrices above
+// kGramMaxBytes: the 8192 x 29568 down_proj of a Qwen2.5-72B-shaped block with
+// 16 blocks of 16384 rows would need about 80 GB.
+constexpr size_t kFpTargetMaxBytes = 64ull << 30;
 
 Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool fp_target = false,
                bool w_f32 = false) {
@@ -221,6 +258,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   P.bn_upd = 256;
   P.bn_gram = 256;
   P.bn_fin = 256;
+  P.gram_nchunk = P.algo == AR_ALGO_GRAM ? std::max<int64_t>(1, cdiv(P.B, P.gram_chunk)) : 1;
   P.wide = wide_groups(in, P.g);
   P.gslots = P.wide ? static_cast<int>(cdiv(P.g, kSegCols) + 1) : 0;
   // Row partial sums: kEpiHalves per n-tile (one per epilogue column half).
@@ -233,7 +271,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
   size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1,
-      wmin, wmax, part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
+      wmin, wmax, part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum, Hacc,
       // full-precision-target mode: this block's dX = X - X_target (pair),
       // M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b (pair), their sum Cs
       // (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the partials of e_b, and W as
@@ -284,6 +322,7 @@ Layout make_layout(const Plan& P) {
     L.Hs_lo = P.split ? take(h) : L.Hs_hi;
     L.Hdiag = take(static_cast<size_t>(P.nb) * P.in * 4);
     L.Hdsum = take(static_cast<size_t>(P.in) * 4);
+    L.Hacc = P.gram_nchunk > 1 ? take(static_cast<size_t>(P.in) * P.in * 4) : 0;
     if (P.fp_target) {
       const size_t blk = static_cast<size_t>(P.B) * P.in * 2;
       L.dX_hi = take(blk);
@@ -368,10 +407,13 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   const Plan P = make_plan(out, in, n_rows, p, X_target != nullptr, w_dtype == AR_F32);
   if (P.fp_target && P.algo != AR_ALGO_GRAM) return AR_EUNSUPPORTED;
   const Layout L = make_layout(P);
-  if (ws_bytes < L.total) return AR_ENOMEM;
+  if (P.fp_target && L.total > kFpTargetMaxBytes) return AR_EUNSUPPORTED;
+  const Fault fault = injected_fault();
+  if (ws_bytes < L.total || fault == kFaultAlloc) return AR_ENOMEM;
   const bool gram = P.algo == AR_ALGO_GRAM;
   const int64_t B = P.B;
   const int iters = p->iters;
+  const bool checks = checks_on();
 
   int dev = 0, sms = 0, major = 0;
   AR_CUDA_TRY(cudaGetDevice(&dev));
@@ -487,6 +529,11 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   prep.D_hi = D_hi;
   prep.D_lo = P.split ? D_lo : nullptr;
   prep.div_slow = div_slow;
+  if (checks) {
+    prep.chk_elems = static_cast<int64_t>(elems);
+    prep.chk_groups = static_cast<int64_t>(groups);
+    prep.status = status;
+  }
   AR_CUDA_TRY(launch_group_quant(prep, st));
   ++launches;
 
@@ -516,6 +563,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     h.C_lo = P.split ? H(L.H_lo) : nullptr;
     h.ldc = in;
     h.diag_out = F(L.Hdiag);
+    h.C_acc = P.gram_nchunk > 1 ? F(L.Hacc) : nullptr;
+    if (checks) h.chk_c = P.nb * in * in;
   }
   // Full-precision-target mode, per block b (dX_b = X_b - X_target,b):
   //   M_b^T = X_b^T dX_b          [in, in]   (pair; A = X_b^T, B = dX_b^T pair)
@@ -599,13 +648,27 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     have_block[b] = 1;
     cudaError_t e = wait_block(b);
     if (e != cudaSuccess || !gram) return e;
-    e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);
-    if (e != cudaSuccess) return e;
-    gram_maps.a1 = gram_maps.b0 = gram_maps.b1 = gram_maps.a0;
+    // H_b over chunks of rows of block b (each chunk's map ends at the chunk, so
+    // its last K tile reads zeros past it), summed in fp32.
+    const int64_t chunk = round_up(static_cast<size_t>(cdiv(B, P.gram_nchunk)), 8);
     h.c_row_off = b * in;
-    ++launches;
-    e = launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
-    if (e != cudaSuccess || !fpt) return e;
+    for (int64_t r0 = 0; r0 < B; r0 += chunk) {
+      const int64_t rows = std::min(chunk, B - r0);
+      GemmMaps cm{};
+      e = make_tmap_bf16(&cm.a0, X + (b * B + r0) * in, rows, in, 64);
+      if (e != cudaSuccess) return e;
+      cm.a1 = cm.b0 = cm.b1 = cm.a0;
+      h.K = static_cast<int>(rows);
+      h.num_k_blk = static_cast<int>(cdiv(rows, kBK));
+      h.acc_first = r0 == 0;
+      h.acc_last = r0 + rows >= B;
+      ++launches;
+      e = launch_gemm(kEpiStore, P.bn_gram, cm, h, sms, st);
+      if (e != cudaSuccess) return e;
+    }
+    if (!fpt) return cudaSuccess;
+    e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);  // the whole block, for M_b
+    if (e != cudaSuccess) return e;
     return fp_target_block(b);
   };
 
@@ -633,6 +696,12 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.mlr = mlr;
   u.gpart = P.wide ? F(L.gpart) : nullptr;
   u.gslots = P.gslots;
+  if (checks) {
+    // AR_FAULT=bounds: the epilogue is told V and D hold one element fewer than
+    // they do, so the last chunk's stores are refused (and reported), not made.
+    u.chk_elems = static_cast<int64_t>(elems) - (fault == kFaultBounds ? 1 : 0);
+    u.chk_groups = static_cast<int64_t>(groups);
+  }
   // Wide groups: the group updates and the next D after each step launch.
   auto finish_groups = [&]() -> cudaError_t {
     if (!P.wide) return cudaSuccess;
@@ -665,6 +734,9 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     f.bits = u.bits;
     f.sym = u.sym;
     f.mlr = u.mlr;
+    f.chk_elems = u.chk_elems;
+    f.chk_groups = u.chk_groups;
+    f.status = status;
     ++launches;
     return launch_group_finish(f, st);
   };
@@ -721,6 +793,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
         u.e_row = F(L.e) + sched[t] * out;
       }
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
+      if (fault == kFaultLaunch) return AR_ECUDA;
       AR_CUDA_TRY(launch_gemm(upd_kind, P.bn_upd, m[cur], u, sms, st));
       AR_CUDA_TRY(finish_groups());
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
@@ -778,6 +851,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     r.ldc = B;
     r.part = part[0];
     r.part_ld = static_cast<int>(P.nparts_res);
+    if (checks) r.chk_c = out * B;
 
     fill_grid(u, out, in, B, P.bn_upd, nseg_d, P.pair_direct);  // update: G = (R_hi + R_lo)^T X_b
     u.raster_m = P.raster_upd;
@@ -799,6 +873,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       r.b_row_off = static_cast<int>(b0);
       AR_CUDA_TRY(ensure_block(sched[t]));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
+      if (fault == kFaultLaunch) return AR_ECUDA;
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
       AR_CUDA_TRY(make_tmap_bf16(&mu.b0, X + b0 * in, B, in, 64));
@@ -848,6 +923,11 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   fin.zp = zp;
   fin.D_hi = final_mse ? D_hi : nullptr;
   fin.D_lo = final_mse && P.split ? D_lo : nullptr;
+  if (checks) {
+    fin.chk_elems = static_cast<int64_t>(elems);
+    fin.chk_groups = static_cast<int64_t>(groups);
+    fin.status = status;
+  }
   AR_CUDA_TRY(launch_group_quant(fin, st));
   ++launches;
 
@@ -927,6 +1007,8 @@ const char* ar_status_string(ar_status s) {
       return "AR_ECUDA: CUDA error";
     case AR_ETIMEOUT:
       return "AR_ETIMEOUT: device wait timed out";
+    case AR_ECHECK:
+      return "AR_ECHECK: a device-side bounds check refused a store (AR_CHECKS)";
   }
   return "unknown ar_status";
 }
@@ -940,6 +1022,7 @@ ar_status ar_rtn(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, int32
 ar_status ar_fake_quant(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const float* V,
                         const float* alpha, const float* beta, int32_t bits, int32_t group_size, int32_t sym,
                         uint8_t* codes, float* scale, int32_t* zp, float* Wq, void* stream) {
+  if (injected_fault() == kFaultParam) return AR_EINVAL;
   if (!bits_ok(bits) || out < 0 || in < 0) return AR_EINVAL;
   if (w_dtype != AR_F32 && w_dtype != AR_BF16) return AR_EINVAL;
   if (out == 0 || in == 0) return AR_OK;
@@ -965,6 +1048,7 @@ ar_status ar_fake_quant(const void* W, ar_dtype w_dtype, int64_t out, int64_t in
 }
 
 ar_status ar_pack(const uint8_t* codes, int64_t rows, int64_t cols, int32_t bits, int32_t* packed, void* stream) {
+  if (injected_fault() == kFaultParam) return AR_EINVAL;
   if (!bits_ok(bits) || rows < 0 || cols < 0) return AR_EINVAL;
   if ((cols * bits) % 32 != 0) return AR_EINVAL;
   if (rows == 0 || cols == 0) return AR_OK;
@@ -1120,6 +1204,7 @@ ar_status ar_tune_layer_host(const void* W_host, ar_dtype w_dtype, int64_t out, 
   const size_t block_bytes = static_cast<size_t>(B) * in * 2;
   uint16_t* Xd = reinterpret_cast<uint16_t*>(ws + HL.X);
 
+  if (injected_fault() == kFaultAlloc) return AR_ENOMEM;
   CopyPipeline cp;
   if (!cp.create(static_cast<size_t>(nb))) return AR_ECUDA;
   // Copies start after the work already queued on the caller's stream; blocks go
@@ -1172,7 +1257,8 @@ size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows
   if (out == 0 || in == 0) return 256;
   const Plan P = make_plan(out, in, n_rows, p, true, w_dtype == AR_F32);
   if (P.algo != AR_ALGO_GRAM) return 0;
-  return make_layout(P).total;
+  const size_t total = make_layout(P).total;
+  return total > kFpTargetMaxBytes ? 0 : total;
 }
 
 ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
@@ -1195,7 +1281,21 @@ ar_status ar_tune_status(const void* workspace, void* stream) {
   if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return AR_ECUDA;
   if (word == kDevOk) return AR_OK;
   if (word == kDevTimeout) return AR_ETIMEOUT;
+  if (word == kDevCheck) return AR_ECHECK;
   return AR_ECUDA;
+}
+
+ar_status ar_tune_row_losses(const void* workspace, size_t ws_bytes, int64_t out, int64_t in, int64_t n_rows,
+                             const ar_tune_params* p, float* row_loss, void* stream) {
+  const ar_status chk = check_tune_args(out, in, n_rows, p);
+  if (chk != AR_OK) return chk;
+  if (out == 0 || in == 0 || p->iters == 0) return AR_OK;
+  if (!workspace || !row_loss) return AR_EINVAL;
+  const Layout L = make_layout(make_plan(out, in, n_rows, p));
+  if (ws_bytes < L.total) return AR_ENOMEM;
+  const size_t bytes = static_cast<size_t>(out) * static_cast<size_t>(p->iters) * sizeof(float);
+  return from_cuda(cudaMemcpyAsync(row_loss, static_cast<const uint8_t*>(workspace) + L.rowloss, bytes,
+                                   cudaMemcpyDefault, static_cast<cudaStream_t>(stream)));
 }
 
 ar_status ar_selftest_division(const float* a, int64_t na, const float* b, int64_t nb, uint64_t* mismatches,
@@ -1270,13 +1370,49 @@ ar_status ar_silu_mul(const uint16_t* a, const uint16_t* b, int64_t count, uint1
 // library's device code is loaded on a GPU and held until the process exits.  In
 // host code `g_static_scratch` names a host-side stand-in, not the device array,
 // so its device address is looked up (cudaGetSymbolAddress) once per device, with
-// that device current, on the first call there, and cached.
+// that device current, on the first call there, and cached together with the id
+// of the CUDA context it belongs to.  A call that finds another context current
+// (after cudaDeviceReset, or a context the caller pushed) looks it up again.
 // ---------------------------------------------------------------------------
 
 static __device__ __align__(256) uint8_t g_static_scratch[AR_STATIC_SCRATCH_BYTES];
 
-static std::mutex g_static_mu;
-static void* g_static_ptr[256];
+namespace {
+
+struct StaticScratch {
+  void* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+
+std::mutex g_static_mu;
+StaticScratch g_static[256];
+
+// Id of the current CUDA context (driver entry points fetched through the runtime,
+// as for the tensor maps).  False if there is none or the driver lacks the call.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t ar_static_scratch_bytes(void) { return AR_STATIC_SCRATCH_BYTES; }
 
 ar_status ar_tune_layer_static(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
                                int64_t n_rows, const ar_tune_params* p, uint8_t* codes, float* scale, int32_t* zp,
@@ -1290,12 +1426,22 @@ ar_status ar_tune_layer_static(const void* W, ar_dtype w_dtype, int64_t out, int
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_ptr[dev]) {
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx);
+    StaticScratch& e = g_static[dev];
+    if (!e.ptr || !have_ctx || e.ctx_id != ctx) {
       void* ptr = nullptr;
       if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return AR_ECUDA;
-      g_static_ptr[dev] = ptr;
+      // The lookup makes the device's context current if none was; without a
+      // context id the address is looked up on every call.
+      unsigned long long now = 0;
+      const bool have_now = current_context_id(&now);
+      e.ptr = have_now ? ptr : nullptr;
+      e.ctx_id = now;
+      scratch = ptr;
+    } else {
+      scratch = e.ptr;
     }
-    scratch = g_static_ptr[dev];
   }
   return tune_impl(W, w_dtype, out, in, X, n_rows, p, nullptr, scratch, AR_STATIC_SCRATCH_BYTES, codes, scale, zp,
                    loss_trace, final_mse, stream, nullptr);

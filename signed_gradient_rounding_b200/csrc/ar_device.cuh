@@ -187,7 +187,17 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_
 }
 
 // Device status words (first int of the workspace).
-enum : int { kDevOk = 0, kDevTimeout = 5 };
+enum : int { kDevOk = 0, kDevTimeout = 5, kDevCheck = 6 };
+
+// Bounds check of the AR_CHECKS mode: true if [idx, idx + n) lies inside a buffer
+// of cap elements, or if checks are off (cap == 0).  Otherwise records kDevCheck
+// in *status (the first error recorded stays) and returns false: the caller skips
+// the access.  Never traps.
+__device__ __forceinline__ bool in_bounds(int64_t idx, int n, int64_t cap, int* status) {
+  if (cap == 0 || (idx >= 0 && idx + n <= cap)) return true;
+  if (status) atomicCAS(status, kDevOk, kDevCheck);
+  return false;
+}
 
 // Wait until the phase with the given parity of `bar` has completed.  Gives up
 // after timeout_ns (checked every few hundred polls), or as soon as another role

@@ -31,6 +31,10 @@ struct GroupQuantArgs {
   __nv_bfloat16* D_lo = nullptr;   // ... and lo = bf16(D - hi) (may be null)
   int* div_slow = nullptr;         // when set: +1 for every group that has a weight
                                    // that is not div_fast_ok (W/s must use __fdiv_rn)
+  // AR_CHECKS: capacities (elements) of the [out, in] and [out, G] outputs; a store
+  // outside them is skipped and recorded in *status.  0: no checks.
+  int64_t chk_elems = 0, chk_groups = 0;
+  int* status = nullptr;
 };
 
 cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream);
@@ -163,6 +167,14 @@ struct GemmArgs {
   // kEpiStore: when set, the diagonal (column == row j) is written here in fp32,
   // at [c_row_off + j], and stored as 0 in the bf16 pair
   float* diag_out = nullptr;
+  // kEpiStore of a product summed over consecutive chunks of K, one launch per
+  // chunk (a Gram matrix over sub-blocks of its calibration block, so that no
+  // tensor-core accumulation runs over more than one chunk): when set, the tile is
+  // added, one fp32 round-to-nearest addition per element, to the running sum
+  // [*, ldc] here (acc_first: the sum starts with this chunk); only the last chunk
+  // (acc_last) goes on to the diagonal, the row sums and the bf16 pair store.
+  float* C_acc = nullptr;
+  int acc_first = 1, acc_last = 1;
   // kEpiUpdate / kEpiDotD: when set, C_jk += D_jk * diag_in[k] in fp32 (the exact
   // diagonal of a Gram matrix whose bf16 pair holds only the off-diagonal part)
   const float* diag_in = nullptr;
@@ -211,6 +223,11 @@ struct GemmArgs {
   // floor(gg * g / 128) + k.
   float* gpart = nullptr;
   int gslots = 0;
+  // AR_CHECKS: capacities (elements) of the buffers the epilogues store to -- C_hi
+  // and C_lo (chk_c), the [M, N] state V_out, V_best, D (chk_elems), the [M, G]
+  // clip factors (chk_groups).  A store outside them is skipped and recorded in
+  // *status (kDevCheck).  0: no checks.
+  int64_t chk_c = 0, chk_elems = 0, chk_groups = 0;
 };
 
 // After a wide-group step launch: per (row, group), d alpha and d beta as the sum
@@ -242,6 +259,8 @@ struct GroupFinishArgs {
   const int* div_slow = nullptr;
   int bits = 4, sym = 0;
   float mlr = 0.f;
+  int64_t chk_elems = 0, chk_groups = 0;  // AR_CHECKS, as in GemmArgs
+  int* status = nullptr;
 };
 cudaError_t launch_group_finish(const GroupFinishArgs& a, cudaStream_t stream);
 

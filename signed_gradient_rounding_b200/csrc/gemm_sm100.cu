@@ -279,6 +279,26 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
     float x[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+    if (kKind == kEpiStore && a.C_acc) {
+      float4* pa = reinterpret_cast<float4*>(a.C_acc + static_cast<int64_t>(j) * a.ldc + col0);
+      if (!a.acc_first) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q * 4 < nvalid) {
+            const float4 s4 = pa[q];
+            x[q * 4 + 0] = __fadd_rn(s4.x, x[q * 4 + 0]);
+            x[q * 4 + 1] = __fadd_rn(s4.y, x[q * 4 + 1]);
+            x[q * 4 + 2] = __fadd_rn(s4.z, x[q * 4 + 2]);
+            x[q * 4 + 3] = __fadd_rn(s4.w, x[q * 4 + 3]);
+          }
+      }
+      if (!a.acc_last) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q * 4 < nvalid) pa[q] = make_float4(x[q * 4 + 0], x[q * 4 + 1], x[q * 4 + 2], x[q * 4 + 3]);
+        continue;
+      }
+    }
     if (kKind == kEpiStore || kKind == kEpiSumSq) {
 #pragma unroll
       for (int i = 0; i < 32; ++i)
@@ -318,6 +338,7 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
     }
     if (kKind == kEpiStore) {
       const int64_t off = (a.c_row_off + j) * a.ldc + col0;
+      if (!in_bounds(off, nvalid, a.chk_c, a.status)) continue;
       if (a.C_add) {
         float ad[32];
         load_bf16x32(a.C_add + off, ad);
@@ -354,6 +375,7 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
             float h, l;
             split_bf16(x[i], h, l);
             const int64_t mo = (a.c_row_off + col) * a.ldc + j;
+            if (!in_bounds(mo, 1, a.chk_c, a.status)) continue;
             a.C_hi[mo] = __float2bfloat16_rn(h);
             if (a.C_lo) a.C_lo[mo] = __float2bfloat16_rn(l);
           }
@@ -527,7 +549,8 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       tmem_ld_16cols(t_row + (col - n0), r);
       tmem_ld_wait();
       if (!row_ok) continue;  // nothing warp-collective follows in this iteration
-      if (snap_old) {
+      const bool e_ok = in_bounds(e0, kUC, a.chk_elems, a.status);
+      if (snap_old && e_ok) {
         float vo[kUC];
         load_f32x16(a.V_out + e0, vo);
         store_f32x16(a.V_best + e0, vo);
@@ -537,23 +560,25 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       for (int i = 0; i < kUC; ++i)
         vn[i] = sign_step_elem<kFp>(a, w[i], v[i], __uint_as_float(r[i]), dg[i], kFp ? cv[i] : 0.0f, gs, gd, Q, fast,
                                     loss_acc, dal, dbe);
-      store_f32x16(a.V_out + e0, vn);
-      if (snap_now) store_f32x16(a.V_best + e0, v);
+      if (e_ok) store_f32x16(a.V_out + e0, vn);
+      if (snap_now && e_ok) store_f32x16(a.V_best + e0, v);
     }
     if (!row_ok) continue;
 
     const float al_n = clip_step(al, a.mlr, dal);
     const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
-    if (snap_now) {
-      a.alpha_best[gidx] = al;
-      a.beta_best[gidx] = be;
+    if (in_bounds(gidx, 1, a.chk_groups, a.status)) {
+      if (snap_now) {
+        a.alpha_best[gidx] = al;
+        a.beta_best[gidx] = be;
+      }
+      if (snap_old) {
+        a.alpha_best[gidx] = a.alpha_out[gidx];
+        a.beta_best[gidx] = a.beta_out[gidx];
+      }
+      a.alpha_out[gidx] = al_n;
+      a.beta_out[gidx] = be_n;
     }
-    if (snap_old) {
-      a.alpha_best[gidx] = a.alpha_out[gidx];
-      a.beta_best[gidx] = a.beta_out[gidx];
-    }
-    a.alpha_out[gidx] = al_n;
-    a.beta_out[gidx] = be_n;
 
     // Pass 2: D = W' - W of the next step, from the updated state, as a bf16 pair
     // (the values were written by this thread in pass 1).
@@ -575,6 +600,7 @@ __device__ __forceinline__ void epi_update(const GemmArgs& a, uint32_t t_row, in
       }
 #pragma unroll
       for (int i = 0; i < kUC; ++i) d[i] = __fsub_rn(quant_elem(w[i], v[i], gn, Q, fast).wq, w[i]);
+      if (!in_bounds(e0, kUC, a.chk_elems, a.status)) continue;
 #pragma unroll
       for (int q = 0; q < kUC / 8; ++q)
         store_pair8(d + q * 8, a.D_hi + e0 + q * 8, a.D_lo ? a.D_lo + e0 + q * 8 : nullptr);
@@ -653,7 +679,8 @@ __device__ __forceinline__ void epi_update_wide(const GemmArgs& a, uint32_t t_ro
     tmem_ld_16cols(t_row + (col - n0), r);
     tmem_ld_wait();
     if (!row_ok) continue;  // nothing warp-collective follows in this iteration
-    if (snap_old) {
+    const bool e_ok = in_bounds(e0, kUC, a.chk_elems, a.status);
+    if (snap_old && e_ok) {
       float vo[kUC];
       load_f32x16(a.V_out + e0, vo);
       store_f32x16(a.V_best + e0, vo);
@@ -663,8 +690,8 @@ __device__ __forceinline__ void epi_update_wide(const GemmArgs& a, uint32_t t_ro
     for (int i = 0; i < kUC; ++i)
       vn[i] = sign_step_elem<kFp>(a, w[i], v[i], __uint_as_float(r[i]), dg[i], kFp ? cv[i] : 0.0f, gs, gd, Q, fast,
                                   loss_acc, dal, dbe);
-    store_f32x16(a.V_out + e0, vn);
-    if (snap_now) store_f32x16(a.V_best + e0, v);
+    if (e_ok) store_f32x16(a.V_out + e0, vn);
+    if (snap_now && e_ok) store_f32x16(a.V_best + e0, v);
   }
   if (cur >= 0 && row_ok) flush();
   if (kFp && row_ok && a.e_row && n_blk == 0 && half == 0) loss_acc += a.e_row[j];

@@ -50,7 +50,7 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
   const float alpha = a.alpha ? a.alpha[warp] : 1.0f;
   const float beta = a.beta ? a.beta[warp] : 1.0f;
   const GroupScale gs = group_scale(wmin, wmax, alpha, beta, a.bits, a.sym != 0);
-  if (lane == 0) {
+  if (lane == 0 && in_bounds(warp, 1, a.chk_groups, a.status)) {
     if (a.wmin_out) {
       a.wmin_out[warp] = wmin;
       a.wmax_out[warp] = wmax;
@@ -64,6 +64,7 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
     const float w = load_w(a.W, a.w_bf16, base + k);
     const float v = a.V ? a.V[base + k] : 0.0f;
     const ElemQuant e = quant_elem(w, v, gs, Q, fast);
+    if (!in_bounds(base + k, 1, a.chk_elems, a.status)) continue;
     if (a.codes) a.codes[base + k] = static_cast<uint8_t>(e.q);
     if (a.Wq) a.Wq[base + k] = e.wq;
     if (a.D_hi) {
@@ -313,7 +314,7 @@ __global__ void group_finish_kernel(GroupFinishArgs a) {
   const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
   const bool better = a.judged && a.keep_best && a.best_out[j] < a.best_in[j];
   __syncwarp();  // every lane has read alpha_in, beta_in (they may alias the outputs)
-  if (lane == 0) {
+  if (lane == 0 && in_bounds(grp, 1, a.chk_groups, a.status)) {
     if (better && !a.snap_prev) {
       a.alpha_best[grp] = al;
       a.beta_best[grp] = be;
@@ -366,6 +367,7 @@ __global__ void group_finish_kernel(GroupFinishArgs a) {
       hi2[h] = *reinterpret_cast<const uint32_t*>(&hp);
       lo2[h] = *reinterpret_cast<const uint32_t*>(&lp);
     }
+    if (!in_bounds(e, 8, a.chk_elems, a.status)) continue;
     *reinterpret_cast<uint4*>(a.D_hi + e) = make_uint4(hi2[0], hi2[1], hi2[2], hi2[3]);
     if (a.D_lo) *reinterpret_cast<uint4*>(a.D_lo + e) = make_uint4(lo2[0], lo2[1], lo2[2], lo2[3]);
   }
