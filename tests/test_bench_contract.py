@@ -29,6 +29,12 @@ def test_reference_arm_line():
     assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["data"] == "synthetic" and d["config"]["workload"].startswith("tiny")
+    # the same config, key for key, as the GPU arm states for this workload
+    sys.path.insert(0, ROOT)
+    import bench
+    assert d["config"] == json.loads(json.dumps(bench._config(bench.WORKLOADS["tiny"], 1)))
+    for key in ("lr", "minmax_lr", "keep_best", "batch_rows", "iters", "bits", "group_size", "sym"):
+        assert key in d["config"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e2e = d["e2e"]

@@ -7,6 +7,7 @@ import torch
 
 import oracle
 from oracle import autoround as oar
+from tests.free_running import code_bound, oracle_drift
 from workloads import bf16_from_bits, make_activations, make_weight
 
 pytestmark = pytest.mark.gpu
@@ -132,7 +133,8 @@ def test_block_7b_full_size_sampled_rows(ar):
     """The LLaMA-7B decoder block at full size (262144 calibration rows, W3 g128 sym,
     200 steps per layer), as the benchmark runs it; per layer the oracle replays 16
     sampled rows on the GPU's own input bytes.  Full-size trajectories are chaotic
-    (see test_gpu_parity), so the bars are the MSE (2%) and a loose code bound."""
+    (see test_gpu_parity), so the bars are the MSE (2%) and twice the oracle's drift
+    against its own jittered run (tests/free_running.py)."""
     from signed_gradient_rounding_b200.block import tune_block
     from workloads import BLOCK_7B, BLOCK_7B_LAYERS, make_activations_cuda
     c = BLOCK_7B
@@ -162,6 +164,8 @@ def test_block_7b_full_size_sampled_rows(ar):
         mse_gpu = oar.layer_mse(Ws[name][rows], wq, X[:16384])
         mse_ref = oar.layer_mse(Ws[name][rows], ref.Wq, X[:16384])
         frac = float(np.mean(codes != ref.codes))
-        print(f"block {name}: {frac:.3%} codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
+        drift = oracle_drift(ref, Ws[name][rows], X, c.bits, c.group_size, True, c.iters, c.lr, -1.0, c.batch_rows)
+        print(f"block {name}: {frac:.3%} codes differ (oracle against its jittered self: {drift:.3%}), "
+              f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
         assert mse_gpu == pytest.approx(mse_ref, rel=0.02), name
-        assert frac <= 0.20, name
+        assert frac <= code_bound(drift), name

@@ -15,6 +15,7 @@ import torch
 
 import oracle
 from oracle import autoround as oar
+from tests.free_running import code_bound, oracle_drift
 from workloads import (DOWN_7B, DOWN_72B, Q_PROJ_7B, TINY, bf16_round, make_activations,
                        make_activations_cuda, make_weight)
 
@@ -22,13 +23,12 @@ pytestmark = pytest.mark.gpu
 
 CODE_TOL = 0.005      # fraction of codes allowed to differ after tuning
 MSE_RTOL = 0.02       # relative tolerance of the final layer MSE
-# Full-size runs (200 minibatch steps): the SignSGD iteration is chaotic.  In the
-# oracle alone, resolving ONE gradient-sign tie per row the other way at step 20
-# leaves 2.6% of the final codes different (keep-best; 13% for the last iterate).
-# The GPU resolves a handful of ties per step differently (|G| < 1e-6 of its rms,
-# see test_one_step_signs), so at full size the code agreement is a sanity bound
-# only; the stated bars there are the MSE and the per-step sign parity.
-CHAOS_CODE_BOUND = 0.20
+# Full-size runs (200 minibatch steps): the SignSGD iteration is chaotic, and a
+# tie resolved the other way forks it.  The stated 0.5% of codes holds on the
+# small and full-batch cases below; at full size the per-step parity is checked
+# step-locked (test_gpu_steplocked.py) and the free-running drift is held to
+# twice the drift of the oracle against itself with its gradients jittered within
+# the tie band (tests/free_running.py), and is printed with its decomposition.
 
 
 @pytest.fixture(scope="module")
@@ -304,6 +304,31 @@ def test_rejects_unsupported(ar):
     assert e.value.status in (ar.AR_EUNSUPPORTED, ar.AR_EINVAL)
 
 
+def _divergence(ar, res, c, rows, ref, params):
+    """Decompose the free-running code divergence of a full-size run (printed):
+    the rows whose applied best step differs from the oracle's, the codes that
+    differ on the rows that kept the same step, and the step at which each row's
+    batch loss first leaves the oracle's by more than 1e-5 (the trajectory fork)."""
+    L = _np(ar.tune_row_losses(res.workspace, c.out, c.inn, c.n_rows, params))[:, rows]     # sums of R^2
+    inv_b = np.float32(1.0) / np.float32(c.batch_rows)
+    means = L.astype(np.float32) * inv_b
+    gpu_best = np.argmin(means, axis=0)            # first minimum: the strict "<" of keep-best
+    same = gpu_best == ref.best_step
+    codes = _np(res.codes)[rows]
+    diff = codes != ref.codes
+    rel = np.abs(L.astype(np.float64) / c.batch_rows - ref.row_loss_trace) / ref.row_loss_trace
+    off = rel > 1e-5
+    fork = np.where(off.any(axis=0), np.argmax(off, axis=0), c.iters)
+    info = dict(rows_best_differs=float(np.mean(~same)),
+                codes_differ_same_best=float(diff[same].mean()) if same.any() else 0.0,
+                codes_differ_other_best=float(diff[~same].mean()) if (~same).any() else 0.0,
+                fork_step_median=float(np.median(fork)), rows_never_forked=float(np.mean(fork == c.iters)),
+                groups_differ=float(np.mean((_np(res.scale)[rows] != ref.scale) |
+                                            (_np(res.zero_point)[rows] != ref.zero_point))))
+    print(f"    divergence: {info}")
+    return info
+
+
 def _full_size_case(c, n_sample):
     """A full-size workload on the device and the oracle replaying sampled rows."""
     W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
@@ -312,15 +337,17 @@ def _full_size_case(c, n_sample):
     Xh = _x_bits(Xd)
     ref = oracle.tune_layer(W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr,
                             c.batch_rows, 0, want_final_mse=False)
-    return c, W, Xd, Xh, rows, ref
+    drift = oracle_drift(ref, W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr, c.batch_rows)
+    return c, W, Xd, Xh, rows, ref, drift
 
 
 def _check_full_size(ar, case, algo, mse_rows=65536):
-    c, W, Xd, Xh, rows, ref = case
+    c, W, Xd, Xh, rows, ref, drift = case
     p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
                        batch_rows=c.batch_rows, seed=0, algo=algo)
     res = ar.tune_layer(_w_dev(W, "bf16"), Xd, p, want_final_mse=False)
     assert ar.tune_status(res.workspace) == ar.AR_OK
+    _divergence(ar, res, c, rows, ref, p)
     del res.workspace
     codes = _np(res.codes)[rows]
     frac = float(np.mean(codes != ref.codes))
@@ -331,9 +358,10 @@ def _check_full_size(ar, case, algo, mse_rows=65536):
     Wq_gpu = np.repeat(s, g, 1) * (codes.astype(np.float32) - np.repeat(z, g, 1))
     mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:mse_rows])
     mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:mse_rows])
-    print(f"{c.name} {algo}: {frac:.3%} of sampled codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
+    print(f"{c.name} {algo}: {frac:.3%} of sampled codes differ (oracle against its jittered self: {drift:.3%}), "
+          f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
     assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert frac <= CHAOS_CODE_BOUND, f"{frac:.4%} of sampled codes differ"
+    assert frac <= code_bound(drift), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
     _, _, _, Wrtn = oracle.rtn(W[rows], c.bits, c.group_size, c.sym)
     assert mse_gpu < oar.layer_mse(W[rows], Wrtn, Xh[:mse_rows])
 
@@ -371,7 +399,8 @@ def q_proj_case():
     Xh = _x_bits(Xd)
     ref = oracle.tune_layer(W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr,
                             c.batch_rows, 0)
-    return c, W, Xd, Xh, rows, ref
+    drift = oracle_drift(ref, W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr, c.batch_rows)
+    return c, W, Xd, Xh, rows, ref, drift
 
 
 @pytest.mark.parametrize("algo", ALGOS)
@@ -380,11 +409,12 @@ def test_q_proj_full_size_sampled_rows(ar, q_proj_case, algo):
     activations, 16384 rows per step, 200 steps), run as the benchmark runs it.
     Rows tune independently, so the oracle replays 64 sampled rows exactly on the
     full activations; the sampled rows' codes and MSE are compared."""
-    c, W, Xd, Xh, rows, ref = q_proj_case
+    c, W, Xd, Xh, rows, ref, drift = q_proj_case
     p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
                        batch_rows=c.batch_rows, seed=0, algo=algo)
     res = ar.tune_layer(_w_dev(W, "bf16"), Xd, p)
     assert ar.tune_status(res.workspace) == ar.AR_OK
+    _divergence(ar, res, c, rows, ref, p)
     codes = _np(res.codes)[rows]
     frac = float(np.mean(codes != ref.codes))
     # MSE of the GPU's sampled rows, evaluated by the oracle's own fp64 loss
@@ -393,8 +423,34 @@ def test_q_proj_full_size_sampled_rows(ar, q_proj_case, algo):
     Wq_gpu = np.repeat(s, c.group_size, 1) * (codes.astype(np.float32) - np.repeat(z, c.group_size, 1))
     mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:65536])
     mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:65536])
-    print(f"q_proj {algo}: {frac:.3%} of sampled codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
+    print(f"q_proj {algo}: {frac:.3%} of sampled codes differ (oracle against its jittered self: {drift:.3%}), "
+          f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
     assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert frac <= CHAOS_CODE_BOUND, f"{frac:.4%} of sampled codes differ"
+    assert frac <= code_bound(drift), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
+    # scales and zero-points: the groups whose clip factors ended elsewhere
+    groups = float(np.mean((_np(res.scale)[rows] != ref.scale) | (_np(res.zero_point)[rows] != ref.zero_point)))
+    print(f"    groups with a differing scale or zero-point: {groups:.3%}")
     _, _, _, Wrtn = oracle.rtn(W[rows], c.bits, c.group_size, c.sym)
     assert mse_gpu < oar.layer_mse(W[rows], Wrtn, Xh[:65536])
+
+
+def test_q_proj_full_size_last_iterate(ar, q_proj_case):
+    """keep_best = 0: the page's own loop, which applies the last iterate ("최종 양자화
+    적용" in "[llm-compressor] AutoRound ..."), on the full-size q_proj (Gram form, as
+    the benchmark runs): the final layer MSE within 2% of the oracle's last iterate."""
+    c, W, Xd, Xh, rows, _, _ = q_proj_case
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
+                       batch_rows=c.batch_rows, seed=0, keep_best=False, algo="gram")
+    res = ar.tune_layer(_w_dev(W, "bf16"), Xd, p, want_final_mse=False)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W[rows], Xh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr, c.batch_rows, 0,
+                            keep_best=False, want_final_mse=False)
+    codes = _np(res.codes)[rows]
+    frac = float(np.mean(codes != ref.codes))
+    s = _np(res.scale)[rows]
+    z = _np(res.zero_point)[rows].astype(np.float32)
+    Wq_gpu = np.repeat(s, c.group_size, 1) * (codes.astype(np.float32) - np.repeat(z, c.group_size, 1))
+    mse_gpu = oar.layer_mse(W[rows], Wq_gpu, Xh[:65536])
+    mse_ref = oar.layer_mse(W[rows], ref.Wq, Xh[:65536])
+    print(f"q_proj last iterate: {frac:.3%} of sampled codes differ, mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
+    assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)

@@ -9,8 +9,10 @@ test first.
 
 The check: through the C ABI, two calls in a row of the static entry point give
 exactly the outputs of ar_tune_layer with a caller-allocated workspace (the same
-kernels on the same inputs are deterministic, so the tolerance is zero), and a
-layer needing more scratch than the array holds is refused before any work.
+kernels on the same inputs are deterministic, so the tolerance is zero), the
+second call leaves the device's free memory and torch's allocated bytes as the
+first left them, and a layer needing more scratch than the array holds is
+refused before any work.
 """
 import ctypes
 
@@ -30,21 +32,27 @@ def ar():
     return ar
 
 
-def _static_call(ar, Wd, Xd, p):
-    out, inn = Wd.shape
+def _outputs(out, inn, p):
     G = inn // p.group_size
-    codes = torch.full((out, inn), 255, dtype=torch.uint8, device="cuda")
-    scale = torch.full((out, G), -1.0, dtype=torch.float32, device="cuda")
-    zp = torch.full((out, G), -1, dtype=torch.int32, device="cuda")
-    trace = torch.full((p.iters,), -1.0, dtype=torch.float32, device="cuda")
-    mse = torch.full((1,), -1.0, dtype=torch.float64, device="cuda")
+    return (torch.full((out, inn), 255, dtype=torch.uint8, device="cuda"),
+            torch.full((out, G), -1.0, dtype=torch.float32, device="cuda"),
+            torch.full((out, G), -1, dtype=torch.int32, device="cuda"),
+            torch.full((p.iters,), -1.0, dtype=torch.float32, device="cuda"),
+            torch.full((1,), -1.0, dtype=torch.float64, device="cuda"))
+
+
+def _static_call(ar, Wd, Xd, p, outs):
+    """One call of the static entry point into preallocated outputs; returns the
+    device's free memory (cudaMemGetInfo) and torch's allocated bytes afterwards."""
+    out, inn = Wd.shape
+    codes, scale, zp, trace, mse = outs
     st = ar.lib.ar_tune_layer_static(ar._ptr(Wd), ar.AR_F32 if Wd.dtype == torch.float32 else ar.AR_BF16,
                                      out, inn, ar._ptr(Xd), Xd.shape[0], ctypes.byref(p), ar._ptr(codes),
                                      ar._ptr(scale), ar._ptr(zp), ar._ptr(trace), ar._ptr(mse),
                                      ar._stream(None))
     assert st == ar.AR_OK, ar.lib.ar_status_string(st)
     torch.cuda.synchronize()
-    return codes, scale, zp, trace, mse
+    return torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
 
 
 @pytest.mark.parametrize("algo", ["gram", "direct"])
@@ -59,13 +67,19 @@ def test_static_scratch_matches_workspace_entry_point(ar, algo):
     assert ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p) <= ar.lib_static_scratch_bytes()
     ref = ar.tune_layer(Wd, Xd, p)
     torch.cuda.synchronize()
-    for _ in range(2):  # two calls in a row: the array keeps the previous call's contents
-        codes, scale, zp, trace, mse = _static_call(ar, Wd, Xd, p)
+    outs = [_outputs(c.out, c.inn, p) for _ in range(2)]
+    # two calls in a row: the array keeps the previous call's contents
+    mem = [_static_call(ar, Wd, Xd, p, o) for o in outs]
+    for o in outs:
+        codes, scale, zp, trace, mse = o
         assert torch.equal(codes, ref.codes)
         assert torch.equal(scale, ref.scale)
         assert torch.equal(zp, ref.zero_point)
         assert torch.equal(trace, ref.loss_trace)
         assert torch.equal(mse, ref.final_mse)
+    # The second call allocated nothing: the device's free memory and torch's
+    # allocated bytes are what the first call left (its outputs were made before).
+    assert mem[1] == mem[0]
 
 
 def test_static_scratch_refuses_oversized_layer(ar):
