@@ -11,10 +11,11 @@ epilogues per step, the final codes and the final MSE pass, and packing.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload q_proj|tiny|down_7b|down_72b]
 
-Prints one JSON line (rank 0).  Metric: SignSGD steps per second (whole job:
-every rank tunes its own 4096-row shard of a layer, no collective on the data
-path, so the scaling is weak), plus the layer tune time and the fraction of
-the bf16 tensor-core peak.  ``--impl reference`` times the CPU oracle on a
+Prints one JSON line (rank 0).  Metric: SignSGD steps per second (whole job).
+With N GPUs the layer has N times the workload's output rows; each rank tunes
+its row shard (shard.row_range) with no exchange in the loop and one all-gather
+of the results per step, so the scaling is weak.  Also the layer tune time and
+the fraction of the bf16 tensor-core peak.  ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload on the host cores.
 """
 from __future__ import annotations
@@ -307,28 +308,43 @@ def run_ours(args):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from signed_gradient_rounding_b200.shard import row_range, tune_layer_sharded
+
     c = _workload(args)
-    # Each rank tunes its own shard of output rows (weak scaling): rank r's rows
-    # are drawn with seed r; the calibration activations are the same on every rank.
-    W = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=rank))
-    Wd = (W.to(torch.bfloat16) if c.w_dtype == "bf16" else W).to(dev)
+    # One layer of out * world rows (weak scaling): rank r tunes its row_range shard
+    # (out rows) on the same calibration activations and block schedule, with no
+    # exchange during the loop; one all-gather of codes, scales and zero-points
+    # over NCCL ends each step.  At world = 1 this is the workload's own layer.
+    out_all = c.out * world
+    a, b = row_range(out_all, rank, world)
+    W_all = torch.from_numpy(make_weight(out_all, c.inn, c.w_std, c.w_dtype, seed=0))
+    W = W_all[a:b].contiguous()
+    Wd_all = (W_all.to(torch.bfloat16) if c.w_dtype == "bf16" else W_all).to(dev)
+    del W_all
     Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
     p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
                        minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
                        split=bool(args.split))
-    ws = torch.empty(ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
+    rows = b - a
+    ws = torch.empty(ar.tune_workspace_bytes(rows, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
     G = c.inn // (c.inn if c.group_size == -1 else c.group_size)
-    outs = (torch.empty((c.out, c.inn), dtype=torch.uint8, device=dev),
-            torch.empty((c.out, G), dtype=torch.float32, device=dev),
-            torch.empty((c.out, G), dtype=torch.int32, device=dev),
+    outs = (torch.empty((rows, c.inn), dtype=torch.uint8, device=dev),
+            torch.empty((rows, G), dtype=torch.float32, device=dev),
+            torch.empty((rows, G), dtype=torch.int32, device=dev),
             torch.empty((c.iters,), dtype=torch.float32, device=dev),
             torch.empty((1,), dtype=torch.float64, device=dev))
     stream = torch.cuda.current_stream(dev)
+    timing_slot = [None]
+
+    def compute(W_shard, X):
+        res = ar.tune_layer(W_shard, X, p, workspace=ws, outputs=outs, timing=timing_slot[0])
+        return res.codes, res.scale, res.zero_point
 
     def one_step(timing=None):
-        res = ar.tune_layer(Wd, Xd, p, workspace=ws, outputs=outs, timing=timing)
-        packed = ar.pack(res.codes, c.bits)
-        return res, packed
+        timing_slot[0] = timing
+        (codes, scale, zp), _ = tune_layer_sharded(Wd_all, Xd, compute)
+        packed = ar.pack(codes, c.bits)
+        return packed
 
     for _ in range(args.warmup):
         one_step()
@@ -361,13 +377,14 @@ def run_ours(args):
     ms_max = float(ms_t.item())
 
     # End to end through the host API: pinned host inputs copied in and the
-    # results copied out inside the timed region, every step.
+    # results copied out inside the timed region, every step (this rank's shard).
     e2e = None
     if args.e2e_steps > 0:
+        del Wd_all
         Wh = W.to(torch.bfloat16 if c.w_dtype == "bf16" else torch.float32).pin_memory()
         Xh = Xd.cpu().pin_memory()
         h2d = Wh.numel() * Wh.element_size() + Xh.numel() * Xh.element_size()
-        d2h = c.out * c.inn + 2 * c.out * G * 4 + c.iters * 4 + 8
+        d2h = rows * c.inn + 2 * rows * G * 4 + c.iters * 4 + 8
         del Xd
         torch.cuda.empty_cache()
         ar.tune_layer_host(Wh, Xh, p, device=dev)          # warm
@@ -421,6 +438,7 @@ def run_ours(args):
     step_ms = res_ms + upd_ms
     step_tflops = (flops_res + flops_upd) / (step_ms * 1e-3) / 1e12
     launches = sum(t.kernel_launches for t in timings) + args.steps    # + one pack per step
+    config = _config(c, world)
     line = {
         "metric": METRIC,
         "value": world * c.iters * args.steps / (ms_max / 1e3),
@@ -434,13 +452,9 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": c.name, "out": c.out, "in": c.inn, "n_rows": c.n_rows,
-                   "batch_rows": c.batch_rows, "iters": c.iters, "bits": c.bits, "group_size": c.group_size,
-                   "sym": c.sym, "lr": c.lr, "minmax_lr": c.minmax_lr, "keep_best": True, "algo": algo,
-                   "bench_step": "one ar_tune_layer call (all iters) + ar_pack",
-                   "l2": "inputs larger than L2: X is %.1f GB, one step reads a %.0f MB block"
-                         % (c.n_rows * c.inn * 2 / 1e9, c.batch_rows * c.inn * 2 / 1e6),
-                   "parallelism": f"row shards x{world}, no data-path collective"},
+        "config": config,
+        "bench_step": "one ar_tune_layer call (all iters) on this rank's row shard, the all-gather of "
+                      "codes/scales/zero-points (N > 1), and ar_pack",
         "layer_tune_s": layer_s,
         "algo": algo,
         "split_operands": bool(args.split),
@@ -464,6 +478,17 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(c, Xd if args.e2e_steps == 0 else None, args.cpu_rows, args.cpu_steps)
     return line
+
+
+def _config(c, world: int) -> dict:
+    """The workload as both arms state it (the same keys and values in each)."""
+    return {"workload": c.name if world == 1 else f"{c.name}, {c.out * world} output rows in {world} row shards",
+            "out": c.out * world, "in": c.inn, "n_rows": c.n_rows, "batch_rows": c.batch_rows, "iters": c.iters,
+            "bits": c.bits, "group_size": c.group_size, "sym": c.sym, "lr": c.lr, "minmax_lr": c.minmax_lr,
+            "keep_best": True, "seed": 0,
+            "l2": "inputs larger than L2: X is %.1f GB, one step reads a %.0f MB block"
+                  % (c.n_rows * c.inn * 2 / 1e9, c.batch_rows * c.inn * 2 / 1e6),
+            "parallelism": f"row shards x{world}; one all-gather of the results per step, none in the loop"}
 
 
 def _threads():
@@ -546,9 +571,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": c.name, "out": c.out, "in": c.inn, "n_rows": c.n_rows,
-                       "batch_rows": c.batch_rows, "iters": c.iters, "bits": c.bits,
-                       "group_size": c.group_size, "sym": c.sym},
+            "config": _config(c, world),
+            "bench_step": f"oracle.tune_layer on {len(sel)} sampled output rows x {args.cpu_steps} SignSGD steps",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": _threads(), "kind": "oracle",
                              "sample": f"each step: {len(sel)} of {c.out} output rows x {args.cpu_steps} "
                                        f"SignSGD steps; rate scaled by rows/out",
