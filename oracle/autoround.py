@@ -279,7 +279,7 @@ class Step:
 
 
 def sign_step(W, Xb, V, alpha, beta, wmin, wmax, group_size: int, bits: int, sym: bool, lr: float,
-              minmax_lr: float, Xt_b=None, with_scale: bool = False) -> Step:
+              minmax_lr: float, Xt_b=None, with_scale: bool = False, jitter=None) -> Step:
     """One step of the per-layer loop ("[llm-compressor] AutoRound ...", "on_event with
     SEQUENTIAL_EPOCH_END": fake-quantise, forward, MSE, backward, sign update).
 
@@ -289,6 +289,8 @@ def sign_step(W, Xb, V, alpha, beta, wmin, wmax, group_size: int, bits: int, sym
     straight-through gradients, then V <- clamp(V - lr*sign(dL/dV), -0.5, 0.5) and
     alpha, beta <- clamp(. - minmax_lr*sign(.), 0.5, 1), all from the same point.
     ``with_scale`` also fills dalpha_abs and dbeta_abs (otherwise None).
+    ``jitter`` (sensitivity studies only, never parity): a callable applied to G
+    before the sign decisions, see ``tune_layer(grad_jitter=...)``.
     """
     W = _to_f32(W)
     g = _group(W.shape[1], group_size)
@@ -302,6 +304,8 @@ def sign_step(W, Xb, V, alpha, beta, wmin, wmax, group_size: int, bits: int, sym
         R = Xb @ Wq.astype(F64).T - Xt_b @ W.astype(F64).T
     row_loss = np.sum(R * R, axis=0) / Xb.shape[0]
     G = R.T @ Xb                                          # dL/dW' * (B*out/2)  [out, in]
+    if jitter is not None:
+        G = jitter(G)
     if with_scale:
         sgn_dV, dalpha, dbeta, abs_a, abs_b = step_gradients(W, V, alpha, beta, wmin, wmax, G, g, bits, sym,
                                                              with_scale=True)
@@ -338,7 +342,8 @@ class TuneResult:
 def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
                minmax_lr: float, batch_rows: int, seed: int, minmax_shrink: float = 1.0,
                keep_best: bool = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
-               best0=None, want_final_mse: bool = True, init: str = "minmax", X_target=None) -> TuneResult:
+               best0=None, want_final_mse: bool = True, init: str = "minmax", X_target=None,
+               grad_jitter=None) -> TuneResult:
     """SignSGD tuning of one linear layer.
 
     "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END": per step,
@@ -378,6 +383,13 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     captured full-precision output ``y_true``.  With X_target the batch residual
     is Y' - Y = X_b W'^T - X_target,b W^T, written out as those two products;
     without it Y = X_b W^T (the layer's own input on both sides).
+
+    ``grad_jitter = (rel, seed)`` is not part of the method: it adds to every
+    gradient G, before its sign is taken, seeded uniform noise in
+    [-rel, rel] * rms(G).  That models an implementation whose gradients are exact
+    only up to rel of their rms, so the loop's own drift from such an
+    implementation can be measured (ties resolved the other way fork the SignSGD
+    trajectory).  None (the default) is the method.
     """
     W = _to_f32(W)
     out, inn = W.shape
@@ -412,13 +424,21 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     trace = np.zeros(iters, dtype=F64)
     row_trace = np.zeros((iters, out), dtype=F64)
     best_step = np.full(out, -1, dtype=np.int64)
+    jitter = None
+    if grad_jitter is not None:
+        rel, jseed = grad_jitter
+        jrng = np.random.default_rng(jseed)
+
+        def jitter(G):
+            rms = float(np.sqrt(np.mean(G * G)))
+            return G + jrng.uniform(-1.0, 1.0, G.shape) * (rel * rms)
     for t in range(iters):
         blk = sched[t]
         if blk not in cache:
             cache[blk] = _rows_f64(X, blk * batch_rows, (blk + 1) * batch_rows)
         Xb = cache[blk]
         Xt_b = None if X_target is None else _rows_f64(X_target, blk * batch_rows, (blk + 1) * batch_rows)
-        st = sign_step(W, Xb, V, alpha, beta, wmin, wmax, g, bits, sym, lr32, mlr32, Xt_b)
+        st = sign_step(W, Xb, V, alpha, beta, wmin, wmax, g, bits, sym, lr32, mlr32, Xt_b, jitter=jitter)
         row_loss = st.row_loss
         row_trace[t] = row_loss
         trace[t] = float(np.sum(row_loss)) / out
