@@ -589,7 +589,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q_proj")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-rows", type=int, default=64)
-    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--cpu-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--algo", choices=["auto", "direct", "gram"], default="auto")
     ap.add_argument("--split", type=int, default=1, help="1: bf16-pair operands (default); 0: single bf16")
