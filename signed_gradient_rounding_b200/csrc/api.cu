@@ -208,14 +208,13 @@ struct Plan {
   // 4096-wide layer, 3-10% slower (more energy per step at the power cap) on the
   // 29568-wide one, which is where the automatic choice picks the direct form.
   bool pair_direct = false;
-  // Gram matrices summed over chunks of at most gram_chunk calibration rows, one
-  // launch per chunk, in an fp32 running sum (round to nearest): no tensor-core
-  // accumulation runs over more than gram_chunk rows.  The tensor cores' fp32
-  // accumulation loses low bits on each of its additions; over a whole 16384-row
-  // block that shrank every entry of H_b by about 6e-5 (relative), enough to turn
-  // gradient signs that sit within about 1e-5 of their rms.
+  // Gram matrices summed over chunks of gram_chunk calibration rows (GemmArgs::
+  // k_chunk): each chunk is its own tensor-core accumulation, and the epilogue adds
+  // the chunks in fp32 (round to nearest).  The tensor cores' fp32 accumulation
+  // loses low bits on each of its additions; over a whole 16384-row block that
+  // shrank every entry of H_b by about 6e-5 (relative), enough to turn gradient
+  // signs that sit within about 1e-5 of their rms.
   int64_t gram_chunk = 2048;
-  int64_t gram_nchunk = 1;
 };
 
 constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
@@ -258,7 +257,6 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   P.bn_upd = 256;
   P.bn_gram = 256;
   P.bn_fin = 256;
-  P.gram_nchunk = P.algo == AR_ALGO_GRAM ? std::max<int64_t>(1, cdiv(P.B, P.gram_chunk)) : 1;
   P.wide = wide_groups(in, P.g);
   P.gslots = P.wide ? static_cast<int>(cdiv(P.g, kSegCols) + 1) : 0;
   // Row partial sums: kEpiHalves per n-tile (one per epilogue column half).
@@ -271,7 +269,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
 // Workspace layout (offsets in bytes from the workspace base).
 struct Layout {
   size_t status, D_hi, D_lo, D_hi1, D_lo1, V0, V1, a0, a1, b0, b1, V_best, alpha_best, beta_best, best0, best1,
-      wmin, wmax, part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum, Hacc,
+      wmin, wmax, part0, part1, rowloss, gpart, Rt_hi, Rt_lo, H_hi, H_lo, Hs_hi, Hs_lo, Hdiag, Hdsum,
       // full-precision-target mode: this block's dX = X - X_target (pair),
       // M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b (pair), their sum Cs
       // (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the partials of e_b, and W as
@@ -322,7 +320,6 @@ Layout make_layout(const Plan& P) {
     L.Hs_lo = P.split ? take(h) : L.Hs_hi;
     L.Hdiag = take(static_cast<size_t>(P.nb) * P.in * 4);
     L.Hdsum = take(static_cast<size_t>(P.in) * 4);
-    L.Hacc = P.gram_nchunk > 1 ? take(static_cast<size_t>(P.in) * P.in * 4) : 0;
     if (P.fp_target) {
       const size_t blk = static_cast<size_t>(P.B) * P.in * 2;
       L.dX_hi = take(blk);
@@ -563,7 +560,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     h.C_lo = P.split ? H(L.H_lo) : nullptr;
     h.ldc = in;
     h.diag_out = F(L.Hdiag);
-    h.C_acc = P.gram_nchunk > 1 ? F(L.Hacc) : nullptr;
+    h.k_chunk = static_cast<int>(P.gram_chunk / kBK);
     if (checks) h.chk_c = P.nb * in * in;
   }
   // Full-precision-target mode, per block b (dX_b = X_b - X_target,b):
@@ -648,27 +645,14 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     have_block[b] = 1;
     cudaError_t e = wait_block(b);
     if (e != cudaSuccess || !gram) return e;
-    // H_b over chunks of rows of block b (each chunk's map ends at the chunk, so
-    // its last K tile reads zeros past it), summed in fp32.
-    const int64_t chunk = round_up(static_cast<size_t>(cdiv(B, P.gram_nchunk)), 8);
-    h.c_row_off = b * in;
-    for (int64_t r0 = 0; r0 < B; r0 += chunk) {
-      const int64_t rows = std::min(chunk, B - r0);
-      GemmMaps cm{};
-      e = make_tmap_bf16(&cm.a0, X + (b * B + r0) * in, rows, in, 64);
-      if (e != cudaSuccess) return e;
-      cm.a1 = cm.b0 = cm.b1 = cm.a0;
-      h.K = static_cast<int>(rows);
-      h.num_k_blk = static_cast<int>(cdiv(rows, kBK));
-      h.acc_first = r0 == 0;
-      h.acc_last = r0 + rows >= B;
-      ++launches;
-      e = launch_gemm(kEpiStore, P.bn_gram, cm, h, sms, st);
-      if (e != cudaSuccess) return e;
-    }
-    if (!fpt) return cudaSuccess;
-    e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);  // the whole block, for M_b
+    e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);
     if (e != cudaSuccess) return e;
+    gram_maps.a1 = gram_maps.b0 = gram_maps.b1 = gram_maps.a0;
+    h.c_row_off = b * in;
+    ++launches;
+    e = launch_gemm(kEpiStore, P.bn_gram, gram_maps, h, sms, st);
+    if (e != cudaSuccess) return e;
+    if (!fpt) return cudaSuccess;
     return fp_target_block(b);
   };
 

@@ -167,14 +167,12 @@ struct GemmArgs {
   // kEpiStore: when set, the diagonal (column == row j) is written here in fp32,
   // at [c_row_off + j], and stored as 0 in the bf16 pair
   float* diag_out = nullptr;
-  // kEpiStore of a product summed over consecutive chunks of K, one launch per
-  // chunk (a Gram matrix over sub-blocks of its calibration block, so that no
-  // tensor-core accumulation runs over more than one chunk): when set, the tile is
-  // added, one fp32 round-to-nearest addition per element, to the running sum
-  // [*, ldc] here (acc_first: the sum starts with this chunk); only the last chunk
-  // (acc_last) goes on to the diagonal, the row sums and the bf16 pair store.
-  float* C_acc = nullptr;
-  int acc_first = 1, acc_last = 1;
+  // kEpiStore of a symmetric MN-major product on pair tiles (the Gram matrices):
+  // K is summed in chunks of k_chunk K blocks, each a separate accumulation in
+  // tensor memory handed to the epilogue, which adds it to the tile's running sums
+  // in fp32 (round to nearest) in registers, so no tensor-core accumulation runs
+  // over more than one chunk.  0: one accumulation over the whole K.
+  int k_chunk = 0;
   // kEpiUpdate / kEpiDotD: when set, C_jk += D_jk * diag_in[k] in fp32 (the exact
   // diagonal of a Gram matrix whose bf16 pair holds only the off-diagonal part)
   const float* diag_in = nullptr;

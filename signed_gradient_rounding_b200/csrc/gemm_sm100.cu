@@ -260,6 +260,64 @@ __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, i
 // epilogues
 // ---------------------------------------------------------------------------
 
+// kEpiStore: 32 consecutive columns col0.. of row j (nvalid of them in range): the
+// diagonal element into diag_out (stored as 0 in the pair), C_add, and the bf16 pair
+// store (a symmetric C writes its upper elements in place and the strictly upper ones
+// again transposed, so every element is written once).
+__device__ __forceinline__ void store_cols32(const GemmArgs& a, int j, int col0, int nvalid, float (&x)[32]) {
+  if (a.diag_out && j >= col0 && j < col0 + 32) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col0 + i == j) {
+        a.diag_out[a.c_row_off + j] = x[i];
+        x[i] = 0.0f;
+      }
+  }
+  const int64_t off = (a.c_row_off + j) * a.ldc + col0;
+  if (!in_bounds(off, nvalid, a.chk_c, a.status)) return;
+  if (a.C_add) {
+    float ad[32];
+    load_bf16x32(a.C_add + off, ad);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] += ad[i];
+  }
+  if (!a.symmetric) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
+    return;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c8 = col0 + q * 8;
+    if (q * 8 >= nvalid || c8 + 7 < j) continue;
+    if (c8 >= j) {
+      store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c8 + i >= j) {
+          float h, l;
+          split_bf16(x[q * 8 + i], h, l);
+          a.C_hi[off + q * 8 + i] = __float2bfloat16_rn(h);
+          if (a.C_lo) a.C_lo[off + q * 8 + i] = __float2bfloat16_rn(l);
+        }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int col = col0 + i;
+    if (i < nvalid && col > j) {
+      float h, l;
+      split_bf16(x[i], h, l);
+      const int64_t mo = (a.c_row_off + col) * a.ldc + j;
+      if (!in_bounds(mo, 1, a.chk_c, a.status)) continue;
+      a.C_hi[mo] = __float2bfloat16_rn(h);
+      if (a.C_lo) a.C_lo[mo] = __float2bfloat16_rn(l);
+    }
+  }
+}
+
 // kEpiStore / kEpiSumSq / kEpiDotD: one pass over the tile's columns.
 template <int kKind, int kBN>
 __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int j, int n0, int n_blk, int half) {
@@ -279,26 +337,6 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
     float x[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
-    if (kKind == kEpiStore && a.C_acc) {
-      float4* pa = reinterpret_cast<float4*>(a.C_acc + static_cast<int64_t>(j) * a.ldc + col0);
-      if (!a.acc_first) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q * 4 < nvalid) {
-            const float4 s4 = pa[q];
-            x[q * 4 + 0] = __fadd_rn(s4.x, x[q * 4 + 0]);
-            x[q * 4 + 1] = __fadd_rn(s4.y, x[q * 4 + 1]);
-            x[q * 4 + 2] = __fadd_rn(s4.z, x[q * 4 + 2]);
-            x[q * 4 + 3] = __fadd_rn(s4.w, x[q * 4 + 3]);
-          }
-      }
-      if (!a.acc_last) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q * 4 < nvalid) pa[q] = make_float4(x[q * 4 + 0], x[q * 4 + 1], x[q * 4 + 2], x[q * 4 + 3]);
-        continue;
-      }
-    }
     if (kKind == kEpiStore || kKind == kEpiSumSq) {
 #pragma unroll
       for (int i = 0; i < 32; ++i)
@@ -328,60 +366,7 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc = fmaf(dh[i], x[i], acc);
     }
-    if (kKind == kEpiStore && a.diag_out && j >= col0 && j < col0 + 32) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col0 + i == j) {
-          a.diag_out[a.c_row_off + j] = x[i];
-          x[i] = 0.0f;
-        }
-    }
-    if (kKind == kEpiStore) {
-      const int64_t off = (a.c_row_off + j) * a.ldc + col0;
-      if (!in_bounds(off, nvalid, a.chk_c, a.status)) continue;
-      if (a.C_add) {
-        float ad[32];
-        load_bf16x32(a.C_add + off, ad);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] += ad[i];
-      }
-      if (!a.symmetric) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q * 8 < nvalid) store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
-      } else {
-        // upper elements (col >= row) in place, strictly upper ones also at [col, row]
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c8 = col0 + q * 8;
-          if (q * 8 >= nvalid || c8 + 7 < j) continue;
-          if (c8 >= j) {
-            store_pair8(x + q * 8, a.C_hi + off + q * 8, a.C_lo ? a.C_lo + off + q * 8 : nullptr);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              if (c8 + i >= j) {
-                float h, l;
-                split_bf16(x[q * 8 + i], h, l);
-                a.C_hi[off + q * 8 + i] = __float2bfloat16_rn(h);
-                if (a.C_lo) a.C_lo[off + q * 8 + i] = __float2bfloat16_rn(l);
-              }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = col0 + i;
-          if (i < nvalid && col > j) {
-            float h, l;
-            split_bf16(x[i], h, l);
-            const int64_t mo = (a.c_row_off + col) * a.ldc + j;
-            if (!in_bounds(mo, 1, a.chk_c, a.status)) continue;
-            a.C_hi[mo] = __float2bfloat16_rn(h);
-            if (a.C_lo) a.C_lo[mo] = __float2bfloat16_rn(l);
-          }
-        }
-      }
-    }
+    if (kKind == kEpiStore) store_cols32(a, j, col0, nvalid, x);
   }
   if (kKind == kEpiDotD && row_ok && a.e_row && n_blk == 0 && half == 0) acc += a.e_row[j];
   if (row_ok && a.part) a.part[static_cast<int64_t>(j) * a.part_ld + n_blk * kEpiHalves + half] = acc;
@@ -744,6 +729,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ GemmArgs args) {
   using C = Cfg<kBN, kPair, kNA, kNB>;
   constexpr bool kFused = C::kFused;
+  // The Gram-matrix instance can sum K in chunks (GemmArgs::k_chunk): the MMAs of
+  // each chunk accumulate afresh in accumulator 1, and the epilogue adds each chunk,
+  // in fp32 round to nearest, to the tile's running sum kept in accumulator 0.
+  constexpr bool kChunkable = kKind == kEpiStore && kPair && kNA == 0 && kNB == 0 && kMaj == 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
@@ -795,6 +784,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // kFused: one stage per K block carries every segment; otherwise one per
   // (segment, K block), segments outermost.
   const int k_blocks = kFused ? args.num_k_blk : args.num_seg * args.num_k_blk;
+  // K blocks per accumulator hand-off: the whole tile, or one chunk.
+  const bool chunked = kChunkable && args.k_chunk > 0 && args.k_chunk < k_blocks;
+  const int k_chunk = chunked ? args.k_chunk : k_blocks;
   // kFused: which of the two maps of A and of B the segments use.
   bool use_a1 = false, use_b1 = false;
   for (int s = 0; s < args.num_seg; ++s) {
@@ -880,15 +872,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      uint32_t chunk_phase = 0;  // chunked: phase of accumulator 1, the only one the MMAs use
       bool ok = true;
       for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
-        if (!mbar_wait<kPair>(&sm->tempty[acc], acc_phase ^ 1, abort_flag, args.status, args.timeout_ns)) {
+       for (int kb0 = 0; ok && kb0 < k_blocks; kb0 += k_chunk) {
+        const int buf = chunked ? 1 : acc;
+        if (!mbar_wait<kPair>(&sm->tempty[buf], (chunked ? chunk_phase : acc_phase) ^ 1, abort_flag, args.status,
+                              args.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kBN;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        const uint32_t d_tmem = tmem_base + buf * kBN;
+        const int kb1 = min(k_blocks, kb0 + k_chunk);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait<kPair>(&sm->full[stage], phase, abort_flag, args.status, args.timeout_ns)) {
             ok = false;
             break;
@@ -903,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   operand_desc(a_addr + ((kNB == 2 && args.seg_b[s]) ? C::kOffB1 : C::kOffB0), kBMn);
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k) {
-                const uint32_t accum = (kb | s | k) != 0 ? 1u : 0u;
+                const uint32_t accum = ((kb - kb0) | s | k) != 0 ? 1u : 0u;
                 if (kPair)
                   umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
                 else
@@ -915,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b_desc = operand_desc(a_addr + kTileABytes, kBMn);
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k) {
-              const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+              const uint32_t accum = ((kb - kb0) | k) != 0 ? 1u : 0u;
               if (kPair)
                 umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
               else
@@ -933,11 +930,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (kPair)
-          umma_commit_pair_both(&sm->tfull[acc]);
+          umma_commit_pair_both(&sm->tfull[buf]);
         else
-          umma_commit(&sm->tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+          umma_commit(&sm->tfull[buf]);
+        if (chunked) {
+          chunk_phase ^= 1;
+        } else {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1;
+        }
+       }
       }
       // Every MMA this thread issued has completed once `drain` flips.
       if (kPair)
@@ -956,6 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t leader_tempty1 = kPair ? mapa_shared(smem_u32(&sm->tempty[1]), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t chunk_phase = 0;  // chunked: phase of accumulator 1
     for (int tile = unit0; tile < args.num_tiles; tile += unit_stride) {
       int m_blk, n_blk;
       tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
@@ -963,6 +966,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = n_blk * kBN;
       if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN, false>(args, j, n0, half);
       if (kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide) epi_update_prefetch<kBN, true>(args, j, n0, half);
+      if constexpr (kChunkable) {
+        if (chunked) {
+          // Each chunk: accumulator 1 (the chunk) added into accumulator 0 (the
+          // running sum) in fp32, then accumulator 1 released; after the last one the
+          // sum is stored.  A warp touches only its own lanes and columns of both.
+          const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+          const uint32_t t_sum = tmem_base + lanes + half * (kBN / kEpiHalves);
+          const uint32_t t_chunk = t_sum + kBN;
+          bool ok = true;
+          for (int kb0 = 0; kb0 < k_blocks; kb0 += k_chunk) {
+            if (!mbar_wait<kPair>(&sm->tfull[1], chunk_phase, abort_flag, args.status, args.timeout_ns, false)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int g = 0; g < kBN / kEpiHalves / 32; ++g) {
+              uint32_t r[32];
+              __syncwarp();
+              tmem_ld_32cols(t_chunk + g * 32, r);
+              tmem_ld_wait();
+              if (kb0 > 0) {
+                uint32_t q[32];
+                tmem_ld_32cols(t_sum + g * 32, q);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__fadd_rn(__uint_as_float(q[i]), __uint_as_float(r[i])));
+              }
+              tmem_st_32cols(t_sum + g * 32, r);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty1);
+            chunk_phase ^= 1;
+          }
+          if (!ok) break;
+          // the tile's sum, from accumulator 0
+#pragma unroll 1
+          for (int g = 0; g < kBN / kEpiHalves / 32; ++g) {
+            uint32_t r[32];
+            __syncwarp();
+            tmem_ld_32cols(t_sum + g * 32, r);
+            tmem_ld_wait();
+            const int col0 = n0 + half * (kBN / kEpiHalves) + g * 32;
+            if (j >= args.M || col0 >= args.N) continue;  // nothing warp-collective follows
+            float x[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+            store_cols32(args, j, col0, min(32, args.N - col0), x);
+          }
+          continue;
+        }
+      }
       // No early exit on another role's abort: every epilogue warp of the CTA takes
       // the same decision here (the phase completes for all of them, or for none).
       if (!mbar_wait<kPair>(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns, false)) break;

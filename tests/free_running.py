@@ -8,8 +8,11 @@ oracle's except where |G| is within TIE_BAND of its rms.  How far two runs that
 differ only there drift apart is a property of the loop itself; it is measured
 here with the oracle alone, by running it once more with every gradient jittered
 by seeded uniform noise of TIE_BAND * rms(G) (oracle.tune_layer's grad_jitter),
-and the GPU's free-running drift must stay within MARGIN times that (and is
-never held to less than the stated 0.5%).
+and the GPU's free-running drift must stay within MARGIN times that, plus the
+granularity of the row sample: a row whose best step (keep-best) differs from the
+oracle's differs in 20-45% of its codes (measured), so one such row among n
+sampled rows moves the fraction by about ROW_GRANULE / n.  The bound is never
+below the stated 0.5%.
 """
 import numpy as np
 
@@ -18,6 +21,7 @@ import oracle
 CODE_TOL = 0.005   # the stated bar: at most 0.5% of the codes differ
 TIE_BAND = 1e-5    # the tie band of the step-locked checks (fraction of rms(G))
 MARGIN = 2.0
+ROW_GRANULE = 0.5  # about half of one sampled row's codes
 
 
 def oracle_drift(ref, W_rows, X, bits, group_size, sym, iters, lr, minmax_lr, batch_rows, seed=0, **kw):
@@ -27,5 +31,6 @@ def oracle_drift(ref, W_rows, X, bits, group_size, sym, iters, lr, minmax_lr, ba
     return float(np.mean(jit.codes != ref.codes))
 
 
-def code_bound(drift: float) -> float:
-    return max(CODE_TOL, MARGIN * drift)
+def code_bound(drift: float, n_rows: int) -> float:
+    """The free-running code bound for a sample of n_rows output rows."""
+    return max(CODE_TOL, MARGIN * drift + ROW_GRANULE / n_rows)

@@ -168,4 +168,4 @@ def test_block_7b_full_size_sampled_rows(ar):
         print(f"block {name}: {frac:.3%} codes differ (oracle against its jittered self: {drift:.3%}), "
               f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
         assert mse_gpu == pytest.approx(mse_ref, rel=0.02), name
-        assert frac <= code_bound(drift), name
+        assert frac <= code_bound(drift, len(rows)), name

@@ -241,7 +241,7 @@ def _full_size_check(ar, res, W, Xh, rows, ref, g, bits, sym, what, mse_rows=655
     print(f"{what}: {frac:.3%} of sampled codes differ (oracle against its jittered self: {drift:.3%}), "
           f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}, rtn {mse_rtn:.6g}")
     assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert frac <= code_bound(drift)
+    assert frac <= code_bound(drift, len(rows))
     assert mse_gpu < mse_rtn
 
 

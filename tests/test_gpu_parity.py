@@ -361,7 +361,7 @@ def _check_full_size(ar, case, algo, mse_rows=65536):
     print(f"{c.name} {algo}: {frac:.3%} of sampled codes differ (oracle against its jittered self: {drift:.3%}), "
           f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
     assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert frac <= code_bound(drift), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
+    assert frac <= code_bound(drift, len(rows)), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
     _, _, _, Wrtn = oracle.rtn(W[rows], c.bits, c.group_size, c.sym)
     assert mse_gpu < oar.layer_mse(W[rows], Wrtn, Xh[:mse_rows])
 
@@ -426,7 +426,7 @@ def test_q_proj_full_size_sampled_rows(ar, q_proj_case, algo):
     print(f"q_proj {algo}: {frac:.3%} of sampled codes differ (oracle against its jittered self: {drift:.3%}), "
           f"mse {mse_gpu:.6g} vs oracle {mse_ref:.6g}")
     assert mse_gpu == pytest.approx(mse_ref, rel=MSE_RTOL)
-    assert frac <= code_bound(drift), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
+    assert frac <= code_bound(drift, len(rows)), f"{frac:.4%} of sampled codes differ (jittered oracle: {drift:.4%})"
     # scales and zero-points: the groups whose clip factors ended elsewhere
     groups = float(np.mean((_np(res.scale)[rows] != ref.scale) | (_np(res.zero_point)[rows] != ref.zero_point)))
     print(f"    groups with a differing scale or zero-point: {groups:.3%}")

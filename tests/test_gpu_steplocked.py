@@ -135,6 +135,7 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
         rms = float(np.sqrt(np.mean(ref.G ** 2)))
         v_diff = s1.V != ref.V
         v_bad = int(np.sum(v_diff & (np.abs(ref.G) > TIE_G * rms)))
+        v_tie = float(np.max(np.abs(ref.G[v_diff]))) / rms if v_diff.any() else 0.0
         a_diff = s1.alpha != ref.alpha
         a_bad = int(np.sum(a_diff & (np.abs(ref.dalpha) > TIE_GROUP * ref.dalpha_abs)))
         b_diff = s1.beta != ref.beta
@@ -153,7 +154,7 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
         fq = oracle.fake_quant(Wr, s1.V_best, sc, z, g, c.bits)
         codes_ok = (np.array_equal(codes, fq.q.astype(np.uint8)) and np.array_equal(scale, sc)
                     and np.array_equal(zp, z.astype(np.int32)))
-        row = dict(k=k, loss_err=loss_err, loss_bias=loss_bias, v_diff=int(v_diff.sum()), v_bad=v_bad, a_diff=int(a_diff.sum()),
+        row = dict(k=k, loss_err=loss_err, loss_bias=loss_bias, v_diff=int(v_diff.sum()), v_bad=v_bad, v_tie=v_tie, a_diff=int(a_diff.sum()),
                    a_bad=a_bad, b_diff=int(b_diff.sum()), b_bad=b_bad, best_diff=int(np.sum(want != got)),
                    best_bad=best_bad, snap_ok=snap_ok, codes_ok=codes_ok,
                    moved=int(np.sum(s1.V != s0.V)), improved=int(np.sum(got)))
@@ -162,8 +163,10 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
                                                          "best_diff", "best_bad", "moved", "improved")}
     worst = max(r["loss_err"] for r in summary)
     bias = float(np.mean([r["loss_bias"] for r in summary]))
+    tie = max(r["v_tie"] for r in summary)
     print(f"\n{c.name} [{algo}] step-locked over {len(summary)} steps x {len(rows)} rows: "
-          f"V moves {tot['moved']}, differing {tot['v_diff']} (clear of a tie: {tot['v_bad']}); "
+          f"V moves {tot['moved']}, differing {tot['v_diff']} (clear of a tie: {tot['v_bad']}; the largest "
+          f"|G| among them {tie:.2e} of rms); "
           f"alpha differing {tot['a_diff']} ({tot['a_bad']}), beta {tot['b_diff']} ({tot['b_bad']}); "
           f"keep-best improvements {tot['improved']}, decisions differing {tot['best_diff']} ({tot['best_bad']}); "
           f"row-loss rel err max {worst:.2e}, mean signed {bias:.2e}")
