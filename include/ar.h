@@ -252,13 +252,18 @@ ar_status ar_tune_layer_timed(const void* W, ar_dtype w_dtype, int64_t out, int6
                               uint8_t* codes, float* scale, int32_t* zp, float* loss_trace,
                               double* final_mse, void* stream, ar_tune_timing* timing);
 
-/* Workspace of ar_tune_layer_fp_target, in bytes (0 if the arguments are invalid,
- * ask for the direct form, or need more than 64 GiB -- the limit of this mode, which
- * runs in the Gram form only; ar_tune_layer_fp_target then returns AR_EUNSUPPORTED).  On top of ar_tune_workspace_bytes' Gram-form layout:
- * two copies of one calibration block as a bf16 pair (4 * batch_rows * in * 2
- * bytes), the in x in pair M_b^T, every block's out x in pair C_b
- * (n_rows/batch_rows * out * in * 4 bytes), their fp32 sum, and W as a pair when it
- * is fp32. */
+/* Workspace of ar_tune_layer_fp_target, in bytes (0 if the arguments are invalid, or if
+ * they ask for the Gram form and its workspace would exceed 64 GiB).  On top of
+ * ar_tune_workspace_bytes' layout of the same form:
+ *   Gram form: two copies of one calibration block as a bf16 pair (4 * batch_rows * in
+ *     * 2 bytes), the in x in pair M_b^T, every block's out x in pair C_b
+ *     (n_rows/batch_rows * out * in * 4 bytes), their fp32 sum, and W as a pair when
+ *     it is fp32;
+ *   direct form: one block's dX as a pair (batch_rows * in * 4 bytes), E^T = W dX^T
+ *     for every block as an out x n_rows pair (out * n_rows * 4 bytes), and W as a
+ *     pair when it is fp32.
+ * AR_ALGO_AUTO takes the Gram form while its workspace stays within 64 GiB, the direct
+ * form otherwise. */
 size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows, ar_dtype w_dtype,
                                          const ar_tune_params* params);
 
@@ -273,14 +278,16 @@ size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows
  * D = W' - W and dX = X - X_target, so with H_b = X_b^T X_b:
  *   gradient  G = D H_b + W M_b,   M_b = dX_b^T X_b            (in x in)
  *   row loss  L_j = d_j H_b d_j^T + 2 d_j (W M_b)_j^T + |dX_b w_j^T|^2.
- * Per calibration block (before its first step) the library forms dX_b as a bf16
- * pair and computes M_b, C_b = W M_b and e_b = |dX_b w_j^T|^2 on the tensor cores;
- * the step kernel adds C_b to G and the two loss terms to the row loss.
- * final_mse = mean((X W'^T - X_target W^T)^2) over all rows.  Gram form only
- * (params->algo AR_ALGO_AUTO or AR_ALGO_GRAM; AR_ALGO_DIRECT gives
- * AR_EUNSUPPORTED), and only for layers whose workspace stays within 64 GiB
- * (AR_EUNSUPPORTED otherwise: e.g. an 8192 x 29568 layer with 262144 calibration
- * rows in blocks of 16384 would need about 80 GB).  X_target NULL: AR_EINVAL.  Otherwise arguments, results and
+ * Gram form: per calibration block (before its first step) the library forms dX_b as
+ * a bf16 pair and computes M_b, C_b = W M_b and e_b = |dX_b w_j^T|^2 on the tensor
+ * cores; the step kernel adds C_b to G and the two loss terms to the row loss.
+ * Direct form: per block it computes E_b^T = W dX_b^T (a bf16 pair), which the
+ * residual's epilogue adds to X_b D^T, so R and everything after it are the plain
+ * loop's.  final_mse = mean((X W'^T - X_target W^T)^2) over all rows.  Either form
+ * (params->algo; see ar_tune_fp_target_workspace_bytes for the automatic choice); an
+ * explicit AR_ALGO_GRAM whose workspace would exceed 64 GiB gives AR_EUNSUPPORTED
+ * (an 8192 x 29568 layer with 262144 calibration rows in blocks of 16384 would need
+ * about 80 GB there, about 14 GB in the direct form).  X_target NULL: AR_EINVAL.  Otherwise arguments, results and
  * errors as ar_tune_layer, with workspace of ar_tune_fp_target_workspace_bytes(). */
 ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in,
                                   const uint16_t* X, const uint16_t* X_target, int64_t n_rows,

@@ -172,6 +172,15 @@ ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune
 // Plan: which algorithm, tile widths, workspace layout.
 // ---------------------------------------------------------------------------
 
+constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
+// The full-precision-target mode in the Gram form keeps, on top of the Gram matrices,
+// every block's C_b = W M_b as a bf16 pair (n_rows/batch_rows * out * in * 4 bytes).
+// It runs in that form while its workspace stays within this, in the direct form
+// otherwise (the automatic choice), and an explicit AR_ALGO_GRAM beyond it is
+// refused: the 8192 x 29568 down_proj with 16 blocks of 16384 rows would need about
+// 80 GB there, and about 14 GB in the direct form.
+constexpr size_t kFpTargetMaxBytes = 64ull << 30;
+
 struct Plan {
   int algo = AR_ALGO_DIRECT;
   int split = 1;
@@ -217,14 +226,7 @@ struct Plan {
   int64_t gram_chunk = 2048;
 };
 
-constexpr double kGramMaxBytes = 64.0 * (1ull << 30);
-// The full-precision-target mode runs in the Gram form only: on top of the Gram
-// matrices it keeps every block's C_b = W M_b as a bf16 pair (n_rows/batch_rows *
-// out * in * 4 bytes).  A layer whose workspace would exceed this is refused
-// (AR_EUNSUPPORTED), as the automatic choice refuses Gram matrices above
-// kGramMaxBytes: the 8192 x 29568 down_proj of a Qwen2.5-72B-shaped block with
-// 16 blocks of 16384 rows would need about 80 GB.
-constexpr size_t kFpTargetMaxBytes = 64ull << 30;
+
 
 Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool fp_target = false,
                bool w_f32 = false) {
@@ -246,9 +248,13 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   const double gram =
       P.iters * pieces_gram * 2.0 * out * in * in + 2.0 * n * in * in + pieces_gram * 2.0 * out * in * in;
   const double gram_bytes = (P.nb + 1.0) * in * in * 2.0 * (P.split ? 2.0 : 1.0);
-  if (p->algo == AR_ALGO_GRAM || (fp_target && p->algo == AR_ALGO_AUTO))
+  // Full-precision target: the Gram form also keeps every block's C_b = W M_b (a bf16
+  // pair) on top of the Gram matrices; it is chosen while that stays within
+  // kFpTargetMaxBytes, the direct form otherwise.
+  const double gram_fpt_bytes = gram_bytes + (P.nb * 4.0 + 24.0) * out * in;
+  if (p->algo == AR_ALGO_GRAM || (fp_target && p->algo == AR_ALGO_AUTO && gram_fpt_bytes <= kFpTargetMaxBytes))
     P.algo = AR_ALGO_GRAM;
-  else if (p->algo == AR_ALGO_DIRECT)
+  else if (p->algo == AR_ALGO_DIRECT || fp_target)
     P.algo = AR_ALGO_DIRECT;
   else
     P.algo = (P.iters > 0 && gram < direct && gram_bytes <= kGramMaxBytes) ? AR_ALGO_GRAM : AR_ALGO_DIRECT;
@@ -274,7 +280,10 @@ struct Layout {
       // M_b^T = X_b^T dX_b (pair), every block's C_b = W M_b (pair), their sum Cs
       // (fp32), e_b[j] = |dX_b w_j^T|^2 and its sum, the partials of e_b, and W as
       // a pair when it is fp32
-      dX_hi, dX_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo, total;
+      dX_hi, dX_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo,
+      // direct form with a full-precision target: E^T = W dX^T for every block, [out, n]
+      // as a bf16 pair (block b in columns b*B ..), added to the residual
+      E_hi, E_lo, total;
 };
 
 Layout make_layout(const Plan& P) {
@@ -340,6 +349,17 @@ Layout make_layout(const Plan& P) {
   } else {
     L.Rt_hi = take(static_cast<size_t>(P.out) * P.B * 2);
     L.Rt_lo = P.split ? take(static_cast<size_t>(P.out) * P.B * 2) : L.Rt_hi;
+    if (P.fp_target) {
+      const size_t blk = static_cast<size_t>(P.B) * P.in * 2;
+      L.dX_hi = take(blk);
+      L.dX_lo = take(blk);
+      L.E_hi = take(static_cast<size_t>(P.out) * P.n * 2);
+      L.E_lo = take(static_cast<size_t>(P.out) * P.n * 2);
+      if (P.w_f32) {
+        L.Wp_hi = take(elems * 2);
+        L.Wp_lo = take(elems * 2);
+      }
+    }
   }
   L.total = off;
   return L;
@@ -402,9 +422,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
 
   if (X_target && !aligned(X_target, 16)) return AR_EINVAL;
   const Plan P = make_plan(out, in, n_rows, p, X_target != nullptr, w_dtype == AR_F32);
-  if (P.fp_target && P.algo != AR_ALGO_GRAM) return AR_EUNSUPPORTED;
   const Layout L = make_layout(P);
-  if (P.fp_target && L.total > kFpTargetMaxBytes) return AR_EUNSUPPORTED;
+  if (P.fp_target && P.algo == AR_ALGO_GRAM && L.total > kFpTargetMaxBytes) return AR_EUNSUPPORTED;
   const Fault fault = injected_fault();
   if (ws_bytes < L.total || fault == kFaultAlloc) return AR_ENOMEM;
   const bool gram = P.algo == AR_ALGO_GRAM;
@@ -497,8 +516,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   const __nv_bfloat16* Wa_hi = static_cast<const __nv_bfloat16*>(W);
   const __nv_bfloat16* Wa_lo = nullptr;
   if (fpt) {
-    AR_CUDA_TRY(cudaMemsetAsync(F(L.Cs), 0, elems * 4, st));
-    AR_CUDA_TRY(cudaMemsetAsync(F(L.es), 0, static_cast<size_t>(out) * 4, st));
+    if (gram) {
+      AR_CUDA_TRY(cudaMemsetAsync(F(L.Cs), 0, elems * 4, st));
+      AR_CUDA_TRY(cudaMemsetAsync(F(L.es), 0, static_cast<size_t>(out) * 4, st));
+    }
     if (P.w_f32) {
       AR_CUDA_TRY(launch_split_pair(static_cast<const float*>(W), static_cast<int64_t>(elems), H(L.Wp_hi),
                                     H(L.Wp_lo), st));
@@ -568,10 +589,14 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   //   C_b   = W M_b               [out, in]  (pair; the step adds it to G)
   //   e_b[j] = |dX_b w_j^T|^2     (row sums of squares of W dX_b^T)
   //   Cs += C_b,  es += e_b       (the final MSE over all blocks)
+  // Direct form instead: per block only E_b^T = W dX_b^T [out, B], stored into
+  // columns b*B .. of the [out, n] pair E; the residual epilogue adds it to
+  // X_b D^T, so R = X_b W'^T - X_target,b W^T.
   GemmMaps mt_maps{}, c_maps{}, e_maps{};
   GemmArgs mg, cg, eg;
   if (fpt) {
     const int nseg_w = P.w_f32 ? 3 : 2;  // W pair x operand pair, or W x operand pair
+   if (gram) {
     AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b0, H(L.dX_hi), B, in, 64));
     AR_CUDA_TRY(make_tmap_bf16(&mt_maps.b1, H(L.dX_lo), B, in, 64));
     fill_grid(mg, in, in, B, 256, 2, P.pair_fpt);
@@ -584,6 +609,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     mg.C_hi = H(L.Mt_hi);
     mg.C_lo = H(L.Mt_lo);
     mg.ldc = in;
+   }
     for (GemmMaps* m : {&c_maps, &e_maps}) {
       AR_CUDA_TRY(make_tmap_bf16(&m->a0, Wa_hi, out, in, kBM));
       if (Wa_lo)
@@ -592,8 +618,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
         m->a1 = m->a0;
     }
     const uint32_t fpt_box = P.pair_fpt ? 128 : 256;  // pair tiles: half the B rows per CTA
-    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b0, H(L.Mt_hi), in, in, fpt_box));
-    AR_CUDA_TRY(make_tmap_bf16(&c_maps.b1, H(L.Mt_lo), in, in, fpt_box));
+    if (gram) {
+      AR_CUDA_TRY(make_tmap_bf16(&c_maps.b0, H(L.Mt_hi), in, in, fpt_box));
+      AR_CUDA_TRY(make_tmap_bf16(&c_maps.b1, H(L.Mt_lo), in, in, fpt_box));
+    }
     AR_CUDA_TRY(make_tmap_bf16(&e_maps.b0, H(L.dX_hi), B, in, fpt_box));
     AR_CUDA_TRY(make_tmap_bf16(&e_maps.b1, H(L.dX_lo), B, in, fpt_box));
     for (GemmArgs* g : {&cg, &eg}) {
@@ -611,8 +639,13 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     cg.C_hi = H(L.Cc_hi);
     cg.C_lo = H(L.Cc_lo);
     cg.ldc = in;
-    eg.part = F(L.epart);
-    eg.part_ld = eg.num_n_blk * kEpiHalves;
+    if (gram) {
+      eg.part = F(L.epart);
+      eg.part_ld = eg.num_n_blk * kEpiHalves;
+    } else {
+      eg.ldc = n_rows;  // C_hi, C_lo point at block b's columns of E
+      if (checks) eg.chk_c = out * n_rows;
+    }
   }
   auto fp_target_block = [&](int64_t b) -> cudaError_t {
     const int64_t blk = B * in;
@@ -640,11 +673,22 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     waited_block[b] = 1;
     return cudaStreamWaitEvent(st, block_ready[b], 0);
   };
+  auto fp_target_block_direct = [&](int64_t b) -> cudaError_t {
+    const int64_t blk = B * in;
+    cudaError_t e = launch_diff_pair(X + b * blk, X_target + b * blk, blk, H(L.dX_hi), H(L.dX_lo), st);
+    eg.C_hi = H(L.E_hi) + b * B;
+    eg.C_lo = H(L.E_lo) + b * B;
+    eg.chk_c = checks ? out * n_rows - b * B : 0;
+    if (e == cudaSuccess) e = launch_gemm(kEpiStore, 256, e_maps, eg, sms, st);
+    launches += 2;
+    return e;
+  };
   auto ensure_block = [&](int64_t b) -> cudaError_t {
     if (have_block[b]) return cudaSuccess;
     have_block[b] = 1;
     cudaError_t e = wait_block(b);
-    if (e != cudaSuccess || !gram) return e;
+    if (e != cudaSuccess) return e;
+    if (!gram) return fpt ? fp_target_block_direct(b) : cudaSuccess;
     e = make_tmap_bf16(&gram_maps.a0, X + b * B * in, B, in, 64);
     if (e != cudaSuccess) return e;
     gram_maps.a1 = gram_maps.b0 = gram_maps.b1 = gram_maps.a0;
@@ -724,7 +768,11 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     ++launches;
     return launch_group_finish(f, st);
   };
-  const EpiKind upd_kind = fpt ? (P.wide ? kEpiUpdateFpWide : kEpiUpdateFp) : (P.wide ? kEpiUpdateWide : kEpiUpdate);
+  // The Gram form's full-precision-target terms enter the step's epilogue; the direct
+  // form's are already in R (E_b^T, added by the residual's epilogue).
+  const bool fpt_step = fpt && gram;
+  const EpiKind upd_kind =
+      fpt_step ? (P.wide ? kEpiUpdateFpWide : kEpiUpdateFp) : (P.wide ? kEpiUpdateWide : kEpiUpdate);
 
   float* best_cur = best_loss;
   float* best_next = best_alt;
@@ -836,6 +884,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     r.part = part[0];
     r.part_ld = static_cast<int>(P.nparts_res);
     if (checks) r.chk_c = out * B;
+    if (fpt) r.ldc_add = n_rows;  // + E_b^T: block b's columns of E
 
     fill_grid(u, out, in, B, P.bn_upd, nseg_d, P.pair_direct);  // update: G = (R_hi + R_lo)^T X_b
     u.raster_m = P.raster_upd;
@@ -856,6 +905,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       const int64_t b0 = sched[t] * B;
       r.b_row_off = static_cast<int>(b0);
       AR_CUDA_TRY(ensure_block(sched[t]));
+      if (fpt) {
+        r.C_add = H(L.E_hi) + b0;
+        r.C_add_lo = H(L.E_lo) + b0;
+      }
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t], st));
       if (fault == kFaultLaunch) return AR_ECUDA;
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
@@ -946,7 +999,12 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       AR_CUDA_TRY(launch_gemm(kEpiDotD, P.bn_fin, m, f, sms, st));
       launches += 2;
     } else {
-      for (int64_t b = 0; b < P.nb; ++b) AR_CUDA_TRY(wait_block(b));
+      for (int64_t b = 0; b < P.nb; ++b) AR_CUDA_TRY(fpt ? ensure_block(b) : wait_block(b));
+      if (fpt) {  // mean((X D^T + E)^2) = mean((X W'^T - X_target W^T)^2)
+        f.C_add = H(L.E_hi);
+        f.C_add_lo = H(L.E_lo);
+        f.ldc_add = n_rows;
+      }
       AR_CUDA_TRY(make_tmap_bf16(&m.a0, D_hi, out, in, kBM));
       AR_CUDA_TRY(make_tmap_bf16(&m.a1, D_lo, out, in, kBM));
       AR_CUDA_TRY(make_tmap_bf16(&m.b0, X, n_rows, in, P.bn_fin));
@@ -1240,9 +1298,8 @@ size_t ar_tune_fp_target_workspace_bytes(int64_t out, int64_t in, int64_t n_rows
   if (w_dtype != AR_F32 && w_dtype != AR_BF16) return 0;
   if (out == 0 || in == 0) return 256;
   const Plan P = make_plan(out, in, n_rows, p, true, w_dtype == AR_F32);
-  if (P.algo != AR_ALGO_GRAM) return 0;
   const size_t total = make_layout(P).total;
-  return total > kFpTargetMaxBytes ? 0 : total;
+  return (P.algo == AR_ALGO_GRAM && total > kFpTargetMaxBytes) ? 0 : total;
 }
 
 ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, const uint16_t* X,
@@ -1253,7 +1310,6 @@ ar_status ar_tune_layer_fp_target(const void* W, ar_dtype w_dtype, int64_t out, 
   if (chk != AR_OK) return chk;
   if (out == 0 || in == 0) return AR_OK;
   if (!X_target) return AR_EINVAL;
-  if (p->algo == AR_ALGO_DIRECT) return AR_EUNSUPPORTED;
   return tune_impl(W, w_dtype, out, in, X, n_rows, p, state, workspace, ws_bytes, codes, scale, zp, loss_trace,
                    final_mse, stream, nullptr, nullptr, X_target);
 }

@@ -145,7 +145,12 @@ struct GemmArgs {
   // kEpiStore: C rows j go to row c_row_off + j of [*, ldc]
   __nv_bfloat16* C_hi = nullptr;
   __nv_bfloat16* C_lo = nullptr;  // may be null
-  const __nv_bfloat16* C_add = nullptr;  // may be null: [*, ldc] added in fp32 before the store
+  // kEpiStore / kEpiSumSq: when set, hi (+ lo) of [*, ldc_add] (0: ldc) are added to C
+  // in fp32 before its row sums and its store (a residual, or the full-precision
+  // target's term of the direct form's residual)
+  const __nv_bfloat16* C_add = nullptr;
+  const __nv_bfloat16* C_add_lo = nullptr;
+  int64_t ldc_add = 0;
   int64_t ldc = 0;
   // kEpiStore of a symmetric C (M == N, A == B): only tiles that reach the upper
   // triangle run (num_tiles counts them); each writes its upper elements in place and

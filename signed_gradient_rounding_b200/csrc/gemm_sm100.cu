@@ -141,6 +141,17 @@ __device__ __forceinline__ void load_w32(const void* W, int w_bf16, int64_t idx,
   }
 }
 
+// 8 consecutive bf16 values (16 bytes, aligned) as fp32.
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 x = *reinterpret_cast<const uint4*>(p);
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    v[2 * h] = __uint_as_float(xs[h] << 16);
+    v[2 * h + 1] = __uint_as_float(xs[h] & 0xFFFF0000u);
+  }
+}
+
 // 32 consecutive bf16 values as fp32.
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&v)[32]) {
   load_w32(p, 1, 0, v);
@@ -261,8 +272,7 @@ __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, i
 // ---------------------------------------------------------------------------
 
 // kEpiStore: 32 consecutive columns col0.. of row j (nvalid of them in range): the
-// diagonal element into diag_out (stored as 0 in the pair), C_add, and the bf16 pair
-// store (a symmetric C writes its upper elements in place and the strictly upper ones
+// diagonal element into diag_out (stored as 0 in the pair), and the bf16 pair store (a symmetric C writes its upper elements in place and the strictly upper ones
 // again transposed, so every element is written once).
 __device__ __forceinline__ void store_cols32(const GemmArgs& a, int j, int col0, int nvalid, float (&x)[32]) {
   if (a.diag_out && j >= col0 && j < col0 + 32) {
@@ -275,12 +285,6 @@ __device__ __forceinline__ void store_cols32(const GemmArgs& a, int j, int col0,
   }
   const int64_t off = (a.c_row_off + j) * a.ldc + col0;
   if (!in_bounds(off, nvalid, a.chk_c, a.status)) return;
-  if (a.C_add) {
-    float ad[32];
-    load_bf16x32(a.C_add + off, ad);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] += ad[i];
-  }
   if (!a.symmetric) {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
@@ -337,6 +341,23 @@ __device__ __forceinline__ void epi_rows(const GemmArgs& a, uint32_t t_row, int 
     float x[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+    if ((kKind == kEpiStore || kKind == kEpiSumSq) && a.C_add) {
+      // C += add_hi + add_lo (the pair's sum is exact in fp32), 8 columns at a time
+      const int64_t offa = (a.c_row_off + j) * (a.ldc_add ? a.ldc_add : a.ldc) + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q * 8 >= nvalid) break;
+        float hv[8], lv[8];
+        load_bf16x8(a.C_add + offa + q * 8, hv);
+        if (a.C_add_lo) {
+          load_bf16x8(a.C_add_lo + offa + q * 8, lv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hv[i] = __fadd_rn(hv[i], lv[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[q * 8 + i] = __fadd_rn(x[q * 8 + i], hv[i]);
+      }
+    }
     if (kKind == kEpiStore || kKind == kEpiSumSq) {
 #pragma unroll
       for (int i = 0; i < 32; ++i)

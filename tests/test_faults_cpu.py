@@ -56,15 +56,21 @@ def test_status_strings_cover_the_check_status(ar):
     assert ar.lib.ar_status_string(ar.AR_ECHECK).decode().startswith("AR_ECHECK")
 
 
-def test_fp_target_refuses_layers_beyond_its_workspace_limit(ar):
-    """The full-precision-target mode runs in the Gram form only; the 8192 x 29568
-    down_proj with 262144 calibration rows (16 blocks) would need about 80 GB of
-    workspace, above the mode's 64 GiB limit: refused before any GPU work."""
-    p = ar.make_params(bits=2, group_size=128, iters=200, batch_rows=16384)
+def test_fp_target_gram_limit_and_direct_form(ar):
+    """The full-precision-target mode keeps every block's C_b = W M_b in the Gram form;
+    for the 8192 x 29568 down_proj with 262144 calibration rows (16 blocks) that would
+    need about 80 GB, above the form's 64 GiB limit.  The automatic choice then takes
+    the direct form (about 14 GB); an explicit Gram form is refused before any GPU work."""
     fpt = ar.lib.ar_tune_fp_target_workspace_bytes
-    assert fpt(8192, 29568, 262144, ar.AR_BF16, ctypes.byref(p)) == 0
-    assert fpt(4096, 4096, 262144, ar.AR_BF16, ctypes.byref(p)) > 0       # q_proj fits
+    auto = ar.make_params(bits=2, group_size=128, iters=200, batch_rows=16384)
+    gram = ar.make_params(bits=2, group_size=128, iters=200, batch_rows=16384, algo="gram")
+    direct = ar.make_params(bits=2, group_size=128, iters=200, batch_rows=16384, algo="direct")
+    ws_auto = fpt(8192, 29568, 262144, ar.AR_BF16, ctypes.byref(auto))
+    assert ws_auto == fpt(8192, 29568, 262144, ar.AR_BF16, ctypes.byref(direct))
+    assert 0 < ws_auto < 20 * 2**30
+    assert fpt(8192, 29568, 262144, ar.AR_BF16, ctypes.byref(gram)) == 0
+    assert fpt(4096, 4096, 262144, ar.AR_BF16, ctypes.byref(auto)) > 0       # q_proj: Gram form
     dummy = ctypes.c_void_p(4096)
-    st = ar.lib.ar_tune_layer_fp_target(dummy, ar.AR_BF16, 8192, 29568, dummy, dummy, 262144, ctypes.byref(p),
+    st = ar.lib.ar_tune_layer_fp_target(dummy, ar.AR_BF16, 8192, 29568, dummy, dummy, 262144, ctypes.byref(gram),
                                         None, dummy, 1 << 40, dummy, dummy, dummy, None, None, None)
     assert st == ar.AR_EUNSUPPORTED

@@ -149,12 +149,12 @@ def test_full_batch_per_step(ar, algo):
 
 # ------------------------------------------------ quant-aware input, full-precision target
 
-def _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed):
+def _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed, algo="gram"):
     from workloads import make_quantised_path_input
     W = make_weight(out, inn, 0.02, wdt, seed=seed)
     Xf = make_activations(n, inn, "llm", seed=seed)
     Xq = make_quantised_path_input(Xf, 0.05, seed=seed)
-    p = ar.make_params(bits=bits, group_size=g, iters=iters, batch_rows=B, algo="gram")
+    p = ar.make_params(bits=bits, group_size=g, iters=iters, batch_rows=B, algo=algo)
     res = ar.tune_layer_fp_target(_w_dev(W, wdt), _x_dev(Xq), _x_dev(Xf), p)
     assert ar.tune_status(res.workspace) == ar.AR_OK
     ref = oracle.tune_layer(W, Xq, bits, g, False, iters, 0.005, -1.0, B, 0, X_target=Xf)
@@ -166,9 +166,12 @@ def _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed):
                                   (200, 384, 2048, 512, 24, 2, 128, "bf16"),
                                   (200, 256, 1560, 520, 20, 3, 128, "bf16")],
                          ids=["tiny-f32-full-batch", "multiblock-bf16", "ragged-W2", "batch-520"])
-def test_fp_target_parity(ar, case):
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_fp_target_parity(ar, case, algo):
+    """Both forms: Gram (C_b = W M_b added to G) and direct (E_b^T = W dX_b^T added to
+    the residual)."""
     out, inn, n, B, iters, bits, g, wdt = case
-    res, ref, *_ = _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed=21)
+    res, ref, *_ = _fp_target_case(ar, out, inn, n, B, iters, bits, g, wdt, seed=21, algo=algo)
     frac = float(np.mean(_np(res.codes) != ref.codes))
     assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
     assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
@@ -177,12 +180,13 @@ def test_fp_target_parity(ar, case):
     np.testing.assert_allclose(trace, ref.loss_trace, rtol=0.05)
 
 
-def test_fp_target_with_own_input_is_the_usual_loop(ar):
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_fp_target_with_own_input_is_the_usual_loop(ar, algo):
     """X_target = X: dX = 0, so every added term is an exact zero and the results
     equal ar_tune_layer's bit for bit."""
     W = make_weight(256, 512, 0.02, "bf16", seed=22)
     X = make_activations(2048, 512, "llm", seed=22)
-    p = ar.make_params(bits=3, group_size=128, iters=20, batch_rows=512, algo="gram")
+    p = ar.make_params(bits=3, group_size=128, iters=20, batch_rows=512, algo=algo)
     a = ar.tune_layer_fp_target(_w_dev(W, "bf16"), _x_dev(X), _x_dev(X), p)
     b = ar.tune_layer(_w_dev(W, "bf16"), _x_dev(X), p)
     torch.cuda.synchronize()
@@ -263,9 +267,11 @@ def test_mse_init_q_proj_full_size(ar):
     _full_size_check(ar, res, W, Xh, rows, ref, c.group_size, c.bits, c.sym, "q_proj mse init", drift=drift)
 
 
-def test_fp_target_q_proj_full_size(ar):
-    """The full-precision-target mode on q_proj at full size: the quantised-path input is
-    the target's input with 5% seeded noise; the oracle replays 32 sampled rows."""
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_fp_target_q_proj_full_size(ar, algo):
+    """The full-precision-target mode on q_proj at full size, in both forms: the
+    quantised-path input is the target's input with 5% seeded noise; the oracle
+    replays 32 sampled rows."""
     from workloads import Q_PROJ_7B as c, make_activations_cuda
     W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)
     Xt = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0)
@@ -276,7 +282,7 @@ def test_fp_target_q_proj_full_size(ar):
     for r0 in range(0, c.n_rows, chunk):
         z = torch.randn((min(chunk, c.n_rows - r0), c.inn), generator=gen, device="cuda")
         Xq[r0:r0 + chunk] = (Xt[r0:r0 + chunk].float() * (1 + 0.05 * z)).to(torch.bfloat16)
-    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, batch_rows=c.batch_rows, algo="gram")
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, batch_rows=c.batch_rows, algo=algo)
     res = ar.tune_layer_fp_target(_w_dev(W, "bf16"), Xq, Xt, p)
     assert ar.tune_status(res.workspace) == ar.AR_OK
     bits16 = lambda t: t.view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
@@ -287,5 +293,5 @@ def test_fp_target_q_proj_full_size(ar):
                             X_target=Xth, want_final_mse=False)
     drift = oracle_drift(ref, W[rows], Xqh, c.bits, c.group_size, c.sym, c.iters, c.lr, c.minmax_lr, c.batch_rows,
                          X_target=Xth)
-    _full_size_check(ar, res, W, Xqh, rows, ref, c.group_size, c.bits, c.sym, "q_proj fp target", mse_rows=32768,
-                     X_target=Xth, drift=drift)
+    _full_size_check(ar, res, W, Xqh, rows, ref, c.group_size, c.bits, c.sym, f"q_proj fp target ({algo})",
+                     mse_rows=32768, X_target=Xth, drift=drift)
