@@ -422,8 +422,11 @@ ar_status ar_tune_status(const void* workspace, void* stream);
  * Asynchronous on `stream`, after the tuning call it reads.  iters == 0, out == 0 or
  * in == 0: nothing to copy.  AR_EINVAL as ar_tune_layer, or a NULL pointer;
  * AR_ENOMEM: ws_bytes smaller than ar_tune_workspace_bytes() for these arguments.
- * (Workspaces of ar_tune_layer_fp_target, ar_tune_layer_host and
- * ar_tune_layer_static have other layouts and are not read by this call.) */
+ * The losses sit at the same place in a workspace of ar_tune_layer_fp_target, so
+ * this call reads those too when params->algo names the form (AR_ALGO_GRAM or
+ * AR_ALGO_DIRECT; with AR_ALGO_AUTO the two entry points may choose differently).
+ * (Workspaces of ar_tune_layer_host and ar_tune_layer_static are not read by this
+ * call.) */
 ar_status ar_tune_row_losses(const void* workspace, size_t ws_bytes, int64_t out, int64_t in, int64_t n_rows,
                              const ar_tune_params* params, float* row_loss, void* stream);
 

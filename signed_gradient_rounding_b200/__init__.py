@@ -349,9 +349,10 @@ def tune_layer(W: torch.Tensor, X: torch.Tensor, params: TuneParams, state: Tune
 
 def tune_layer_fp_target(W: torch.Tensor, X: torch.Tensor, X_target: torch.Tensor, params: TuneParams,
                          workspace: torch.Tensor | None = None, want_final_mse: bool = True,
-                         stream=None) -> TuneResult:
+                         stream=None, state: TuneState | None = None) -> TuneResult:
     """ar_tune_layer_fp_target on device tensors: the layer sees X (its input on the
-    quantised path) and is tuned against the full-precision output X_target W^T."""
+    quantised path) and is tuned against the full-precision output X_target W^T.
+    ``state`` as for tune_layer (inspection and resume)."""
     _dev(W, "W")
     _dev(X, "X", torch.bfloat16)
     _dev(X_target, "X_target", torch.bfloat16)
@@ -371,10 +372,13 @@ def tune_layer_fp_target(W: torch.Tensor, X: torch.Tensor, X_target: torch.Tenso
     zp = torch.empty((out, G), dtype=torch.int32, device=W.device)
     trace = torch.empty((max(params.iters, 1),), dtype=torch.float32, device=W.device)
     mse = torch.empty((1,), dtype=torch.float64, device=W.device) if want_final_mse else None
+    st = ctypes.byref(state._c()) if state is not None else None
     _check(_lib.ar_tune_layer_fp_target(_ptr(W), wdt, out, inn, _ptr(X), _ptr(X_target), n_rows,
-                                        ctypes.byref(params), None, _ptr(workspace), workspace.numel(),
+                                        ctypes.byref(params), st, _ptr(workspace), workspace.numel(),
                                         _ptr(codes), _ptr(scale), _ptr(zp), _ptr(trace), _ptr(mse),
                                         _stream(stream)), "ar_tune_layer_fp_target")
+    if state is not None:
+        state.initialized = True
     return TuneResult(codes, scale, zp, trace[:params.iters], mse, workspace)
 
 

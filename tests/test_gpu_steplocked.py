@@ -26,6 +26,7 @@ the trajectories) is measured and printed by the full-size tests in
 test_gpu_parity.py, which decompose it into rows whose best step differs and
 rows that kept the same step.
 """
+import ctypes
 import dataclasses
 
 import numpy as np
@@ -73,15 +74,34 @@ def _snap(st, rows_t) -> _Snap:
                    ("V", "alpha", "beta", "best_loss", "V_best", "alpha_best", "beta_best")))
 
 
-def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
+def _quantised_path_input(Xt):
+    """The layer's input on the quantised path for the full-precision-target mode: the
+    target's input with 5% seeded multiplicative noise, in bf16 (as the full-size
+    fp-target test and the benchmark make it)."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    Xq = torch.empty_like(Xt)
+    chunk = (1 << 27) // Xt.shape[1]
+    for r0 in range(0, Xt.shape[0], chunk):
+        z = torch.randn((min(chunk, Xt.shape[0] - r0), Xt.shape[1]), generator=gen, device="cuda")
+        Xq[r0:r0 + chunk] = (Xt[r0:r0 + chunk].float() * (1 + 0.05 * z)).to(torch.bfloat16)
+    return Xq
+
+
+def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0, fp_target=False):
     """Run workload ``c`` on the GPU step by step through the checkpoints and compare
-    each checked step with the oracle's step from the GPU's state.  Returns a
-    per-checkpoint summary (also printed)."""
+    each checked step with the oracle's step from the GPU's state.  With fp_target the
+    layer sees a noisy copy of the activations and is tuned against the full-precision
+    output (ar_tune_layer_fp_target).  Returns a per-checkpoint summary (also printed)."""
     g = c.inn if c.group_size == -1 else c.group_size
     W = make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=seed)
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=seed)
+    Xt = None
+    if fp_target:
+        Xt, Xd = Xd, _quantised_path_input(Xd)
     Xh = _bits(Xd)
+    Xth = _bits(Xt) if fp_target else None
     rows = np.sort(np.random.default_rng(seed).choice(c.out, n_rows_sample, replace=False))
     rows_t = torch.from_numpy(rows).cuda()
     Wr = W[rows]
@@ -97,21 +117,30 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
                               minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=seed, start_step=start,
                               algo=algo)
 
-    need = max(ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, params(it, 0)) for it in (0, 1, c.iters))
+    def need_bytes(p):
+        if fp_target:
+            return int(ar.lib.ar_tune_fp_target_workspace_bytes(c.out, c.inn, c.n_rows, ar.AR_BF16, ctypes.byref(p)))
+        return ar.tune_workspace_bytes(c.out, c.inn, c.n_rows, p)
+
+    def run(p):
+        if fp_target:
+            return ar.tune_layer_fp_target(Wd, Xd, Xt, p, workspace=ws, want_final_mse=False, state=st)
+        return ar.tune_layer(Wd, Xd, p, state=st, workspace=ws, want_loss_trace=False, want_final_mse=False)
+
+    need = max(need_bytes(params(it, 0)) for it in (0, 1, c.iters))
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     # iters = 0 initialises the state (V = 0, alpha = beta = 1, best = +inf).
-    ar.tune_layer(Wd, Xd, params(0, 0), state=st, workspace=ws, want_loss_trace=False, want_final_mse=False)
+    run(params(0, 0))
     cache = {}
     summary = []
     cur = 0
     for k in checkpoints:
         if k > cur:
-            ar.tune_layer(Wd, Xd, params(k - cur, cur), state=st, workspace=ws, want_loss_trace=False,
-                          want_final_mse=False)
+            run(params(k - cur, cur))
             cur = k
         s0 = _snap(st, rows_t)
         p1 = params(1, k)
-        res = ar.tune_layer(Wd, Xd, p1, state=st, workspace=ws, want_loss_trace=False, want_final_mse=False)
+        res = run(p1)
         assert ar.tune_status(ws) == ar.AR_OK
         loss_gpu = _np(ar.tune_row_losses(ws, c.out, c.inn, c.n_rows, p1)[0].index_select(0, rows_t))
         loss_gpu = loss_gpu.astype(np.float64) / c.batch_rows
@@ -125,9 +154,11 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
         if blk not in cache:
             if len(cache) >= 4:
                 cache.pop(next(iter(cache)))
-            cache[blk] = oracle.autoround._rows_f64(Xh, blk * c.batch_rows, (blk + 1) * c.batch_rows)
-        ref = oracle.sign_step(Wr, cache[blk], s0.V, s0.alpha, s0.beta, wmin, wmax, g, c.bits, c.sym, c.lr, mlr,
-                               with_scale=True)
+            r0, r1 = blk * c.batch_rows, (blk + 1) * c.batch_rows
+            cache[blk] = (oracle.autoround._rows_f64(Xh, r0, r1),
+                          oracle.autoround._rows_f64(Xth, r0, r1) if fp_target else None)
+        ref = oracle.sign_step(Wr, cache[blk][0], s0.V, s0.alpha, s0.beta, wmin, wmax, g, c.bits, c.sym, c.lr, mlr,
+                               Xt_b=cache[blk][1], with_scale=True)
 
         rel = (loss_gpu - ref.row_loss) / ref.row_loss
         loss_err = float(np.max(np.abs(rel)))
@@ -164,7 +195,7 @@ def _step_locked(ar, c, algo, n_rows_sample, checkpoints, seed=0):
     worst = max(r["loss_err"] for r in summary)
     bias = float(np.mean([r["loss_bias"] for r in summary]))
     tie = max(r["v_tie"] for r in summary)
-    print(f"\n{c.name} [{algo}] step-locked over {len(summary)} steps x {len(rows)} rows: "
+    print(f"\n{c.name} [{algo}{', full-precision target' if fp_target else ''}] step-locked over {len(summary)} steps x {len(rows)} rows: "
           f"V moves {tot['moved']}, differing {tot['v_diff']} (clear of a tie: {tot['v_bad']}; the largest "
           f"|G| among them {tie:.2e} of rms); "
           f"alpha differing {tot['a_diff']} ({tot['a_bad']}), beta {tot['b_diff']} ({tot['b_bad']}); "
@@ -213,3 +244,21 @@ def test_down_72b_step_locked(ar):
     """Qwen2.5-72B down_proj 8192 x 29568 W2 g128 (direct form, as the full run picks)."""
     _assert_locked(_step_locked(ar, DOWN_72B, "direct", 32, [0, 50, 100, 150, 199]),
                    loss_rtol(DOWN_72B, "direct"))
+
+
+def test_q_proj_per_channel_step_locked(ar):
+    """The 4096 x 4096 W4 layer with one group per row (the wide-group path: the step
+    kernel's per-segment partials and the group-finish kernel), Gram form."""
+    c = dataclasses.replace(Q_PROJ_7B, group_size=-1, name="q_proj per-channel")
+    _assert_locked(_step_locked(ar, c, "gram", 32, [0, 50, 100, 150, 199]), loss_rtol(c, "gram"))
+
+
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_q_proj_fp_target_step_locked(ar, algo):
+    """The full-precision-target mode ("enable_quanted_input"): the layer sees a noisy
+    copy of the activations and is tuned against the full-precision output, in both
+    forms (Gram: C_b joins G; direct: E_b joins R)."""
+    # the target's terms of the loss (|dX_b w_j^T|^2, or E_b inside R) accumulate over
+    # K = in, as the direct form's residual does: its bound applies in both forms
+    _assert_locked(_step_locked(ar, Q_PROJ_7B, algo, 32, [0, 50, 100, 150, 199], fp_target=True),
+                   loss_rtol(Q_PROJ_7B, "direct"))
