@@ -263,10 +263,11 @@ def run_fp_target(args):
         z = torch.randn((r1 - r0, c.inn), generator=gen, device=dev)
         Xq[r0:r1] = (Xt[r0:r1].float() * (1 + 0.05 * z)).to(torch.bfloat16)
     p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
-                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo="gram")
-    ws = torch.empty(int(ar._lib.ar_tune_fp_target_workspace_bytes(c.out, c.inn, c.n_rows,
-                                                                    ar._wdtype(Wd), ctypes.byref(p))),
-                     dtype=torch.uint8, device=dev)
+                       minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo)
+    need = int(ar._lib.ar_tune_fp_target_workspace_bytes(c.out, c.inn, c.n_rows, ar._wdtype(Wd), ctypes.byref(p)))
+    if need == 0:
+        raise SystemExit("full-precision-target mode: this form does not fit its workspace limit")
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         res = ar.tune_layer_fp_target(Wd, Xq, Xt, p, workspace=ws)
     torch.cuda.synchronize()
@@ -289,7 +290,7 @@ def run_fp_target(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": c.name, "mode": "quant-aware input, full-precision target",
-                       "quantised_path_input": "target input x (1 + 0.05 N(0,1)), bf16", "algo": "gram",
+                       "quantised_path_input": "target input x (1 + 0.05 N(0,1)), bf16", "algo": args.algo,
                        "n_rows": c.n_rows, "batch_rows": c.batch_rows, "iters": c.iters,
                        "bench_step": "one ar_tune_layer_fp_target call (all iters) + ar_pack"},
             "layer_tune_s": ms / args.steps / 1e3, "final_mse": float(res.final_mse.item()),

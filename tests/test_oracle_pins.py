@@ -446,6 +446,26 @@ def test_resume_equals_uninterrupted():
     np.testing.assert_array_equal(np.concatenate([a.loss_trace, b.loss_trace]), full.loss_trace)
 
 
+def test_best_step_is_the_applied_state():
+    """The per-row loss trace and best step the oracle reports describe the state it
+    applies: the trace's row mean is the batch loss, the best loss is the trace's first
+    minimum per row, and re-running the loop for exactly best_step steps yields, on each
+    row, the live state that keep-best applied (a run of k steps ends in the state that
+    step k is evaluated at)."""
+    W = make_weight(12, 64, 0.02, "f32", seed=83)
+    X = _tiny_x(128, 64, seed=84)
+    r = oracle.tune_layer(W, X, 3, 32, False, 16, 0.01, 0.01, 32, 5)
+    np.testing.assert_allclose(r.row_loss_trace.mean(axis=1), r.loss_trace, rtol=1e-12)
+    first_min = np.argmin(r.row_loss_trace, axis=0)
+    assert np.array_equal(r.best_step, first_min)
+    assert np.array_equal(r.best_loss, r.row_loss_trace[first_min, np.arange(12)])
+    for j in range(12):
+        k = int(r.best_step[j])
+        part = oracle.tune_layer(W, X, 3, 32, False, k, 0.01, 0.01, 32, 5, want_final_mse=False)
+        assert np.array_equal(part.V[j], r.V_best[j]), j
+        assert np.array_equal(part.alpha[j], r.alpha_best[j]) and np.array_equal(part.beta[j], r.beta_best[j])
+
+
 # ---------------------------------------------------------------- schedule, pack
 
 def test_splitmix64_reference_vectors():
