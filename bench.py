@@ -14,7 +14,8 @@ epilogues per step, the final codes and the final MSE pass, and packing.
 Prints one JSON line (rank 0).  Metric: SignSGD steps per second (whole job).
 With N GPUs the layer has N times the workload's output rows; each rank tunes
 its row shard (shard.row_range) with no exchange in the loop and one all-gather
-of the results per step, so the scaling is weak.  Also the layer tune time and
+of the results per step, so the scaling is weak (NCCL; AR_BENCH_BACKEND=gloo runs
+the same ranks over gloo, sharing GPUs, to test the path).  Also the layer tune time and
 the fraction of the bf16 tensor-core peak.  ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload on the host cores.
 """
@@ -304,11 +305,24 @@ def run_ours(args):
     import signed_gradient_rounding_b200 as ar
 
     world, rank, local = _dist()
+    # One process per GPU; AR_BENCH_BACKEND=gloo (with the final gather on the host)
+    # lets the multi-rank path run where ranks share a GPU, as a test of the code path:
+    # its times then mean nothing.
+    backend = os.environ.get("AR_BENCH_BACKEND", "nccl")
+    local = local % torch.cuda.device_count() if backend == "gloo" else local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        if backend == "gloo":
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        else:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def all_max(x: float) -> float:
+        t = torch.tensor([x], dtype=torch.float64, device=dev if backend == "nccl" else "cpu")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
     from signed_gradient_rounding_b200.shard import row_range, tune_layer_sharded
 
     c = _workload(args)
@@ -372,10 +386,7 @@ def run_ours(args):
     if ar.tune_status(ws) != ar.AR_OK:
         raise RuntimeError("device status not OK after the timed region")
     mse = float(outs[4].item())
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = all_max(ms) if world > 1 else ms
 
     # End to end through the host API: pinned host inputs copied in and the
     # results copied out inside the timed region, every step (this rank's shard).
@@ -398,10 +409,10 @@ def run_ours(args):
             ar.tune_layer_host(Wh, Xh, p, device=dev)
         f1.record(stream)
         torch.cuda.synchronize()
-        ems = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device=dev)
+        ems = f0.elapsed_time(f1)
         if world > 1:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * c.iters * args.e2e_steps / (float(ems.item()) / 1e3), "unit": UNIT,
+            ems = all_max(ems)
+        e2e = {"value": world * c.iters * args.e2e_steps / (ems / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps}
 
     if world > 1:

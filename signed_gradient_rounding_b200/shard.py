@@ -31,12 +31,19 @@ def row_range(out: int, rank: int, world: int, align: int = ROW_TILE) -> tuple[i
 
 
 def _gather_rows(local: torch.Tensor, out: int, world: int, group=None) -> torch.Tensor:
-    """All-gather row slices of different lengths (padded to the longest)."""
+    """All-gather row slices of different lengths (padded to the longest).  Under the
+    gloo backend device tensors travel through host memory."""
     rows_max = max(row_range(out, r, world)[1] - row_range(out, r, world)[0] for r in range(world))
+    staged = local.is_cuda and dist.get_backend(group) == "gloo"
+    dev = local.device
+    if staged:
+        local = local.cpu()
     pad = torch.zeros((rows_max,) + tuple(local.shape[1:]), dtype=local.dtype, device=local.device)
     pad[:local.shape[0]] = local
     bufs = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(bufs, pad, group=group)
+    if staged:
+        bufs = [b.to(dev) for b in bufs]
     parts = []
     for r in range(world):
         a, b = row_range(out, r, world)

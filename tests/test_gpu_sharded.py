@@ -101,3 +101,30 @@ def test_two_ranks_on_libar_equal_one_run(name):
     assert np.array_equal(codes, ref.codes.cpu().numpy())
     assert np.array_equal(scale, ref.scale.cpu().numpy())
     assert np.array_equal(zp, ref.zero_point.cpu().numpy())
+
+
+def test_bench_two_ranks_runs_its_multi_rank_path():
+    """bench.py --gpus 2 under torchrun: both ranks tune their row shard of one
+    512-row layer, all-gather the results and reduce their times; the backend is
+    gloo (AR_BENCH_BACKEND) because both ranks share this one GPU, so the line's
+    times mean nothing here, only that the path runs and reports the whole layer."""
+    import json
+    import subprocess
+    import sys
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, AR_BENCH_BACKEND="gloo")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--gpus", "2",
+           "--steps", "2", "--warmup", "3", "--workload", "tiny", "--e2e-steps", "1"]
+    out = subprocess.run(["timeout", "-k", "30", "300", *cmd], cwd=root, env=env, capture_output=True,
+                         text=True)
+    assert out.returncode == 0, out.stderr[-3000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-3000:]
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak"
+    assert line["config"]["out"] == 512 and "2 row shards" in line["config"]["workload"]
+    assert line["value"] > 0 and line["e2e"]["value"] > 0
+    assert line["gpu_launches"] > 0
+    assert np.isfinite(line["final_mse"])
