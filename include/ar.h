@@ -44,6 +44,10 @@
  *                        outputs against the buffer sizes; a store outside is
  *                        skipped and recorded in the workspace's status word
  *                        (ar_tune_status returns AR_ECHECK).  Never traps.
+ *       AR_TAIL_SPLIT=0  the step contractions run every tile whole; by default
+ *                        the tiles of a last partial wave that fills at most half
+ *                        of the GPU's SM pairs run as two column halves each.  The
+ *                        results are bit-identical either way (a schedule switch).
  *   - Shapes: W is [out, in]; a quantisation group is `group_size` consecutive
  *     elements of one row (-1: the whole row); G = in / group_size groups per row.
  *     Q = 2^bits - 1.  Codes are unsigned in [0, Q].

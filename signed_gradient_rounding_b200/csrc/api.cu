@@ -133,6 +133,13 @@ bool checks_on() {
   return c && *c && strcmp(c, "0") != 0;
 }
 
+// AR_TAIL_SPLIT=0 turns off the column-half split of the step launches' last
+// partial wave (GemmArgs::tail_split); it changes the schedule, not the results.
+bool tail_split_on() {
+  const char* c = getenv("AR_TAIL_SPLIT");
+  return !(c && !strcmp(c, "0"));
+}
+
 #define AR_CUDA_TRY(expr)                   \
   do {                                      \
     cudaError_t e_ = (expr);                \
@@ -724,6 +731,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.mlr = mlr;
   u.gpart = P.wide ? F(L.gpart) : nullptr;
   u.gslots = P.gslots;
+  u.tail_split = tail_split_on() ? 1 : 0;
   if (checks) {
     // AR_FAULT=bounds: the epilogue is told V and D hold one element fewer than
     // they do, so the last chunk's stores are refused (and reported), not made.

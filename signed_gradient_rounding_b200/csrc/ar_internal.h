@@ -166,6 +166,11 @@ struct GemmArgs {
   // inside a group, the group's n-blocks in turn (keeps a wave's operands compact).
   int raster_m = 0;
   int64_t c_row_off = 0;
+  // Step kinds on pair tiles: tail_split asks that the tiles of a last partial wave
+  // of at most half the clusters each run as two column-half units; launch_gemm
+  // sets split_tiles (the number of such tiles, the last in tile order).
+  int tail_split = 0;
+  int split_tiles = 0;
   // kEpiStore / kEpiSumSq / kEpiDotD / kEpiUpdate (Gram loss): per-(row, n-tile) sums
   float* part = nullptr;  // [M, part_ld], part_ld >= num_n_blk * kEpiHalves (kEpiUpdate: part_out)
   int part_ld = 0;

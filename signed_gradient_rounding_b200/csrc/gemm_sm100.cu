@@ -267,6 +267,20 @@ __device__ __forceinline__ void tile_pos(const GemmArgs& a, int t, int& m_blk, i
   m_blk = t;
 }
 
+// Work unit u -> tile, and the column half it covers: the last split_tiles tiles in
+// tile order are two units each, one per column half (nh = 0, 1); every other tile
+// is one unit (nh = -1).  A launch whose tile count leaves a last partial wave of at
+// most half the clusters splits those tiles, so that wave takes half as long.
+__device__ __forceinline__ int unit_tile(int num_tiles, int split_tiles, int u, int& nh) {
+  const int whole = num_tiles - split_tiles;
+  if (u < whole) {
+    nh = -1;
+    return u;
+  }
+  nh = (u - whole) & 1;
+  return whole + ((u - whole) >> 1);
+}
+
 // ---------------------------------------------------------------------------
 // epilogues
 // ---------------------------------------------------------------------------
@@ -754,6 +768,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // each chunk accumulate afresh in accumulator 1, and the epilogue adds each chunk,
   // in fp32 round to nearest, to the tile's running sum kept in accumulator 0.
   constexpr bool kChunkable = kKind == kEpiStore && kPair && kNA == 0 && kNB == 0 && kMaj == 3;
+  // The step instances on pair tiles may split the tiles of their last partial wave
+  // into column halves (GemmArgs::split_tiles): a half unit issues N = kBN / 2 MMAs
+  // into the half's own columns of the accumulator, and only that half's epilogue
+  // warps run the epilogue, exactly as they do in a whole tile.  Each output element
+  // is the same accumulation over K either way.
+  constexpr bool kWideKind = kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide;
+  constexpr bool kSplittable =
+      kPair && kMaj == 0 && (kKind == kEpiUpdate || kKind == kEpiUpdateFp || kWideKind);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem* sm = reinterpret_cast<Smem*>(smem + C::kBarOffset);
@@ -822,6 +844,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // descriptor, and its start-address step per K16 (32 B K-major, 2 KB MN-major).
   constexpr bool kAMn = (kMaj & 1) != 0, kBMn = (kMaj & 2) != 0;
   constexpr uint32_t idesc = C::kIdesc | (kAMn ? kIdescAMn : 0u) | (kBMn ? kIdescBMn : 0u);
+  constexpr uint32_t idesc_half =
+      umma_idesc_bf16(kPair ? 2 * kBM : kBM, kBN / 2) | (kAMn ? kIdescAMn : 0u) | (kBMn ? kIdescBMn : 0u);
+  // A non-wide epilogue keeps groups inside a column half only when g <= kBN / 2.
+  const int split_tiles =
+      (kSplittable && (kWideKind || args.g <= kBN / kEpiHalves)) ? args.split_tiles : 0;
+  const int num_units = args.num_tiles + split_tiles;
   constexpr uint32_t a_kstep = kAMn ? 128u : 2u, b_kstep = kBMn ? 128u : 2u;
 
   if (warp == 0) {
@@ -831,11 +859,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
+      for (int u = unit0; ok && u < num_units; u += unit_stride) {
+        int nh;
+        const int tile = unit_tile(args.num_tiles, split_tiles, u, nh);
         int m_blk, n_blk;
         tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
         const int a_row = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM;
-        const int b_row = n_blk * kBN + args.b_row_off + (kPair ? static_cast<int>(rank) * (kBN / 2) : 0);
+        // A half unit's MMAs read the first kBN / 4 of the B rows each CTA stages
+        // (the box is loaded whole).
+        const int b_col = nh < 0 ? static_cast<int>(rank) * (kBN / 2)
+                                 : nh * (kBN / 2) + static_cast<int>(rank) * (kBN / 4);
+        const int b_row = n_blk * kBN + args.b_row_off + (kPair ? b_col : 0);
         for (int kb = 0; kb < k_blocks; ++kb) {
           const int seg = kb / args.num_k_blk;
           const int kk = kb - seg * args.num_k_blk;
@@ -895,7 +929,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       uint32_t chunk_phase = 0;  // chunked: phase of accumulator 1, the only one the MMAs use
       bool ok = true;
-      for (int tile = unit0; ok && tile < args.num_tiles; tile += unit_stride) {
+      for (int u = unit0; ok && u < num_units; u += unit_stride) {
+       int nh;
+       unit_tile(args.num_tiles, split_tiles, u, nh);
+       const uint32_t idesc_u = nh < 0 ? idesc : idesc_half;
        for (int kb0 = 0; ok && kb0 < k_blocks; kb0 += k_chunk) {
         const int buf = chunked ? 1 : acc;
         if (!mbar_wait<kPair>(&sm->tempty[buf], (chunked ? chunk_phase : acc_phase) ^ 1, abort_flag, args.status,
@@ -904,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * kBN;
+        const uint32_t d_tmem = tmem_base + buf * kBN + (nh > 0 ? kBN / 2 : 0);
         const int kb1 = min(k_blocks, kb0 + k_chunk);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait<kPair>(&sm->full[stage], phase, abort_flag, args.status, args.timeout_ns)) {
@@ -923,9 +960,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int k = 0; k < kBK / 16; ++k) {
                 const uint32_t accum = ((kb - kb0) | s | k) != 0 ? 1u : 0u;
                 if (kPair)
-                  umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
+                  umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc_u, accum);
                 else
-                  umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
+                  umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc_u, accum);
               }
             }
           } else {
@@ -935,9 +972,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < kBK / 16; ++k) {
               const uint32_t accum = ((kb - kb0) | k) != 0 ? 1u : 0u;
               if (kPair)
-                umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
+                umma_bf16_pair(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc_u, accum);
               else
-                umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc, accum);
+                umma_bf16(d_tmem, a_desc + a_kstep * k, b_desc + b_kstep * k, idesc_u, accum);
             }
           }
           if (kPair)
@@ -980,13 +1017,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t chunk_phase = 0;  // chunked: phase of accumulator 1
-    for (int tile = unit0; tile < args.num_tiles; tile += unit_stride) {
+    for (int u = unit0; u < num_units; u += unit_stride) {
+      int nh;
+      const int tile = unit_tile(args.num_tiles, split_tiles, u, nh);
+      // A half unit's accumulator holds only its half's columns: the other half's
+      // warps only hand the accumulator back.
+      const bool active = nh < 0 || nh == half;
       int m_blk, n_blk;
       tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
       const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
-      if (kKind == kEpiUpdate || kKind == kEpiUpdateFp) epi_update_prefetch<kBN, false>(args, j, n0, half);
-      if (kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide) epi_update_prefetch<kBN, true>(args, j, n0, half);
+      if ((kKind == kEpiUpdate || kKind == kEpiUpdateFp) && active) epi_update_prefetch<kBN, false>(args, j, n0, half);
+      if (kWideKind && active) epi_update_prefetch<kBN, true>(args, j, n0, half);
       if constexpr (kChunkable) {
         if (chunked) {
           // Each chunk: accumulator 1 (the chunk) added into accumulator 0 (the
@@ -1046,16 +1088,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait<kPair>(&sm->tfull[acc], acc_phase, abort_flag, args.status, args.timeout_ns, false)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
-      if constexpr (kKind == kEpiUpdate)
-        epi_update<kBN, false>(args, t_row, j, n0, n_blk, half);
-      else if constexpr (kKind == kEpiUpdateFp)
-        epi_update<kBN, true>(args, t_row, j, n0, n_blk, half);
-      else if constexpr (kKind == kEpiUpdateWide)
-        epi_update_wide<kBN, false>(args, t_row, j, n0, n_blk, half);
-      else if constexpr (kKind == kEpiUpdateFpWide)
-        epi_update_wide<kBN, true>(args, t_row, j, n0, n_blk, half);
-      else
-        epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk, half);
+      if (active) {
+        if constexpr (kKind == kEpiUpdate)
+          epi_update<kBN, false>(args, t_row, j, n0, n_blk, half);
+        else if constexpr (kKind == kEpiUpdateFp)
+          epi_update<kBN, true>(args, t_row, j, n0, n_blk, half);
+        else if constexpr (kKind == kEpiUpdateWide)
+          epi_update_wide<kBN, false>(args, t_row, j, n0, n_blk, half);
+        else if constexpr (kKind == kEpiUpdateFpWide)
+          epi_update_wide<kBN, true>(args, t_row, j, n0, n_blk, half);
+        else
+          epi_rows<kKind, kBN>(args, t_row, j, n0, n_blk, half);
+      }
       tc_fence_before();
       if (kPair) {
         __syncwarp();
@@ -1157,11 +1201,21 @@ cudaError_t launch_kind(const GemmMaps& m, const GemmArgs& args, int num_sms, cu
       if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
       if (dev >= 0 && dev < 64) resident[dev].store(max_pairs, std::memory_order_relaxed);
     }
-    int pairs = args.num_tiles < num_sms / 2 ? args.num_tiles : num_sms / 2;
-    if (pairs > max_pairs) pairs = max_pairs;
-    if (pairs <= 0) return cudaSuccess;
+    int pairs_max = num_sms / 2 < max_pairs ? num_sms / 2 : max_pairs;
+    if (pairs_max <= 0 || args.num_tiles <= 0) return cudaSuccess;
+    // A last partial wave of at most half the clusters: its tiles become two
+    // column-half units each (the kernel ignores the request where it cannot split).
+    GemmArgs a = args;
+    a.split_tiles = 0;
+    const int tail = args.num_tiles % pairs_max;
+    constexpr bool kWideKind = kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide;
+    constexpr bool kSplitKind = kMaj == 0 && (kKind == kEpiUpdate || kKind == kEpiUpdateFp || kWideKind);
+    const bool can_split = kSplitKind && (kWideKind || args.g <= kBN / kEpiHalves);
+    if (args.tail_split && can_split && tail > 0 && 2 * tail <= pairs_max) a.split_tiles = tail;
+    const int units = a.num_tiles + a.split_tiles;
+    const int pairs = units < pairs_max ? units : pairs_max;
     cfg.gridDim = dim3(2 * pairs, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, fn, m.a0, m.a1, m.b0, m.b1, args);
+    e = cudaLaunchKernelEx(&cfg, fn, m.a0, m.a1, m.b0, m.b1, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
