@@ -70,3 +70,18 @@ def test_group_size_override_names_the_workload():
     assert c.group_size == 64 and " g64" in c.name
     c = bench._workload(argparse.Namespace(workload="q_proj", group_size=None))
     assert c is bench.WORKLOADS["q_proj"]
+
+
+def test_clock_summary_parses_samples():
+    """The clocks object: median SM clock and power draw, the max clock, and every throttle
+    reason seen active in any sample (nvidia-smi csv, noheader, nounits)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.lines = ["0, 1500, 1965, 980.5, Not Active, Not Active, Not Active, Active",
+               "0, 1440, 1965, 995.0, Not Active, Not Active, Not Active, Active",
+               "0, 1470, 1965, 990.0, Not Active, Not Active, Not Active, Not Active",
+               "garbage"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1470 and s["sm_max_mhz"] == 1965 and s["power_w"] == 990.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
