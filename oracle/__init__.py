@@ -36,9 +36,10 @@ symmetric mode s = 2*alpha*amax/Q with zp = 2^(b-1); alpha, beta clamped to
 [0.5, 1]; straight-through identity through every rint (zp's included), masked
 by clamps with inclusive bounds; sign(0) = 0; one calibration block per step
 chosen by a SplitMix64-driven Fisher-Yates permutation per epoch; the state
-with the lowest step loss is applied at the end (keep_best, the default; the
-page's listing applies the last state, available as keep_best=False); group_size
--1 is one group per row.
+with the lowest step loss is applied at the end, chosen per output row
+(keep_best, the default) or once for the whole layer (keep_best=2); the page's
+listing applies the last state, available as keep_best=False; group_size -1 is
+one group per row.
 """
 from .autoround import (  # noqa: F401
     TuneResult,

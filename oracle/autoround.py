@@ -341,7 +341,7 @@ class TuneResult:
 
 def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: float,
                minmax_lr: float, batch_rows: int, seed: int, minmax_shrink: float = 1.0,
-               keep_best: bool = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
+               keep_best: bool | int = True, V0=None, alpha0=None, beta0=None, start_step: int = 0,
                best0=None, want_final_mse: bool = True, init: str = "minmax", X_target=None,
                grad_jitter=None) -> TuneResult:
     """SignSGD tuning of one linear layer.
@@ -366,7 +366,11 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     of the others, and is never worse than one layer-wide choice.  Step 0, the
     min-max RTN state, is a candidate, so with one full batch the result is never
     worse than RTN.  keep_best=False applies the last state, as the page's
-    listing does.  The comparison is strict (a tie keeps the earlier state).
+    listing does.  keep_best=2 makes one layer-wide choice instead: the state of
+    the step whose layer batch loss (the sum over rows of the row losses) was
+    lowest, every row together, as the page's loop would with its ``total_loss``
+    tracked across steps.  The comparison is strict (a tie keeps the earlier
+    state).  In that mode every entry of ``best_loss`` holds the layer's best.
 
     W: [out, in] fp32 values (or bf16 bit patterns); X: [n, in] bf16-exact values.
     ``start_step`` continues the block schedule of an interrupted run, with the
@@ -411,12 +415,14 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
     V = np.zeros_like(W) if V0 is None else _to_f32(V0).copy()
     alpha = p0.copy() if alpha0 is None else _to_f32(alpha0).copy()
     beta = p0.copy() if beta0 is None else _to_f32(beta0).copy()
+    layer_wide = keep_best == 2 and keep_best is not True
     if best0 is None:
         best_loss = np.full(out, np.inf)
         V_best, a_best, b_best = V.copy(), alpha.copy(), beta.copy()
     else:
         best_loss = np.asarray(best0[0], dtype=F64).copy()
         V_best, a_best, b_best = (_to_f32(x).copy() for x in best0[1:])
+    best_layer = float(best_loss[0]) if (layer_wide and out > 0) else np.inf
 
     sched = block_schedule(n // batch_rows, start_step + iters, seed)[start_step:]
     W64 = W.astype(F64)
@@ -442,8 +448,17 @@ def tune_layer(W, X, bits: int, group_size: int, sym: bool, iters: int, lr: floa
         row_loss = st.row_loss
         row_trace[t] = row_loss
         trace[t] = float(np.sum(row_loss)) / out
-        better = row_loss < best_loss
-        best_loss = np.where(better, row_loss, best_loss)
+        if layer_wide:
+            layer_loss = float(np.sum(row_loss))
+            improved = layer_loss < best_layer
+            if improved:
+                best_layer = layer_loss
+            better = np.full(out, improved)
+            row_best = np.full(out, layer_loss)
+        else:
+            better = row_loss < best_loss
+            row_best = row_loss
+        best_loss = np.where(better, row_best, best_loss)
         best_step[better] = start_step + t
         V_best[better] = V[better]
         a_best[better] = alpha[better]

@@ -194,3 +194,21 @@ def _tune_shrink_alpha_only(W, X, bits, group_size, sym, iters, lr, minmax_lr, b
 def test_minmax_shrink_mistakes_are_caught(monkeypatch, slip):
     _plant(monkeypatch, "tune_layer", slip)
     assert _caught(lambda: pins.test_minmax_shrink_worked_example(0), lambda: pins.test_minmax_shrink_worked_example(1))
+
+
+def _tune_layer_wide_as_per_row(*args, **kw):
+    if kw.get("keep_best") == 2:
+        kw["keep_best"] = True                                           # the layer choice made per row
+    return _orig_tune(*args, **kw)
+
+
+def _tune_layer_wide_as_last(*args, **kw):
+    if kw.get("keep_best") == 2:
+        kw["keep_best"] = False                                          # the last state applied
+    return _orig_tune(*args, **kw)
+
+
+@pytest.mark.parametrize("slip", [_tune_layer_wide_as_per_row, _tune_layer_wide_as_last])
+def test_layer_wide_keep_best_mistakes_are_caught(monkeypatch, slip):
+    _plant(monkeypatch, "tune_layer", slip)
+    assert _caught(lambda: pins.test_layer_wide_keep_best_applies_one_step())

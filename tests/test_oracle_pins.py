@@ -466,6 +466,41 @@ def test_best_step_is_the_applied_state():
         assert np.array_equal(part.alpha[j], r.alpha_best[j]) and np.array_equal(part.beta[j], r.beta_best[j])
 
 
+def test_layer_wide_keep_best_applies_one_step():
+    """keep_best=2: one step for every row, the first minimum of the layer's batch loss
+    (the trace), and its state is the live state after exactly that many steps, so a
+    keep_best=False run of best_step steps gives the same codes, scales and zero-points.
+    The per-row choice on the same case picks different steps for different rows (so the
+    case separates the two modes), and with one row the two modes coincide."""
+    W = make_weight(12, 64, 0.02, "f32", seed=83)
+    X = _tiny_x(128, 64, seed=84)
+    args = (W, X, 3, 32, False, 16, 0.01, 0.01, 32, 5)
+    lw = oracle.tune_layer(*args, keep_best=2)
+    per_row = oracle.tune_layer(*args)
+    assert len(set(per_row.best_step.tolist())) > 1
+    k = int(np.argmin(lw.loss_trace))
+    assert np.all(lw.best_step == k)
+    np.testing.assert_allclose(lw.best_loss, lw.row_loss_trace[k].sum(), rtol=1e-12)
+    part = oracle.tune_layer(*args[:5], k, *args[6:], keep_best=False)
+    assert np.array_equal(lw.codes, part.codes)
+    assert np.array_equal(lw.scale, part.scale) and np.array_equal(lw.zero_point, part.zero_point)
+    one = (W[:1], X, 3, 32, False, 16, 0.01, 0.01, 32, 5)
+    a, b = oracle.tune_layer(*one, keep_best=2), oracle.tune_layer(*one)
+    assert np.array_equal(a.codes, b.codes) and np.array_equal(a.best_step, b.best_step)
+
+
+def test_layer_wide_keep_best_resumes():
+    """A layer-wide run split at step k (live and best state handed over) equals one run."""
+    W = make_weight(8, 64, 0.02, "f32", seed=85)
+    X = _tiny_x(128, 64, seed=86)
+    full = oracle.tune_layer(W, X, 2, 32, False, 20, 0.01, 0.01, 32, 7, keep_best=2, want_final_mse=False)
+    first = oracle.tune_layer(W, X, 2, 32, False, 9, 0.01, 0.01, 32, 7, keep_best=2, want_final_mse=False)
+    rest = oracle.tune_layer(W, X, 2, 32, False, 11, 0.01, 0.01, 32, 7, keep_best=2, want_final_mse=False,
+                             V0=first.V, alpha0=first.alpha, beta0=first.beta, start_step=9,
+                             best0=(first.best_loss, first.V_best, first.alpha_best, first.beta_best))
+    assert np.array_equal(rest.codes, full.codes) and np.array_equal(rest.best_loss, full.best_loss)
+
+
 # ---------------------------------------------------------------- schedule, pack
 
 def test_splitmix64_reference_vectors():
