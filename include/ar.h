@@ -105,8 +105,7 @@ typedef struct {
   float lr;              /* step of V, >= 0 (0.005) */
   float minmax_lr;       /* step of alpha and beta; < 0 means "same as lr" */
   float minmax_shrink;   /* initial alpha = beta (1.0) */
-  int32_t keep_best;     /* 1: apply, per output row, the state of its lowest batch
-                            loss (step 0 = RTN state included); 0: the last state */
+  int32_t keep_best;     /* ar_keep_best: which state is applied (1: per row) */
   int64_t batch_rows;    /* rows of X per step; n_rows must be a multiple */
   uint64_t seed;         /* seeds the calibration-block schedule */
   int64_t start_step;    /* first step index (resume); 0 for a fresh run */
@@ -131,6 +130,21 @@ typedef struct {
  *                   library's reading of it.) */
 typedef enum { AR_INIT_MINMAX = 0, AR_INIT_MSE = 1 } ar_init;
 
+/* Which state ar_tune_layer applies at the end ("[llm-compressor] AutoRound ...",
+ * "on_event with SEQUENTIAL_EPOCH_END": the loop computes each step's loss,
+ * total_loss, and applies the final V).  A step's batch loss is taken at the state
+ * the step starts from; step 0's state (the min-max or MSE start) is a candidate.
+ *   AR_KEEP_LAST:       the state after the last step (the page's listing).
+ *   AR_KEEP_BEST_ROW:   per output row, the state of the step with that row's
+ *                       lowest batch loss mean_b (Y' - Y)_bj^2 (fp32, strictly
+ *                       lower; the default).  Rows stay independent.
+ *   AR_KEEP_BEST_LAYER: for the whole layer, the state of the step whose layer
+ *                       batch loss, the sum over rows of the row losses (taken in
+ *                       fp64 in a fixed order), was strictly lowest; every row
+ *                       takes that step.  ar_tune_state.best_loss then holds the
+ *                       layer's best in every entry. */
+typedef enum { AR_KEEP_LAST = 0, AR_KEEP_BEST_ROW = 1, AR_KEEP_BEST_LAYER = 2 } ar_keep_best;
+
 /* Optional caller-owned tuning state (device memory, fp32).  Lets a caller
  * inspect the learned variables, and resume: a run of k steps followed by a run
  * with start_step = k and initialized = 1 equals one run of both. */
@@ -138,7 +152,8 @@ typedef struct {
   float* V;            /* [out, in]  rounding offsets, in [-0.5, 0.5] */
   float* alpha;        /* [out, G]   clip factor of the maximum, in [0.5, 1] */
   float* beta;         /* [out, G]   clip factor of the minimum, in [0.5, 1] */
-  float* best_loss;    /* [out]      per row, lowest batch loss seen (+inf if none) */
+  float* best_loss;    /* [out]      per row, lowest batch loss seen (+inf if none);
+                          AR_KEEP_BEST_LAYER: the layer's lowest, in every entry */
   float* V_best;       /* [out, in]  per row, the state at that row's best step */
   float* alpha_best;   /* [out, G] */
   float* beta_best;    /* [out, G] */

@@ -26,6 +26,8 @@ AR_ALGO_AUTO, AR_ALGO_DIRECT, AR_ALGO_GRAM = 0, 1, 2
 ALGOS = {"auto": AR_ALGO_AUTO, "direct": AR_ALGO_DIRECT, "gram": AR_ALGO_GRAM}
 AR_INIT_MINMAX, AR_INIT_MSE = 0, 1
 INITS = {"minmax": AR_INIT_MINMAX, "mse": AR_INIT_MSE}
+AR_KEEP_LAST, AR_KEEP_BEST_ROW, AR_KEEP_BEST_LAYER = 0, 1, 2
+KEEPS = {"last": AR_KEEP_LAST, "row": AR_KEEP_BEST_ROW, "layer": AR_KEEP_BEST_LAYER}
 
 # Every exported symbol of include/ar.h.
 EXPORTS = ("ar_version", "ar_status_string", "ar_rtn", "ar_fake_quant", "ar_pack",
@@ -250,8 +252,10 @@ def make_params(bits=4, group_size=128, sym=False, iters=200, lr=0.005, minmax_l
                 keep_best=True, batch_rows=16384, seed=0, start_step=0, algo="auto", split=True,
                 init="minmax") -> TuneParams:
     """ar_tune_params; algo is "auto", "direct" or "gram" (ar_algo in include/ar.h);
-    init is "minmax" or "mse" (ar_init)."""
-    return TuneParams(bits, group_size, int(sym), iters, lr, minmax_lr, minmax_shrink, int(keep_best),
+    init is "minmax" or "mse" (ar_init); keep_best is True / "row", False / "last" or
+    "layer" (ar_keep_best)."""
+    keep = KEEPS[keep_best] if isinstance(keep_best, str) else int(keep_best)
+    return TuneParams(bits, group_size, int(sym), iters, lr, minmax_lr, minmax_shrink, keep,
                       batch_rows, seed, start_step, ALGOS[algo] if isinstance(algo, str) else int(algo),
                       int(split), INITS[init] if isinstance(init, str) else int(init))
 

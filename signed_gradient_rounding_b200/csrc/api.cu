@@ -167,6 +167,7 @@ ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune
   if (p->start_step < 0) return AR_EINVAL;
   if (p->algo < AR_ALGO_AUTO || p->algo > AR_ALGO_GRAM) return AR_EINVAL;
   if (p->init != AR_INIT_MINMAX && p->init != AR_INIT_MSE) return AR_EINVAL;
+  if (p->keep_best < AR_KEEP_LAST || p->keep_best > AR_KEEP_BEST_LAYER) return AR_EINVAL;
   if (out == 0 || in == 0) return AR_OK;
   if (!group_ok(in, p->group_size)) return AR_EINVAL;
   if (p->batch_rows <= 0 || n_rows < p->batch_rows || n_rows % p->batch_rows != 0) return AR_EINVAL;
@@ -290,7 +291,10 @@ struct Layout {
       dX_hi, dX_lo, Mt_hi, Mt_lo, Cc_hi, Cc_lo, Cs, e, es, epart, Wp_hi, Wp_lo,
       // direct form with a full-precision target: E^T = W dX^T for every block, [out, n]
       // as a bf16 pair (block b in columns b*B ..), added to the residual
-      E_hi, E_lo, total;
+      E_hi, E_lo,
+      // layer-wide keep-best: the best loss (fp64), the step's decision, the
+      // reduction's ticket and its per-range sums
+      layer, total;
 };
 
 Layout make_layout(const Plan& P) {
@@ -306,6 +310,7 @@ Layout make_layout(const Plan& P) {
   const bool gram = P.algo == AR_ALGO_GRAM;
   const int64_t nparts = std::max(std::max(P.nparts_res, P.nparts_upd), P.nparts_fin);
   L.status = take(256);
+  L.layer = take(16 + kLayerBlocks * 8);
   L.D_hi = take(elems * 2);
   L.D_lo = take(elems * 2);
   // The Gram form reads D_t and writes D_{t+1} in the same launch: two buffers.
@@ -517,6 +522,32 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     launches += 1;
   }
 
+  // Layer-wide keep-best: after each step's partials are complete, one small
+  // reduction takes the layer's decision, which the launch that judges the step
+  // (and the wide-group finish, and the last step's finalize) apply to every row.
+  const bool layer_best = p->keep_best == AR_KEEP_BEST_LAYER && iters > 0;
+  LayerBestArgs lb;
+  lb.out = out;
+  lb.inv_batch = 1.0f / static_cast<float>(B);
+  lb.best = reinterpret_cast<double*>(ws + L.layer);
+  lb.flag = reinterpret_cast<int*>(ws + L.layer + 8);
+  lb.ticket = reinterpret_cast<unsigned int*>(ws + L.layer + 12);
+  lb.blocksum = reinterpret_cast<double*>(ws + L.layer + 16);
+  lb.best_rows = best_loss;
+  if (layer_best) {
+    lb.init = 1;  // the best so far: best_loss[0] (+inf on a fresh state)
+    AR_CUDA_TRY(launch_layer_best(lb, st));
+    lb.init = 0;
+    ++launches;
+  }
+  auto judge_layer = [&](const float* parts, int64_t nparts) -> cudaError_t {
+    if (!layer_best) return cudaSuccess;
+    lb.part = parts;
+    lb.nparts = static_cast<int>(nparts);
+    ++launches;
+    return launch_layer_best(lb, st);
+  };
+
   // Full-precision-target mode: the block sums start at zero; an fp32 W is held as
   // a bf16 pair for its contractions.
   const bool fpt = P.fp_target;
@@ -727,6 +758,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.bits = p->bits;
   u.sym = p->sym != 0;
   u.keep_best = p->keep_best != 0;
+  u.layer_flag = layer_best ? lb.flag : nullptr;
   u.lr = p->lr;
   u.mlr = mlr;
   u.gpart = P.wide ? F(L.gpart) : nullptr;
@@ -761,6 +793,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     f.beta_best = u.beta_best;
     f.judged = u.part_in != nullptr;
     f.keep_best = u.keep_best;
+    f.layer_flag = u.layer_flag;
     f.snap_prev = u.snap_prev;
     f.best_in = u.best_in;
     f.best_out = u.best_out;
@@ -836,6 +869,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       if (fault == kFaultLaunch) return AR_ECUDA;
       AR_CUDA_TRY(launch_gemm(upd_kind, P.bn_upd, m[cur], u, sms, st));
       AR_CUDA_TRY(finish_groups());
+      AR_CUDA_TRY(judge_layer(part[cur], P.nparts_upd));  // this step's loss, judged by the next launch
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
       ++launches;
       if (t > 0) std::swap(best_cur, best_next);
@@ -850,6 +884,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       f.G = static_cast<int>(P.G);
       f.inv_batch = 1.0f / static_cast<float>(B);
       f.keep_best = p->keep_best != 0;
+      f.layer_flag = u.layer_flag;  // the last step's decision, taken after its launch
       f.best_in = best_cur;
       f.best_out = best_next;
       f.rowloss = rowloss + static_cast<int64_t>(iters - 1) * out;
@@ -921,6 +956,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       if (fault == kFaultLaunch) return AR_ECUDA;
       AR_CUDA_TRY(launch_gemm(kEpiStore, P.bn_res, mr, r, sms, st));
       if (timer) AR_CUDA_TRY(cudaEventRecord(timer->ev[3 * t + 1], st));
+      AR_CUDA_TRY(judge_layer(part[0], P.nparts_res));  // this step's loss, judged by its update
       AR_CUDA_TRY(make_tmap_bf16(&mu.b0, X + b0 * in, B, in, 64));
       mu.b1 = mu.b0;
       u.best_in = best_cur;
@@ -935,7 +971,7 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   }
 
   if (iters > 0) {
-    if (p->keep_best && best_cur != best_loss)
+    if (p->keep_best == AR_KEEP_BEST_ROW && best_cur != best_loss)
       AR_CUDA_TRY(cudaMemcpyAsync(best_loss, best_cur, static_cast<size_t>(out) * 4, cudaMemcpyDeviceToDevice, st));
     if (live != 0) {  // hand the live state back in buffer 0
       AR_CUDA_TRY(cudaMemcpyAsync(Vb[0], Vb[live], elems * 4, cudaMemcpyDeviceToDevice, st));

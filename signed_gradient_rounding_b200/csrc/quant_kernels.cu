@@ -276,7 +276,9 @@ __global__ void finalize_best_kernel(FinalizeBestArgs a) {
   const float* p = a.part + j * a.nparts;
   for (int q = 0; q < a.nparts; ++q) L += p[q];  // same order as the update epilogue
   bool better = false;
-  if (a.keep_best) {
+  if (a.keep_best && a.layer_flag) {
+    better = *a.layer_flag != 0;
+  } else if (a.keep_best) {
     const float mean = L * a.inv_batch;
     better = mean < a.best_in[j];
     if (lane == 0) a.best_out[j] = better ? mean : a.best_in[j];
@@ -312,7 +314,8 @@ __global__ void group_finish_kernel(GroupFinishArgs a) {
   const float al = a.alpha_in[grp], be = a.beta_in[grp];
   const float al_n = clip_step(al, a.mlr, dal);
   const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
-  const bool better = a.judged && a.keep_best && a.best_out[j] < a.best_in[j];
+  const bool better =
+      a.judged && a.keep_best && (a.layer_flag ? *a.layer_flag != 0 : a.best_out[j] < a.best_in[j]);
   __syncwarp();  // every lane has read alpha_in, beta_in (they may alias the outputs)
   if (lane == 0 && in_bounds(grp, 1, a.chk_groups, a.status)) {
     if (better && !a.snap_prev) {
@@ -451,6 +454,64 @@ cudaError_t launch_silu_mul(const __nv_bfloat16* a, const __nv_bfloat16* b, int6
 cudaError_t launch_diag_sum(const float* diag, int nb, int64_t in, float* dsum, cudaStream_t stream) {
   if (in == 0) return cudaSuccess;
   diag_sum_kernel<<<static_cast<unsigned>((in + 255) / 256), 256, 0, stream>>>(diag, nb, in, dsum);
+  return cudaGetLastError();
+}
+
+// kLayerBlocks blocks of 256 threads; block b sums rows [b * rpb, (b + 1) * rpb).
+__global__ void layer_best_kernel(LayerBestArgs a) {
+  __shared__ double red[256];
+  __shared__ int last_block;
+  __shared__ int improved;
+  const int tid = threadIdx.x;
+  if (a.init) {
+    if (blockIdx.x == 0 && tid == 0) {
+      *a.best = a.out > 0 ? static_cast<double>(a.best_rows[0]) : static_cast<double>(INFINITY);
+      *a.flag = 0;
+      *a.ticket = 0u;
+    }
+    return;
+  }
+  const int64_t rpb = (a.out + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rpb;
+  const int64_t r1 = min(a.out, r0 + rpb);
+  double acc = 0.0;
+  for (int64_t j = r0 + tid; j < r1; j += blockDim.x) {
+    float L = 0.0f;
+    const float* p = a.part + j * a.nparts;
+    for (int q = 0; q < a.nparts; ++q) L += p[q];  // as the epilogues sum a row
+    acc += static_cast<double>(L * a.inv_batch);
+  }
+  red[tid] = acc;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (tid < w) red[tid] += red[tid + w];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    a.blocksum[blockIdx.x] = red[0];
+    __threadfence();
+    last_block = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last_block) return;
+  if (tid == 0) {
+    __threadfence();
+    double total = 0.0;
+    for (unsigned int b = 0; b < gridDim.x; ++b) total += __ldcg(a.blocksum + b);
+    improved = total < *a.best;
+    *a.flag = improved;
+    if (improved) *a.best = total;
+    red[0] = total;
+    *a.ticket = 0u;
+  }
+  __syncthreads();
+  if (!improved) return;
+  const float v = static_cast<float>(red[0]);
+  for (int64_t j = tid; j < a.out; j += blockDim.x) a.best_rows[j] = v;
+}
+
+cudaError_t launch_layer_best(const LayerBestArgs& a, cudaStream_t stream) {
+  layer_best_kernel<<<a.init ? 1 : kLayerBlocks, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -73,6 +73,11 @@ def test_tune_validation(ar):
     assert call(64, 250, 1024, batch_rows=512, group_size=-1) == ar.AR_EUNSUPPORTED   # in % 32
     assert call(0, 256, 1024, batch_rows=512, group_size=64) == ar.AR_OK              # empty layer
     assert call(64, 256, 1024, batch_rows=512, group_size=64, init=2) == ar.AR_EINVAL  # unknown init
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, keep_best=3) == ar.AR_EINVAL  # unknown keep-best
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, keep_best=-1) == ar.AR_EINVAL
+    assert ar.make_params(keep_best="layer").keep_best == ar.AR_KEEP_BEST_LAYER
+    assert ar.make_params(keep_best=True).keep_best == ar.AR_KEEP_BEST_ROW
+    assert ar.make_params(keep_best="last").keep_best == ar.AR_KEEP_LAST
     # too small a workspace
     p = ar.make_params(batch_rows=512, group_size=64)
     assert lib.ar_tune_layer(dummy, 1, 64, 256, dummy, 1024, ctypes.byref(p), None, dummy, 1024,

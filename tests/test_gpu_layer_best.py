@@ -1,0 +1,146 @@
+"""Layer-wide keep-best (AR_KEEP_BEST_LAYER) on the GPU against the oracle.
+
+The loop in "[llm-compressor] AutoRound ...", "on_event with SEQUENTIAL_EPOCH_END"
+computes one step loss for the whole layer (total_loss); tracking its lowest value
+picks one step, and every row takes that step's state.  Checked here:
+- the step the GPU chose is the first minimum of the layer loss recomputed on the
+  host from the GPU's own per-row losses (ar_tune_row_losses), shown by a
+  keep_best = 0 run of exactly that many steps ending in the same codes, scales and
+  zero-points (the runs share their first steps bit for bit);
+- against the oracle over every row: the same chosen step wherever the oracle's
+  two lowest layer losses are not within 1e-6 of each other, at most 0.5% of the
+  codes differing and the final MSE within 2%;
+- resume at a step in the middle equals one run, bit for bit;
+- the full-size q_proj layer (Gram form) makes the same host-checked choice.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import Q_PROJ_7B, TINY, make_activations, make_activations_cuda, make_weight
+
+pytestmark = pytest.mark.gpu
+
+CODE_TOL = 0.005
+MSE_RTOL = 0.02
+
+CASES = {
+    "tiny_full_batch": dict(out=TINY.out, inn=TINY.inn, n=TINY.n_rows, B=TINY.batch_rows, bits=4, g=64,
+                            sym=False, iters=TINY.iters, wdt="f32", kind="tiny"),
+    "multiblock_bf16": dict(out=200, inn=384, n=1536, B=512, bits=3, g=128, sym=False, iters=30, wdt="bf16",
+                            kind="llm"),
+    "per_channel_sym": dict(out=130, inn=320, n=1024, B=512, bits=4, g=-1, sym=True, iters=30, wdt="bf16",
+                            kind="llm"),
+}
+
+
+@pytest.fixture(scope="module")
+def ar():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import signed_gradient_rounding_b200 as ar
+    return ar
+
+
+def _inputs(c, seed):
+    W = make_weight(c["out"], c["inn"], 0.02, c["wdt"], seed=seed)
+    X = make_activations(c["n"], c["inn"], c["kind"], seed=seed)
+    return W, X
+
+
+def _dev(W, X, wdt):
+    Wt = torch.from_numpy(W)
+    return (Wt.to(torch.bfloat16) if wdt == "bf16" else Wt).cuda(), torch.from_numpy(X).to(torch.bfloat16).cuda()
+
+
+def _params(ar, c, keep_best, iters=None, algo="auto"):
+    return ar.make_params(bits=c["bits"], group_size=c["g"], sym=c["sym"], iters=c["iters"] if iters is None else iters,
+                          lr=0.005, minmax_lr=0.005, batch_rows=c["B"], seed=4, keep_best=keep_best, algo=algo)
+
+
+def _host_choice(row_losses: np.ndarray, B: int) -> tuple[int, float]:
+    """First minimum of the layer loss sum_j fp32(L_j * fp32(1/B)), summed in fp64, and
+    the relative gap to the next-lowest step."""
+    per_row = row_losses.astype(np.float32) * np.float32(1.0 / B)
+    layer = per_row.astype(np.float64).sum(axis=1)
+    k = int(np.argmin(layer))
+    rest = np.delete(layer, k)
+    gap = float((rest.min() - layer[k]) / abs(layer[k])) if rest.size else np.inf
+    return k, gap
+
+
+def _check_choice(ar, Wd, Xd, p_layer, res, n, B, algo):
+    out, inn = Wd.shape
+    rl = ar.tune_row_losses(res.workspace, out, inn, n, p_layer).cpu().numpy()
+    k, _ = _host_choice(rl, B)
+    p_trunc = ar.make_params(bits=p_layer.bits, group_size=p_layer.group_size, sym=bool(p_layer.sym), iters=k,
+                             lr=p_layer.lr, minmax_lr=p_layer.minmax_lr, batch_rows=B, seed=p_layer.seed,
+                             keep_best=False, algo=algo)
+    trunc = ar.tune_layer(Wd, Xd, p_trunc, want_final_mse=False)
+    assert ar.tune_status(trunc.workspace) == ar.AR_OK
+    assert torch.equal(trunc.codes, res.codes), f"layer choice is not step {k}"
+    assert torch.equal(trunc.scale, res.scale) and torch.equal(trunc.zero_point, res.zero_point)
+    return k
+
+
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_layer_best_against_oracle(ar, name, algo):
+    c = CASES[name]
+    W, X = _inputs(c, seed=17)
+    Wd, Xd = _dev(W, X, c["wdt"])
+    p = _params(ar, c, "layer", algo=algo)
+    res = ar.tune_layer(Wd, Xd, p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    k = _check_choice(ar, Wd, Xd, p, res, c["n"], c["B"], algo)
+    ref = oracle.tune_layer(W, X, c["bits"], c["g"], c["sym"], c["iters"], 0.005, 0.005, c["B"], 4, keep_best=2)
+    k_ref = int(ref.best_step[0])
+    layer = np.sort(ref.row_loss_trace.sum(axis=1))
+    tie = layer.size > 1 and (layer[1] - layer[0]) <= 1e-6 * abs(layer[0])
+    if not tie:
+        assert k == k_ref, f"GPU chose step {k}, the oracle step {k_ref}"
+    frac = float(np.mean(res.codes.cpu().numpy() != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
+
+
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_layer_best_resume(ar, algo):
+    c = CASES["multiblock_bf16"]
+    W, X = _inputs(c, seed=23)
+    Wd, Xd = _dev(W, X, c["wdt"])
+    full_state = ar.TuneState.empty(c["out"], c["inn"], c["g"])
+    full = ar.tune_layer(Wd, Xd, _params(ar, c, "layer", algo=algo), state=full_state, want_final_mse=False)
+    st = ar.TuneState.empty(c["out"], c["inn"], c["g"])
+    ar.tune_layer(Wd, Xd, _params(ar, c, "layer", iters=13, algo=algo), state=st, want_final_mse=False)
+    st.initialized = True
+    p2 = _params(ar, c, "layer", iters=c["iters"] - 13, algo=algo)
+    p2.start_step = 13
+    rest = ar.tune_layer(Wd, Xd, p2, state=st, want_final_mse=False)
+    torch.cuda.synchronize()
+    assert torch.equal(rest.codes, full.codes)
+    for name in ("V", "alpha", "beta", "V_best", "alpha_best", "beta_best", "best_loss"):
+        assert torch.equal(getattr(st, name), getattr(full_state, name)), name
+    assert bool(torch.all(full_state.best_loss == full_state.best_loss[0]))
+
+
+def test_layer_best_q_proj_full_size(ar):
+    """The benchmark's layer with one layer-wide choice: the GPU takes the step the host
+    finds from its per-row losses; printed beside the per-row choice's final MSE."""
+    c = Q_PROJ_7B
+    Wd = torch.from_numpy(make_weight(c.out, c.inn, c.w_std, c.w_dtype, seed=0)).to(torch.bfloat16).cuda()
+    Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device="cuda")
+    p = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
+                       batch_rows=c.batch_rows, seed=0, keep_best="layer", algo="gram")
+    res = ar.tune_layer(Wd, Xd, p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    k = _check_choice(ar, Wd, Xd, p, res, c.n_rows, c.batch_rows, "gram")
+    mse_layer = float(res.final_mse.item())
+    del res
+    torch.cuda.empty_cache()
+    p_row = ar.make_params(bits=c.bits, group_size=c.group_size, iters=c.iters, lr=c.lr, minmax_lr=c.minmax_lr,
+                           batch_rows=c.batch_rows, seed=0, keep_best=True, algo="gram")
+    row = ar.tune_layer(Wd, Xd, p_row)
+    print(f"\nq_proj layer-wide keep-best: step {k}, final MSE {mse_layer:.6g}; "
+          f"per-row keep-best final MSE {float(row.final_mse.item()):.6g}")
+    assert np.isfinite(mse_layer) and 0 <= k < c.iters
