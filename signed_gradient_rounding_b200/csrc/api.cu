@@ -12,6 +12,7 @@
 #include "../../include/ar.h"
 #include "ar_device.cuh"
 #include "ar_internal.h"
+#include "ar_layer_best.h"
 
 namespace ar {
 
@@ -292,9 +293,9 @@ struct Layout {
       // direct form with a full-precision target: E^T = W dX^T for every block, [out, n]
       // as a bf16 pair (block b in columns b*B ..), added to the residual
       E_hi, E_lo,
-      // layer-wide keep-best: the best loss (fp64), the step's decision, the
-      // reduction's ticket and its per-range sums
-      layer, total;
+      // layer-wide keep-best: the best loss (fp64), the reduction's ticket and its
+      // per-range sums; the per-row thresholds and the judging launch's scratch
+      layer, layer_rows, total;
 };
 
 Layout make_layout(const Plan& P) {
@@ -311,6 +312,7 @@ Layout make_layout(const Plan& P) {
   const int64_t nparts = std::max(std::max(P.nparts_res, P.nparts_upd), P.nparts_fin);
   L.status = take(256);
   L.layer = take(16 + kLayerBlocks * 8);
+  L.layer_rows = take(static_cast<size_t>(P.out) * 2 * 4);
   L.D_hi = take(elems * 2);
   L.D_lo = take(elems * 2);
   // The Gram form reads D_t and writes D_{t+1} in the same launch: two buffers.
@@ -523,17 +525,20 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   }
 
   // Layer-wide keep-best: after each step's partials are complete, one small
-  // reduction takes the layer's decision, which the launch that judges the step
-  // (and the wide-group finish, and the last step's finalize) apply to every row.
+  // reduction takes the layer's decision and hands it to the per-row keep-best code
+  // as thresholds (+inf: every row takes the step, -inf: none), which the launch that
+  // judges the step (and the wide-group finish, and the last step's finalize) read as
+  // best_in; their best_out goes to a scratch array.
   const bool layer_best = p->keep_best == AR_KEEP_BEST_LAYER && iters > 0;
   LayerBestArgs lb;
   lb.out = out;
   lb.inv_batch = 1.0f / static_cast<float>(B);
   lb.best = reinterpret_cast<double*>(ws + L.layer);
-  lb.flag = reinterpret_cast<int*>(ws + L.layer + 8);
-  lb.ticket = reinterpret_cast<unsigned int*>(ws + L.layer + 12);
+  lb.ticket = reinterpret_cast<unsigned int*>(ws + L.layer + 8);
   lb.blocksum = reinterpret_cast<double*>(ws + L.layer + 16);
   lb.best_rows = best_loss;
+  lb.thresh = F(L.layer_rows);
+  float* layer_scratch = F(L.layer_rows) + out;
   if (layer_best) {
     lb.init = 1;  // the best so far: best_loss[0] (+inf on a fresh state)
     AR_CUDA_TRY(launch_layer_best(lb, st));
@@ -758,7 +763,6 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   u.bits = p->bits;
   u.sym = p->sym != 0;
   u.keep_best = p->keep_best != 0;
-  u.layer_flag = layer_best ? lb.flag : nullptr;
   u.lr = p->lr;
   u.mlr = mlr;
   u.gpart = P.wide ? F(L.gpart) : nullptr;
@@ -793,7 +797,6 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
     f.beta_best = u.beta_best;
     f.judged = u.part_in != nullptr;
     f.keep_best = u.keep_best;
-    f.layer_flag = u.layer_flag;
     f.snap_prev = u.snap_prev;
     f.best_in = u.best_in;
     f.best_out = u.best_out;
@@ -857,8 +860,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       u.part_out = part[cur];
       u.part_in = t > 0 ? part[nxt] : nullptr;  // the previous step's partials
       u.rowloss = t > 0 ? rowloss + static_cast<int64_t>(t - 1) * out : nullptr;
-      u.best_in = best_cur;
-      u.best_out = best_next;
+      u.best_in = layer_best ? lb.thresh : best_cur;
+      u.best_out = layer_best ? layer_scratch : best_next;
       AR_CUDA_TRY(ensure_block(sched[t]));
       if (fpt) {
         u.Cc_hi = H(L.Cc_hi) + sched[t] * static_cast<int64_t>(elems);
@@ -884,9 +887,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       f.G = static_cast<int>(P.G);
       f.inv_batch = 1.0f / static_cast<float>(B);
       f.keep_best = p->keep_best != 0;
-      f.layer_flag = u.layer_flag;  // the last step's decision, taken after its launch
-      f.best_in = best_cur;
-      f.best_out = best_next;
+      f.best_in = layer_best ? lb.thresh : best_cur;  // the last step's decision, taken after its launch
+      f.best_out = layer_best ? layer_scratch : best_next;
       f.rowloss = rowloss + static_cast<int64_t>(iters - 1) * out;
       f.V_last = Vb[last];
       f.alpha_last = ab[last];
@@ -959,8 +961,8 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
       AR_CUDA_TRY(judge_layer(part[0], P.nparts_res));  // this step's loss, judged by its update
       AR_CUDA_TRY(make_tmap_bf16(&mu.b0, X + b0 * in, B, in, 64));
       mu.b1 = mu.b0;
-      u.best_in = best_cur;
-      u.best_out = best_next;
+      u.best_in = layer_best ? lb.thresh : best_cur;
+      u.best_out = layer_best ? layer_scratch : best_next;
       u.rowloss = rowloss + static_cast<int64_t>(t) * out;
       AR_CUDA_TRY(launch_gemm(upd_kind, P.bn_upd, mu, u, sms, st));
       AR_CUDA_TRY(finish_groups());

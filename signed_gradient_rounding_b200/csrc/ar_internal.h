@@ -74,31 +74,8 @@ struct FinalizeBestArgs {
   float* V_best = nullptr;
   float* alpha_best = nullptr;
   float* beta_best = nullptr;
-  const int* layer_flag = nullptr;  // layer-wide keep-best: the decision for every row
 };
 cudaError_t launch_finalize_best(const FinalizeBestArgs& a, cudaStream_t stream);
-
-// Layer-wide keep-best (keep_best = 2): after a step's row-loss partials are
-// complete, the layer's batch loss Lsum = sum over rows j of fp32(L_j) * inv_batch
-// (L_j the fp32 sum of part[j, 0 .. nparts) in index order, as the epilogues take it),
-// summed in fp64 in a fixed order (kLayerBlocks row ranges, each a fixed tree, then
-// the ranges in index order).  *flag = Lsum < *best; if so *best = Lsum and every
-// best_rows[j] = Lsum (the state's best_loss in this mode).  The launch that judges
-// the step reads *flag for every row.  init: set *best = best_rows[0], clear *flag.
-constexpr int kLayerBlocks = 32;
-struct LayerBestArgs {
-  const float* part = nullptr;
-  int nparts = 0;
-  int64_t out = 0;
-  float inv_batch = 1.f;
-  int init = 0;
-  double* best = nullptr;             // workspace
-  int* flag = nullptr;                // workspace
-  unsigned int* ticket = nullptr;     // workspace, 0 between launches
-  double* blocksum = nullptr;         // workspace [kLayerBlocks]
-  float* best_rows = nullptr;         // [out]
-};
-cudaError_t launch_layer_best(const LayerBestArgs& a, cudaStream_t stream);
 
 // Hs = sum over nb blocks of (H_hi[b] + H_lo[b]) in fp32, returned as a bf16 pair,
 // and dsum[k] = sum over blocks of diag[b*in + k] (the exact diagonals).
@@ -235,10 +212,6 @@ struct GemmArgs {
   const float* part_in = nullptr;  // [M, nparts] partials of the judged step (null: none)
   int nparts = 0;
   int snap_prev = 0;      // 0: judge this step (snapshot V_in); 1: judge the previous one (snapshot V_out)
-  // Layer-wide keep-best: every row takes the decision in *layer_flag (written by
-  // launch_layer_best from the judged step's partials) and best_in / best_out are
-  // not used.  Null: each row compares its own loss.
-  const int* layer_flag = nullptr;
   float* part_out = nullptr;  // [M, part_ld] this step's sum_k D G partials (Gram form), or null
   // Full-precision-target mode (Gram form): G += C (this block's W M_b, a bf16 pair
   // [M, N]); the row loss gains 2 sum_k D_jk C_jk, and e_row[j] once per row.
@@ -289,7 +262,6 @@ struct GroupFinishArgs {
   int judged = 0, keep_best = 1, snap_prev = 0;
   const float* best_in = nullptr;
   const float* best_out = nullptr;
-  const int* layer_flag = nullptr;  // as in GemmArgs
   __nv_bfloat16* D_hi = nullptr;
   __nv_bfloat16* D_lo = nullptr;
   const int* div_slow = nullptr;

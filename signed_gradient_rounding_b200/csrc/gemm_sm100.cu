@@ -440,8 +440,7 @@ __device__ __forceinline__ void load_upd_chunk(const GemmArgs& a, int64_t e0, in
 // the loss of this step (computed by the residual GEMM), snapshot of the state read
 // now.  Gram form: the loss of the previous step (computed by the previous
 // launch), snapshot of the previous state, which still sits in the output buffers
-// until this epilogue overwrites it.  Layer-wide keep-best: the decision already
-// taken for the whole layer (GemmArgs::layer_flag), the same on every row.
+// until this epilogue overwrites it.
 __device__ __forceinline__ bool row_better(const GemmArgs& a, int j, bool row_ok, int n_blk, int half) {
   bool better = false;
   if (row_ok && a.part_in) {
@@ -457,9 +456,7 @@ __device__ __forceinline__ bool row_better(const GemmArgs& a, int j, bool row_ok
       for (int i = 0; i < 8; ++i) L += x[i];
     }
     for (; q < a.nparts; ++q) L += p[q];
-    if (a.keep_best && a.layer_flag) {
-      better = *a.layer_flag != 0;  // one decision for the whole layer
-    } else if (a.keep_best) {
+    if (a.keep_best) {
       const float mean = L * a.inv_batch;
       better = mean < a.best_in[j];
       if (n_blk == 0 && half == 0) a.best_out[j] = better ? mean : a.best_in[j];

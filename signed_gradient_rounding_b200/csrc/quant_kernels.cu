@@ -5,6 +5,7 @@
 
 #include "ar_device.cuh"
 #include "ar_internal.h"
+#include "ar_layer_best.h"
 
 namespace ar {
 
@@ -276,9 +277,7 @@ __global__ void finalize_best_kernel(FinalizeBestArgs a) {
   const float* p = a.part + j * a.nparts;
   for (int q = 0; q < a.nparts; ++q) L += p[q];  // same order as the update epilogue
   bool better = false;
-  if (a.keep_best && a.layer_flag) {
-    better = *a.layer_flag != 0;
-  } else if (a.keep_best) {
+  if (a.keep_best) {
     const float mean = L * a.inv_batch;
     better = mean < a.best_in[j];
     if (lane == 0) a.best_out[j] = better ? mean : a.best_in[j];
@@ -314,8 +313,7 @@ __global__ void group_finish_kernel(GroupFinishArgs a) {
   const float al = a.alpha_in[grp], be = a.beta_in[grp];
   const float al_n = clip_step(al, a.mlr, dal);
   const float be_n = sym ? be : clip_step(be, a.mlr, dbe);
-  const bool better =
-      a.judged && a.keep_best && (a.layer_flag ? *a.layer_flag != 0 : a.best_out[j] < a.best_in[j]);
+  const bool better = a.judged && a.keep_best && a.best_out[j] < a.best_in[j];
   __syncwarp();  // every lane has read alpha_in, beta_in (they may alias the outputs)
   if (lane == 0 && in_bounds(grp, 1, a.chk_groups, a.status)) {
     if (better && !a.snap_prev) {
@@ -466,7 +464,6 @@ __global__ void layer_best_kernel(LayerBestArgs a) {
   if (a.init) {
     if (blockIdx.x == 0 && tid == 0) {
       *a.best = a.out > 0 ? static_cast<double>(a.best_rows[0]) : static_cast<double>(INFINITY);
-      *a.flag = 0;
       *a.ticket = 0u;
     }
     return;
@@ -499,15 +496,17 @@ __global__ void layer_best_kernel(LayerBestArgs a) {
     double total = 0.0;
     for (unsigned int b = 0; b < gridDim.x; ++b) total += __ldcg(a.blocksum + b);
     improved = total < *a.best;
-    *a.flag = improved;
     if (improved) *a.best = total;
     red[0] = total;
     *a.ticket = 0u;
   }
   __syncthreads();
-  if (!improved) return;
+  const float th = improved ? INFINITY : -INFINITY;
   const float v = static_cast<float>(red[0]);
-  for (int64_t j = tid; j < a.out; j += blockDim.x) a.best_rows[j] = v;
+  for (int64_t j = tid; j < a.out; j += blockDim.x) {
+    a.thresh[j] = th;
+    if (improved) a.best_rows[j] = v;
+  }
 }
 
 cudaError_t launch_layer_best(const LayerBestArgs& a, cudaStream_t stream) {
