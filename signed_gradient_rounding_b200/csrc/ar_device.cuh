@@ -369,6 +369,29 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// The same MMA with the A collector buffer: kFill reads A from shared memory and
+// keeps it in the tensor core's A collector; !kFill (lastuse) takes A from the
+// collector, filled by the MMA issued just before with the same A descriptor, and
+// releases it.  Two products that share their A tile read it from shared memory once.
+template <bool kFill>
+__device__ __forceinline__ void umma_bf16_pair_collect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                       uint32_t idesc, uint32_t accumulate) {
+  if (kFill)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::fill [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on the mbarrier at the same shared-memory offset in both CTAs of the pair
 // once the pair MMAs issued so far have completed.
 __device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {

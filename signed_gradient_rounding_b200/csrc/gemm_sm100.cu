@@ -16,9 +16,11 @@
 //               map the segments use, each staged once; completion counted on the
 //               stage's mbarrier.
 //   warp 1      MMA issuer: tcgen05.mma (M=128 or 256, N=BN, K=16), four per
-//               segment in the stage, into one of two BN-column fp32 accumulators
-//               in tensor memory; tcgen05.commit frees the stage and, after the
-//               last K block, hands the accumulator to the epilogue.
+//               segment in the stage (the Gram step's three pair products go per
+//               K16 step, the two that share D_hi through the A collector buffer),
+//               into one of two BN-column fp32 accumulators in tensor memory;
+//               tcgen05.commit frees the stage and, after the last K block, hands
+//               the accumulator to the epilogue.
 //   warps 2..9  epilogue: two warps per 32-lane slice of tensor memory (a warp may
 //               only read the slice warp % 4), one per column half of the tile.
 //               Each thread owns one accumulator row and walks its half's columns
@@ -836,6 +838,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     use_a1 = use_a1 || args.seg_a[s] != 0;
     use_b1 = use_b1 || args.seg_b[s] != 0;
   }
+  // The pair-precision product (D_hi + D_lo)(H_hi + H_lo) of the Gram step on fused
+  // stages: segments (A0, B0), (A1, B0), (A0, B1).  Per K16 step the MMA warp issues
+  // the two products of A0 back to back, the first filling the A collector buffer and
+  // the second reading it, so A0 leaves shared memory once per step (then A1's).
+  const bool collect = kPair && kFused && kNA == 2 && kNB == 2 && args.num_seg == 3 && args.seg_a[0] == 0 &&
+                       args.seg_b[0] == 0 && args.seg_a[1] == 1 && args.seg_b[1] == 0 && args.seg_a[2] == 0 &&
+                       args.seg_b[2] == 1;
   // With one map of an operand staged, it is whichever one the segments use.
   const CUtensorMap* map_a0 = (kNA == 1 && use_a1) ? &tmA1 : &tmA0;
   const CUtensorMap* map_b0 = (kNB == 1 && use_b1) ? &tmB1 : &tmB0;
@@ -950,7 +959,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          if (kFused) {
+          if (kFused && collect) {
+            const uint64_t a0 = operand_desc(a_addr, kAMn), a1 = operand_desc(a_addr + C::kOffA1, kAMn);
+            const uint64_t b0 = operand_desc(a_addr + C::kOffB0, kBMn);
+            const uint64_t b1 = operand_desc(a_addr + C::kOffB1, kBMn);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint32_t accum = ((kb - kb0) | k) != 0 ? 1u : 0u;
+              umma_bf16_pair_collect<true>(d_tmem, a0 + a_kstep * k, b0 + b_kstep * k, idesc_u, accum);
+              umma_bf16_pair_collect<false>(d_tmem, a0 + a_kstep * k, b1 + b_kstep * k, idesc_u, 1u);
+              umma_bf16_pair(d_tmem, a1 + a_kstep * k, b0 + b_kstep * k, idesc_u, 1u);
+            }
+          } else if (kFused) {
             for (int s = 0; s < args.num_seg; ++s) {
               const uint64_t a_desc =
                   operand_desc(a_addr + ((kNA == 2 && args.seg_a[s]) ? C::kOffA1 : 0), kAMn);
