@@ -16,8 +16,41 @@ __device__ __forceinline__ float load_w(const void* W, int w_bf16, int64_t idx) 
   return static_cast<const float*>(W)[idx];
 }
 
+// Two fp32 values that are already bf16 values (exactly representable), as a bf16x2 word.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// kVec consecutive weights as fp32 (kVec = 4: 8- or 16-byte aligned vector load).
+template <int kVec>
+__device__ __forceinline__ void load_wv(const void* W, int w_bf16, int64_t idx, float (&w)[kVec]) {
+  if (kVec == 4) {
+    if (w_bf16) {
+      const uint2 x = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(W) + idx);
+      w[0] = __uint_as_float(x.x << 16);
+      w[1] = __uint_as_float(x.x & 0xFFFF0000u);
+      w[2] = __uint_as_float(x.y << 16);
+      w[3] = __uint_as_float(x.y & 0xFFFF0000u);
+    } else {
+      const float4 x = *reinterpret_cast<const float4*>(static_cast<const float*>(W) + idx);
+      w[0] = x.x;
+      w[1] = x.y;
+      w[2] = x.z;
+      w[3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) w[i] = load_w(W, w_bf16, idx + i);
+  }
+}
+
 // One warp per group ("[llm-compressor] AutoRound ...", _fake_quantize_with_offset,
-// min-max init).  Group j*G + gi covers W[j, gi*g : (gi+1)*g].
+// min-max init).  Group j*G + gi covers W[j, gi*g : (gi+1)*g].  Each lane takes kVec
+// consecutive weights at a time (kVec = 4 when every pointer is 16-byte aligned and
+// in and g are multiples of 4, so the loads and stores are vectors; else 1).  The
+// per-element arithmetic is the same either way.
+template <int kVec>
 __global__ void group_quant_kernel(GroupQuantArgs a) {
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -30,11 +63,15 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
   // correctly rounded division by the group's scale (div_fast_ok).
   float mn = 0.0f, mx = 0.0f;  // min(0, min W), max(0, max W)
   bool ok = true;
-  for (int k = lane; k < a.g; k += 32) {
-    const float w = load_w(a.W, a.w_bf16, base + k);
-    mn = fminf(mn, w);
-    mx = fmaxf(mx, w);
-    ok = ok && div_fast_ok(w);
+  for (int k = lane * kVec; k < a.g; k += 32 * kVec) {
+    float w[kVec];
+    load_wv<kVec>(a.W, a.w_bf16, base + k, w);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      mn = fminf(mn, w[i]);
+      mx = fmaxf(mx, w[i]);
+      ok = ok && div_fast_ok(w[i]);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -61,18 +98,57 @@ __global__ void group_quant_kernel(GroupQuantArgs a) {
   }
   if (!a.codes && !a.Wq && !a.D_hi) return;
   const float Q = qmaxf(a.bits);
-  for (int k = lane; k < a.g; k += 32) {
-    const float w = load_w(a.W, a.w_bf16, base + k);
-    const float v = a.V ? a.V[base + k] : 0.0f;
-    const ElemQuant e = quant_elem(w, v, gs, Q, fast);
-    if (!in_bounds(base + k, 1, a.chk_elems, a.status)) continue;
-    if (a.codes) a.codes[base + k] = static_cast<uint8_t>(e.q);
-    if (a.Wq) a.Wq[base + k] = e.wq;
-    if (a.D_hi) {
-      const float d = __fsub_rn(e.wq, w);
+  for (int k = lane * kVec; k < a.g; k += 32 * kVec) {
+    const int64_t e0 = base + k;
+    float w[kVec], v[kVec];
+    load_wv<kVec>(a.W, a.w_bf16, e0, w);
+    if (!a.V) {
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) v[i] = 0.0f;
+    } else if (kVec == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(a.V + e0);
+      v[0] = x.x;
+      v[1] = x.y;
+      v[2] = x.z;
+      v[3] = x.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) v[i] = a.V[e0 + i];
+    }
+    float q[kVec], wq[kVec], dh[kVec], dl[kVec];
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const ElemQuant e = quant_elem(w[i], v[i], gs, Q, fast);
+      q[i] = e.q;
+      wq[i] = e.wq;
+      const float d = __fsub_rn(e.wq, w[i]);
       const __nv_bfloat16 hi = __float2bfloat16_rn(d);
-      a.D_hi[base + k] = hi;
-      if (a.D_lo) a.D_lo[base + k] = __float2bfloat16_rn(__fsub_rn(d, __bfloat162float(hi)));
+      dh[i] = __bfloat162float(hi);
+      dl[i] = __fsub_rn(d, dh[i]);
+    }
+    if (!in_bounds(e0, kVec, a.chk_elems, a.status)) continue;
+    if (kVec == 4) {
+      if (a.codes)
+        *reinterpret_cast<uint32_t*>(a.codes + e0) =
+            static_cast<uint32_t>(q[0]) | (static_cast<uint32_t>(q[1]) << 8) |
+            (static_cast<uint32_t>(q[2]) << 16) | (static_cast<uint32_t>(q[3]) << 24);
+      if (a.Wq) *reinterpret_cast<float4*>(a.Wq + e0) = make_float4(wq[0], wq[1], wq[2], wq[3]);
+      if (a.D_hi) {
+        *reinterpret_cast<uint2*>(a.D_hi + e0) = make_uint2(pack_bf16x2_rn(dh[0], dh[1]), pack_bf16x2_rn(dh[2], dh[3]));
+        if (a.D_lo)
+          *reinterpret_cast<uint2*>(a.D_lo + e0) =
+              make_uint2(pack_bf16x2_rn(dl[0], dl[1]), pack_bf16x2_rn(dl[2], dl[3]));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) {
+        if (a.codes) a.codes[e0 + i] = static_cast<uint8_t>(q[i]);
+        if (a.Wq) a.Wq[e0 + i] = wq[i];
+        if (a.D_hi) {
+          a.D_hi[e0 + i] = __float2bfloat16_rn(dh[i]);
+          if (a.D_lo) a.D_lo[e0 + i] = __float2bfloat16_rn(dl[i]);
+        }
+      }
     }
   }
 }
@@ -99,6 +175,37 @@ __global__ void pack_kernel(const uint8_t* __restrict__ codes, int64_t rows, int
       word |= c >> (-shift);
     }
   }
+  packed[idx] = word;
+}
+
+// The same for bits 2, 4 and 8 (32 / bits codes per word, whole words per row):
+// one vector load of the word's codes (4, 8 or 16 bytes, aligned when the codes
+// are) instead of one byte load per code.
+template <int kBits>
+__global__ void pack_pow2_kernel(const uint8_t* __restrict__ codes, int64_t total_words,
+                                 uint32_t* __restrict__ packed) {
+  constexpr int kPer = 32 / kBits;  // codes per word; rows hold whole words
+  constexpr uint32_t kMask = (1u << kBits) - 1u;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total_words) return;
+  const uint8_t* src = codes + idx * kPer;
+  uint32_t b[kPer / 4];
+  if constexpr (kPer == 4) {
+    b[0] = *reinterpret_cast<const uint32_t*>(src);
+  } else if constexpr (kPer == 8) {
+    const uint2 x = *reinterpret_cast<const uint2*>(src);
+    b[0] = x.x;
+    b[1] = x.y;
+  } else {
+    const uint4 x = *reinterpret_cast<const uint4*>(src);
+    b[0] = x.x;
+    b[1] = x.y;
+    b[2] = x.z;
+    b[3] = x.w;
+  }
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) word |= ((b[i / 4] >> (8 * (i % 4))) & kMask) << (kBits * i);
   packed[idx] = word;
 }
 
@@ -536,7 +643,13 @@ cudaError_t launch_group_quant(const GroupQuantArgs& a, cudaStream_t stream) {
   if (groups == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (groups * 32 + threads - 1) / threads;
-  group_quant_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  const bool vec = a.in % 4 == 0 && a.g % 4 == 0 && al16(a.W) && al16(a.V) && al16(a.codes) && al16(a.Wq) &&
+                   al16(a.D_hi) && al16(a.D_lo);
+  if (vec)
+    group_quant_kernel<4><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
+  else
+    group_quant_kernel<1><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -546,8 +659,18 @@ cudaError_t launch_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bi
   const int64_t total = rows * wpr;
   if (total == 0) return cudaSuccess;
   const int threads = 256;
-  pack_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, stream>>>(
-      codes, rows, cols, bits, wpr, reinterpret_cast<uint32_t*>(packed));
+  const unsigned blocks = static_cast<unsigned>((total + threads - 1) / threads);
+  uint32_t* out = reinterpret_cast<uint32_t*>(packed);
+  // Rows hold whole words, so word idx covers codes [idx * 32/bits, ...) of the flat array.
+  const bool aligned = (reinterpret_cast<uintptr_t>(codes) & 15u) == 0;
+  if (aligned && bits == 8)
+    pack_pow2_kernel<8><<<blocks, threads, 0, stream>>>(codes, total, out);
+  else if (aligned && bits == 4)
+    pack_pow2_kernel<4><<<blocks, threads, 0, stream>>>(codes, total, out);
+  else if (aligned && bits == 2)
+    pack_pow2_kernel<2><<<blocks, threads, 0, stream>>>(codes, total, out);
+  else
+    pack_kernel<<<blocks, threads, 0, stream>>>(codes, rows, cols, bits, wpr, out);
   return cudaGetLastError();
 }
 

@@ -121,6 +121,29 @@ def test_pack_bitexact(ar, bits, shape):
         assert np.array_equal(oracle.unpack_codes(_np(packed), bits, cols), codes)
 
 
+def test_unaligned_buffers_take_the_scalar_paths(ar):
+    """RTN and pack load and store vectors when their buffers are 16-byte aligned, and one
+    element or code at a time otherwise: both give the oracle's results."""
+    out, inn, g = 9, 96, 32
+    W = make_weight(out, inn, 0.02, "f32", seed=5)
+    flat = torch.empty(out * inn + 1, dtype=torch.float32, device="cuda")
+    flat[1:] = torch.from_numpy(W).reshape(-1).cuda()
+    Wd = flat[1:].view(out, inn)
+    assert Wd.data_ptr() % 16 != 0
+    codes, scale, zp = ar.rtn(Wd, 4, g, False)
+    torch.cuda.synchronize()
+    c, sc, z, _ = oracle.rtn(W, 4, g, False)
+    assert np.array_equal(_np(codes), c) and np.array_equal(_np(scale), sc) and np.array_equal(_np(zp), z)
+    for bits in (2, 4, 8):
+        rows, cols = 5, 64
+        cd = np.random.default_rng(bits).integers(0, 2 ** bits, size=(rows, cols), dtype=np.uint8)
+        buf = torch.empty(rows * cols + 1, dtype=torch.uint8, device="cuda")
+        buf[1:] = torch.from_numpy(cd).reshape(-1).cuda()
+        packed = ar.pack(buf[1:].view(rows, cols), bits)
+        torch.cuda.synchronize()
+        assert np.array_equal(_np(packed), oracle.pack_codes(cd, bits)), bits
+
+
 def test_timeout_path_reports_and_recovers(ar):
     """A bounded wait that nothing satisfies gives up, reports AR_ETIMEOUT and the
     context stays usable."""
