@@ -313,6 +313,8 @@ def run_ours(args):
     # lets the multi-rank path run where ranks share a GPU, as a test of the code path:
     # its times then mean nothing.
     backend = os.environ.get("AR_BENCH_BACKEND", "nccl")
+    if backend not in ("nccl", "gloo"):
+        raise SystemExit(f"AR_BENCH_BACKEND must be nccl or gloo, not {backend!r}")
     local = local % torch.cuda.device_count() if backend == "gloo" else local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
