@@ -11,7 +11,9 @@ picks one step, and every row takes that step's state.  Checked here:
   two lowest layer losses are not within 1e-6 of each other, at most 0.5% of the
   codes differing and the final MSE within 2%;
 - resume at a step in the middle equals one run, bit for bit;
-- the full-size q_proj layer (Gram form) makes the same host-checked choice.
+- the full-size q_proj layer (Gram form) makes the same host-checked choice;
+- the quant-aware mode with a full-precision target meets the bars in both forms, and
+  the host-buffer entry point gives the device entry point's results.
 """
 import numpy as np
 import pytest
@@ -144,3 +146,36 @@ def test_layer_best_q_proj_full_size(ar):
     print(f"\nq_proj layer-wide keep-best: step {k}, final MSE {mse_layer:.6g}; "
           f"per-row keep-best final MSE {float(row.final_mse.item()):.6g}")
     assert np.isfinite(mse_layer) and 0 <= k < c.iters
+
+
+@pytest.mark.parametrize("algo", ["gram", "direct"])
+def test_layer_best_with_full_precision_target(ar, algo):
+    """The layer-wide choice in the quant-aware mode, both forms: the codes and the final MSE
+    within the bars against the oracle over every row."""
+    from workloads import make_quantised_path_input
+    out, inn, n, B, iters = 200, 384, 2048, 512, 24
+    W = make_weight(out, inn, 0.02, "bf16", seed=29)
+    Xf = make_activations(n, inn, "llm", seed=29)
+    Xq = make_quantised_path_input(Xf, 0.05, seed=29)
+    p = ar.make_params(bits=3, group_size=128, iters=iters, batch_rows=B, seed=2, keep_best="layer", algo=algo)
+    Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
+    res = ar.tune_layer_fp_target(Wd, torch.from_numpy(Xq).to(torch.bfloat16).cuda(),
+                                  torch.from_numpy(Xf).to(torch.bfloat16).cuda(), p)
+    assert ar.tune_status(res.workspace) == ar.AR_OK
+    ref = oracle.tune_layer(W, Xq, 3, 128, False, iters, 0.005, -1.0, B, 2, keep_best=2, X_target=Xf)
+    frac = float(np.mean(res.codes.cpu().numpy() != ref.codes))
+    assert frac <= CODE_TOL, f"{frac:.4%} of codes differ"
+    assert float(res.final_mse.item()) == pytest.approx(ref.final_mse, rel=MSE_RTOL)
+
+
+def test_layer_best_host_entry_equals_device_entry(ar):
+    """ar_tune_layer_host (host buffers, blockwise copies) makes the same layer-wide choice."""
+    c = CASES["multiblock_bf16"]
+    W, X = _inputs(c, seed=31)
+    Wd, Xd = _dev(W, X, c["wdt"])
+    p = _params(ar, c, "layer", algo="gram")
+    dev_res = ar.tune_layer(Wd, Xd, p)
+    host = ar.tune_layer_host(Wd.cpu(), Xd.cpu(), p)
+    torch.cuda.synchronize()
+    assert torch.equal(host["codes"], dev_res.codes.cpu())
+    assert torch.equal(host["scale"], dev_res.scale.cpu()) and torch.equal(host["zero_point"], dev_res.zero_point.cpu())
