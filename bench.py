@@ -201,7 +201,7 @@ def run_block(args):
     x0 = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
     p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
                        minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
-                       split=bool(args.split))
+                       split=int(args.split))
     ws = torch.empty(block_workspace_bytes(weights, c.n_rows, p), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -345,7 +345,7 @@ def run_ours(args):
     Xd = make_activations_cuda(c.n_rows, c.inn, c.x_kind, seed=0, device=dev)
     p = ar.make_params(bits=c.bits, group_size=c.group_size, sym=c.sym, iters=c.iters, lr=c.lr,
                        minmax_lr=c.minmax_lr, batch_rows=c.batch_rows, seed=0, algo=args.algo,
-                       split=bool(args.split))
+                       split=int(args.split))
     rows = b - a
     ws = torch.empty(ar.tune_workspace_bytes(rows, c.inn, c.n_rows, p), dtype=torch.uint8, device=dev)
     G = c.inn // (c.inn if c.group_size == -1 else c.group_size)
@@ -476,6 +476,7 @@ def run_ours(args):
         "layer_tune_s": layer_s,
         "algo": algo,
         "split_operands": bool(args.split),
+        "chunked_accumulation": args.split == 2,
         "step_ms": step_ms,
         "setup_ms": sum(t.setup_ms for t in timings) / len(timings),
         "executed_tflop_per_step": (flops_res + flops_upd) / 1e12,
@@ -610,7 +611,8 @@ def main():
     ap.add_argument("--cpu-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--algo", choices=["auto", "direct", "gram"], default="auto")
-    ap.add_argument("--split", type=int, default=1, help="1: bf16-pair operands (default); 0: single bf16")
+    ap.add_argument("--split", type=int, default=1, choices=[0, 1, 2],
+                    help="1: bf16-pair operands (default); 0: single bf16; 2: pairs and chunked K accumulation")
     ap.add_argument("--group-size", type=int, default=None,
                     help="override the workload's group size (-1: one group per row)")
     ap.add_argument("--mode", choices=["layer", "fp_target"], default="layer",

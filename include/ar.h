@@ -113,7 +113,12 @@ typedef struct {
   int32_t split;         /* 1: tensor-core operands as exact bf16 pairs hi + lo
                             (hi = bf16(x), lo = bf16(x - hi): ~16 significant bits);
                             0: single bf16 (faster, the tuning trajectory drifts
-                            further from an exact evaluation) */
+                            further from an exact evaluation); 2: pairs, and the
+                            Gram step sums K in chunks of 512 (each a fresh
+                            tensor-core accumulation, added in fp32 round to
+                            nearest): closer to an exact evaluation, slower; Gram
+                            form with groups of at most 256 columns that divide
+                            256, no full-precision target (else AR_EUNSUPPORTED) */
   int32_t init;          /* ar_init: how alpha and beta start (0: min-max) */
 } ar_tune_params;
 

@@ -169,6 +169,7 @@ ar_status check_tune_args(int64_t out, int64_t in, int64_t n_rows, const ar_tune
   if (p->algo < AR_ALGO_AUTO || p->algo > AR_ALGO_GRAM) return AR_EINVAL;
   if (p->init != AR_INIT_MINMAX && p->init != AR_INIT_MSE) return AR_EINVAL;
   if (p->keep_best < AR_KEEP_LAST || p->keep_best > AR_KEEP_BEST_LAYER) return AR_EINVAL;
+  if (p->split < 0 || p->split > 2) return AR_EINVAL;
   if (out == 0 || in == 0) return AR_OK;
   if (!group_ok(in, p->group_size)) return AR_EINVAL;
   if (p->batch_rows <= 0 || n_rows < p->batch_rows || n_rows % p->batch_rows != 0) return AR_EINVAL;
@@ -193,6 +194,9 @@ constexpr size_t kFpTargetMaxBytes = 64ull << 30;
 struct Plan {
   int algo = AR_ALGO_DIRECT;
   int split = 1;
+  // split = 2: the Gram step sums K in chunks of exact_chunk K blocks (kEpiUpdateExact).
+  bool exact = false;
+  int exact_chunk = 8;
   int64_t out = 0, in = 0, n = 0, B = 0, g = 0, G = 0, nb = 0, iters = 0;
   int bn_res = 256;   // direct: residual GEMM (N = B)
   int bn_upd = 256;   // update GEMM (N = in)
@@ -243,6 +247,7 @@ Plan make_plan(int64_t out, int64_t in, int64_t n, const ar_tune_params* p, bool
   P.fp_target = fp_target;
   P.w_f32 = w_f32;
   P.split = p->split != 0;
+  P.exact = p->split == 2;
   P.out = out;
   P.in = in;
   P.n = n;
@@ -438,6 +443,9 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   const Plan P = make_plan(out, in, n_rows, p, X_target != nullptr, w_dtype == AR_F32);
   const Layout L = make_layout(P);
   if (P.fp_target && P.algo == AR_ALGO_GRAM && L.total > kFpTargetMaxBytes) return AR_EUNSUPPORTED;
+  // The chunked accumulation exists for the plain Gram step with groups inside a thread's
+  // columns.
+  if (P.exact && (P.algo != AR_ALGO_GRAM || P.wide || P.fp_target)) return AR_EUNSUPPORTED;
   const Fault fault = injected_fault();
   if (ws_bytes < L.total || fault == kFaultAlloc) return AR_ENOMEM;
   const bool gram = P.algo == AR_ALGO_GRAM;
@@ -815,8 +823,10 @@ ar_status tune_impl(const void* W, ar_dtype w_dtype, int64_t out, int64_t in, co
   // The Gram form's full-precision-target terms enter the step's epilogue; the direct
   // form's are already in R (E_b^T, added by the residual's epilogue).
   const bool fpt_step = fpt && gram;
-  const EpiKind upd_kind =
-      fpt_step ? (P.wide ? kEpiUpdateFpWide : kEpiUpdateFp) : (P.wide ? kEpiUpdateWide : kEpiUpdate);
+  const EpiKind upd_kind = P.exact ? kEpiUpdateExact
+                           : fpt_step ? (P.wide ? kEpiUpdateFpWide : kEpiUpdateFp)
+                                      : (P.wide ? kEpiUpdateWide : kEpiUpdate);
+  if (P.exact) u.k_chunk = P.exact_chunk;
 
   float* best_cur = best_loss;
   float* best_next = best_alt;

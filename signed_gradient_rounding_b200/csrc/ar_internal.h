@@ -114,7 +114,11 @@ enum EpiKind : int {
   // 128-column segment) partials of d alpha, d beta into GemmArgs::gpart; the
   // group's update and the next D follow in launch_group_finish.
   kEpiUpdateWide = 5,
-  kEpiUpdateFpWide = 6
+  kEpiUpdateFpWide = 6,
+  // kEpiUpdate on K summed in chunks of GemmArgs::k_chunk K blocks: each chunk a fresh
+  // tensor-core accumulation, added in fp32 (round to nearest) to the tile's running
+  // sum by the epilogue before the step runs on the sum (ar_tune_params.split = 2).
+  kEpiUpdateExact = 7
 };
 
 // Columns per thread in the update epilogue (one column half of a 256-wide tile):

@@ -769,7 +769,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The Gram-matrix instance can sum K in chunks (GemmArgs::k_chunk): the MMAs of
   // each chunk accumulate afresh in accumulator 1, and the epilogue adds each chunk,
   // in fp32 round to nearest, to the tile's running sum kept in accumulator 0.
-  constexpr bool kChunkable = kKind == kEpiStore && kPair && kNA == 0 && kNB == 0 && kMaj == 3;
+  constexpr bool kChunkable = (kKind == kEpiStore && kPair && kNA == 0 && kNB == 0 && kMaj == 3) ||
+                              (kKind == kEpiUpdateExact && kPair && kNA == 2 && kNB == 2 && kMaj == 0);
   // The step instances on pair tiles may split the tiles of their last partial wave
   // into column halves (GemmArgs::split_tiles): a half unit issues N = kBN / 2 MMAs
   // into the half's own columns of the accumulator, and only that half's epilogue
@@ -830,8 +831,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (segment, K block), segments outermost.
   const int k_blocks = kFused ? args.num_k_blk : args.num_seg * args.num_k_blk;
   // K blocks per accumulator hand-off: the whole tile, or one chunk.
-  const bool chunked = kChunkable && args.k_chunk > 0 && args.k_chunk < k_blocks;
-  const int k_chunk = chunked ? args.k_chunk : k_blocks;
+  // (kEpiUpdateExact always takes the chunked path, with one chunk when K is short.)
+  const bool chunk_arg = args.k_chunk > 0 && args.k_chunk < k_blocks;
+  const bool chunked = kChunkable && (kKind == kEpiUpdateExact || chunk_arg);
+  const int k_chunk = chunked && chunk_arg ? args.k_chunk : k_blocks;
   // kFused: which of the two maps of A and of B the segments use.
   bool use_a1 = false, use_b1 = false;
   for (int s = 0; s < args.num_seg; ++s) {
@@ -1047,7 +1050,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_pos<kBN, kPair>(args, tile, m_blk, n_blk);
       const int j = (kPair ? 2 * m_blk + static_cast<int>(rank) : m_blk) * kBM + row_in_tile;
       const int n0 = n_blk * kBN;
-      if ((kKind == kEpiUpdate || kKind == kEpiUpdateFp) && active) epi_update_prefetch<kBN, false>(args, j, n0, half);
+      if ((kKind == kEpiUpdate || kKind == kEpiUpdateFp || kKind == kEpiUpdateExact) && active)
+        epi_update_prefetch<kBN, false>(args, j, n0, half);
       if (kWideKind && active) epi_update_prefetch<kBN, true>(args, j, n0, half);
       if constexpr (kChunkable) {
         if (chunked) {
@@ -1086,21 +1090,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             chunk_phase ^= 1;
           }
           if (!ok) break;
-          // the tile's sum, from accumulator 0
+          if constexpr (kKind == kEpiUpdateExact) {
+            // the step on the tile's sum in accumulator 0, which no MMA writes
+            tc_fence_after();
+            epi_update<kBN, false>(args, tmem_base + lanes, j, n0, n_blk, half);
+            continue;
+          } else {
+            // the tile's sum, from accumulator 0
 #pragma unroll 1
-          for (int g = 0; g < kBN / kEpiHalves / 32; ++g) {
-            uint32_t r[32];
-            __syncwarp();
-            tmem_ld_32cols(t_sum + g * 32, r);
-            tmem_ld_wait();
-            const int col0 = n0 + half * (kBN / kEpiHalves) + g * 32;
-            if (j >= args.M || col0 >= args.N) continue;  // nothing warp-collective follows
-            float x[32];
+            for (int g = 0; g < kBN / kEpiHalves / 32; ++g) {
+              uint32_t r[32];
+              __syncwarp();
+              tmem_ld_32cols(t_sum + g * 32, r);
+              tmem_ld_wait();
+              const int col0 = n0 + half * (kBN / kEpiHalves) + g * 32;
+              if (j >= args.M || col0 >= args.N) continue;  // nothing warp-collective follows
+              float x[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
-            store_cols32(args, j, col0, min(32, args.N - col0), x);
+              for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+              store_cols32(args, j, col0, min(32, args.N - col0), x);
+            }
+            continue;
           }
-          continue;
         }
       }
       // No early exit on another role's abort: every epilogue warp of the CTA takes
@@ -1109,7 +1120,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       if (active) {
-        if constexpr (kKind == kEpiUpdate)
+        if constexpr (kKind == kEpiUpdateExact) {
+          // always chunked (above)
+        } else if constexpr (kKind == kEpiUpdate)
           epi_update<kBN, false>(args, t_row, j, n0, n_blk, half);
         else if constexpr (kKind == kEpiUpdateFp)
           epi_update<kBN, true>(args, t_row, j, n0, n_blk, half);
@@ -1153,7 +1166,8 @@ template <int kKind, int kBN, bool kPair, int kNA, int kNB>
 constexpr bool stage_instance() {
   if (kNA == 0) return kNB == 0;
   if (kPair && kNA == 2 && kNB == 2)
-    return kKind == kEpiUpdate || kKind == kEpiUpdateFp || kKind == kEpiStore || kKind == kEpiSumSq;
+    return kKind == kEpiUpdate || kKind == kEpiUpdateFp || kKind == kEpiStore || kKind == kEpiSumSq ||
+           kKind == kEpiUpdateExact;
   if (kPair && kNA == 1 && kNB == 2) return kKind == kEpiStore || kKind == kEpiSumSq;
   if (kPair && kNA == 2 && kNB == 1) return kKind == kEpiStore || kKind == kEpiUpdate;
   if (!kPair && kBN == 256 && kNA == 2 && kNB == 1)
@@ -1165,6 +1179,8 @@ constexpr bool stage_instance() {
 // and the full-precision-target M_b (kEpiStore), B for the direct update.
 template <int kKind, int kBN, bool kPair, int kNA, int kNB, int kMaj>
 constexpr bool kernel_instance() {
+  // The chunked-accumulation step: the Gram step's pair tiles and fused 2 + 2 stages only.
+  if (kKind == kEpiUpdateExact) return kPair && kBN == 256 && kNA == 2 && kNB == 2 && kMaj == 0;
   // Wide-group steps: the Gram step on pair tiles (pair or single operands, with or
   // without a full-precision target) and the direct update on 1-SM tiles.
   if (kKind == kEpiUpdateWide || kKind == kEpiUpdateFpWide) {
@@ -1258,6 +1274,8 @@ cudaError_t launch_bn(EpiKind kind, const GemmMaps& m, const GemmArgs& args, int
       return launch_kind<kEpiUpdateWide, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
     case kEpiUpdateFpWide:
       return launch_kind<kEpiUpdateFpWide, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
+    case kEpiUpdateExact:
+      return launch_kind<kEpiUpdateExact, kBN, kPair, kNA, kNB, kMaj>(m, args, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

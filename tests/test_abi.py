@@ -75,6 +75,10 @@ def test_tune_validation(ar):
     assert call(64, 256, 1024, batch_rows=512, group_size=64, init=2) == ar.AR_EINVAL  # unknown init
     assert call(64, 256, 1024, batch_rows=512, group_size=64, keep_best=3) == ar.AR_EINVAL  # unknown keep-best
     assert call(64, 256, 1024, batch_rows=512, group_size=64, keep_best=-1) == ar.AR_EINVAL
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, split=3) == ar.AR_EINVAL
+    # the chunked accumulation (split = 2): the plain Gram step with narrow groups only
+    assert call(64, 256, 1024, batch_rows=512, group_size=64, split=2, algo="direct") == ar.AR_EUNSUPPORTED
+    assert call(64, 1024, 1024, batch_rows=512, group_size=512, split=2, algo="gram") == ar.AR_EUNSUPPORTED
     assert ar.make_params(keep_best="layer").keep_best == ar.AR_KEEP_BEST_LAYER
     assert ar.make_params(keep_best=True).keep_best == ar.AR_KEEP_BEST_ROW
     assert ar.make_params(keep_best="last").keep_best == ar.AR_KEEP_LAST
